@@ -1,0 +1,434 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties one oracle step to a hand-worked example (tests/golden/), a
+published generator, a library routine (scikit-learn's Lloyd, torch SDPA), a
+closed form or an invariant of the method on the AdaCluster pages
+(arXiv 2604.18348) and the ClusterAttention error split.
+"""
+import ctypes
+import json
+import os
+
+import numpy as np
+import pytest
+
+from conftest import GOLDEN
+from oracle import oracle as orc
+from cluster_routed_sparse_b200 import synth
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def bf(x):
+    return synth.f32_to_bf16_bits(np.asarray(x, np.float32))
+
+
+# ----------------------------------------------------------------- generator
+
+def test_splitmix64_published_vectors():
+    g = _golden("splitmix64_vectors.json")
+    lib = orc.lib()
+    lib.or_splitmix64.restype = ctypes.c_uint64
+    lib.or_splitmix64.argtypes = [ctypes.c_uint64, ctypes.c_int64]
+    got0 = ["%016x" % lib.or_splitmix64(0, i) for i in range(3)]
+    assert got0 == g["state_0_hex"]
+    got1 = [lib.or_splitmix64(1234567, i) for i in range(5)]
+    assert got1 == g["state_1234567"]
+
+
+@pytest.mark.parametrize("n,m", [(1, 1), (7, 7), (10, 3), (4096, 16), (75600, 256), (5, 2)])
+def test_seed_pick_strata(n, m):
+    pos = orc.seed_pick(99, 3, 5, n, m)
+    assert len(set(pos.tolist())) == m
+    for j, p in enumerate(pos):
+        assert (j * n) // m <= p < ((j + 1) * n) // m
+    if m == n:
+        assert (pos == np.arange(n)).all()
+
+
+# ----------------------------------------------------------------- Sec. 3.1
+
+def test_qnorm_against_fp64_norm():
+    rng = np.random.default_rng(0)
+    q = bf(rng.standard_normal((257, 64)) * rng.lognormal(0, 1, (257, 1)))
+    q[5] = 0
+    inv, xh = orc.qnorm(q)
+    qf = synth.bf16_bits_to_f32(q).astype(np.float64)
+    n = np.linalg.norm(qf, axis=1)
+    ok = n > 0
+    assert np.allclose(inv[ok] * n[ok], 1.0, rtol=0, atol=3e-7)
+    assert inv[5] == 0 and (xh[5] == 0).all()
+    assert np.allclose(np.linalg.norm(xh[ok].astype(np.float64), axis=1), 1.0, atol=1e-6)
+
+
+def test_angular_clustering_scale_invariance():
+    """Check (e): rescaling a query by a positive factor leaves its direction,
+    hence the angular clustering, unchanged (App. A.2).  Powers of two scale
+    bf16 exactly, so labels and centres must be bit-identical."""
+    cfg = synth.CONFIGS[1]
+    Q, _, _ = synth.make_layer(cfg, heads=[0])
+    p = orc.Params.from_layer_config(cfg)
+    lab0, C0, _ = orc.cluster_q(Q[0], p)
+    rng = np.random.default_rng(1)
+    e = rng.integers(-3, 4, size=(cfg.L, 1)).astype(np.float32)
+    Qs = bf(synth.bf16_bits_to_f32(Q[0, 0]) * np.exp2(e))[None]
+    lab1, C1, _ = orc.cluster_q(Qs, p)
+    assert (lab0 == lab1).all()
+    assert np.array_equal(C0, C1)
+
+
+def test_angular_clustering_arbitrary_scale_near_invariant():
+    """Check (e) with arbitrary factors in [0.1, 10]: the bf16 rounding of the
+    rescaled query moves its direction by about 2^-9, so one assignment to the
+    same centres agrees except on rows whose best/second gap is that small."""
+    cfg = synth.CONFIGS[1]
+    Q, _, _ = synth.make_layer(cfg, heads=[1])
+    p = orc.Params.from_layer_config(cfg)
+    _, C0, _ = orc.cluster_q(Q[0], p)
+    rng = np.random.default_rng(2)
+    s = rng.uniform(0.1, 10, size=(cfg.L, 1)).astype(np.float32)
+    Qs = bf(synth.bf16_bits_to_f32(Q[0, 0]) * s)
+    x0 = orc.qnorm(Q[0, 0])[1]
+    x1 = orc.qnorm(Qs)[1]
+    lab0, _ = orc.assign(x0, C0[0])
+    lab1, _ = orc.assign(x1, C0[0])
+    D = ((x0[:, None, :].astype(np.float64) - C0[0][None].astype(np.float64)) ** 2).sum(-1)
+    srt = np.sort(D, axis=1)
+    near = (srt[:, 1] - srt[:, 0]) < 2e-2
+    assert (lab0[~near] == lab1[~near]).all()
+    assert (lab0 != lab1).mean() < 0.01
+
+
+# ----------------------------------------------------------------- k-means
+
+def test_assign_bruteforce_fp64():
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((500, 16)).astype(np.float32)
+    C = rng.standard_normal((37, 16)).astype(np.float32)
+    C[9] = C[4]  # exact duplicate: ties go to the lower id
+    lab, dm = orc.assign(X, C)
+    D = ((X[:, None, :].astype(np.float64) - C[None].astype(np.float64)) ** 2).sum(-1)
+    srt = np.sort(D, axis=1)
+    clear = (srt[:, 1] - srt[:, 0]) > 1e-5 * srt[:, 0]
+    assert (lab[clear] == D[clear].argmin(1)).all()
+    assert np.allclose(dm, D[np.arange(500), lab], rtol=1e-5)
+    assert not (lab == 9).any()
+
+
+def test_update_is_member_mean_and_keeps_empty():
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((300, 8)).astype(np.float32)
+    lab = rng.integers(0, 5, 300).astype(np.int32)
+    lab[lab == 3] = 2  # cluster 3 empty
+    C0 = rng.standard_normal((5, 8)).astype(np.float32)
+    C, cnt = orc.update(X, lab, C0)
+    for c in range(5):
+        if c == 3:
+            assert cnt[c] == 0 and np.array_equal(C[c], C0[c])
+        else:
+            m = X[lab == c].astype(np.float64).mean(0)
+            assert cnt[c] == (lab == c).sum()
+            assert np.allclose(C[c], m, rtol=1e-5, atol=1e-6)
+
+
+def test_kmeans_matches_sklearn_lloyd():
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(5)
+    centres = rng.standard_normal((6, 5)) * 10
+    X = (centres[rng.integers(0, 6, 600)] + rng.standard_normal((600, 5))).astype(np.float32)
+    init = X[orc.seed_pick(7, 0, 0, 600, 6)]
+    lab, dm, C = orc.kmeans(X, init, 8)
+    km = KMeans(n_clusters=6, init=init.astype(np.float64), n_init=1, max_iter=8, tol=0.0,
+                algorithm="lloyd").fit(X.astype(np.float64))
+    assert (km.labels_ == lab).all()
+    assert np.allclose(km.cluster_centers_, C, rtol=1e-5, atol=1e-5)
+
+
+def test_lloyd_objective_monotone():
+    """Check (b): J never increases across an assignment or an update."""
+    cfg = synth.CONFIGS[1]
+    Q, K, _ = synth.make_layer(cfg, heads=[0])
+    for X in (synth.bf16_bits_to_f32(K[0, 0]), orc.qnorm(Q[0, 0])[1]):
+        init = X[orc.seed_pick(11, 0, 0, X.shape[0], 24)]
+        _, _, _, jt = orc.kmeans(X, init, 10, trace=True)
+        assert (np.diff(jt) <= 1e-6 * jt[:-1]).all(), jt
+
+
+def test_planted_partition_recovery():
+    """Well-separated mixture (Sec. 3.2.2: stages continue until every token
+    sits in a compact cluster): every multi-stage key cluster is pure."""
+    rng = np.random.default_rng(6)
+    L, d, nc = 2048, 16, 12
+    mu = rng.standard_normal((nc, d)) * 8
+    comp = rng.integers(0, nc, L)
+    Kf = mu[comp] + 0.05 * rng.standard_normal((L, d))
+    K16 = bf(Kf)[None]
+    p = orc.Params(Cq=4, m0=8, n_max=200, tau_mode=orc.TAU_ABSOLUTE, tau_value=1.0, topk=2,
+                   iters_k=10)
+    kc = orc.cluster_k_multistage(K16, p)
+    lab = kc.labels[0]
+    for c in np.unique(lab):
+        assert len(np.unique(comp[lab == c])) == 1
+    assert kc.F[0] == 0
+
+
+# ----------------------------------------------------------------- tau
+
+def test_tau_rules_by_hand():
+    d = np.arange(1, 11, dtype=np.float32)
+    assert orc.tau(d, orc.TAU_PERCENTILE, 900) == 9.0     # nearest rank ceil(0.9*10) = 9
+    assert orc.tau(d, orc.TAU_PERCENTILE, 1000) == 10.0
+    assert orc.tau(d, orc.TAU_PERCENTILE, 1) == 1.0
+    assert orc.tau(np.array([1, 2, 3], np.float32), orc.TAU_MEAN_FACTOR, 1.5) == 3.0
+    assert orc.tau(d, orc.TAU_ABSOLUTE, 4.25) == 4.25
+    rng = np.random.default_rng(7)
+    x = rng.uniform(0, 20, 100000).astype(np.float32)
+    assert abs(orc.tau(x, orc.TAU_MEAN_FACTOR, 1.5) - 1.5 * x.astype(np.float64).mean()) < 1e-5
+
+
+# ----------------------------------------------------------------- Algorithm 1
+
+@pytest.mark.parametrize("case", [0, 1])
+def test_multistage_hand_example(case):
+    g = _golden("multistage_hand.json")
+    c = g["cases"][case]
+    K16 = bf(np.array(g["keys"], np.float32))[None]
+    p = orc.Params(Cq=1, m0=g["m0"], n_max=c["n_max"], tau_mode=orc.TAU_ABSOLUTE,
+                   tau_value=c["tau"], topk=1, iters_k=g["iters"])
+    kc = orc.cluster_k_multistage(K16, p)
+    assert kc.n_k[0] == c["n_k"] and kc.F[0] == c["F"] and kc.stages[0] == c["stages"]
+    assert kc.labels[0].tolist() == c["labels"]
+    assert kc.removed_stage[0].tolist() == c["removed_stage"]
+    assert np.allclose(kc.C[0, :c["n_k"]], np.array(c["centres"]), rtol=1e-6)
+    r0 = np.array(c["removed_stage"]) == 0
+    # fp32 centres of ~100-sized coordinates carry ~2^-24 * 100 absolute error
+    assert np.allclose(kc.removed_dist[0][r0], np.array(g["stage0_distances"])[r0], rtol=0,
+                       atol=1e-5)
+
+
+def test_multistage_invariants_tiny_config():
+    cfg = synth.CONFIGS[1]
+    _, K, _ = synth.make_layer(cfg)
+    p = orc.Params.from_layer_config(cfg)
+    kc = orc.cluster_k_multistage(K[0], p)
+    L = cfg.L
+    # tau follows the pooled mean rule
+    assert kc.tau > 0
+    for h in range(cfg.H):
+        nk, rs, rd = int(kc.n_k[h]), kc.removed_stage[h], kc.removed_dist[h]
+        assert (kc.labels[h] >= 0).all() and (kc.labels[h] < nk).all()
+        # every token that left U had d < tau at that stage
+        assert (rd[rs >= 0] < kc.tau).all()
+        # tokens only stay unabsorbed when the fallback fired
+        assert ((rs < 0).any()) == bool(kc.F[h])
+        # n_k is the sum of the stage sizes m_t
+        tot, nU = 0, L
+        for t in range(int(kc.stages[h])):
+            m = orc.stage_clusters(cfg.m0, nU, L, t)
+            tot += m
+            nU -= int((rs == t).sum())
+        assert tot == nk
+    # recompute the stage-0 mean from the stage-0 distances is not possible
+    # from outputs alone; check the rule on tokens absorbed at stage 0
+    assert (kc.removed_dist[kc.removed_stage == 0] < kc.tau).all()
+
+
+def test_multistage_infinite_tau_is_plain_kmeans():
+    """tau = inf: stage 0 absorbs everything, so Algorithm 1 reduces to one
+    k-means with m0 centres (seeded with tag 1) and its final assignment."""
+    cfg = synth.CONFIGS[1]
+    _, K, _ = synth.make_layer(cfg, heads=[0])
+    p = orc.Params(Cq=4, m0=32, n_max=128, tau_mode=orc.TAU_ABSOLUTE, tau_value=np.inf,
+                   topk=4, iters_k=10, seed=77)
+    kc = orc.cluster_k_multistage(K[0], p)
+    assert kc.n_k[0] == 32 and kc.F[0] == 0 and kc.stages[0] == 1
+    X = synth.bf16_bits_to_f32(K[0, 0])
+    init = X[orc.seed_pick(77, 0, 1, cfg.L, 32)]
+    lab, _, C = orc.kmeans(X, init, 10)
+    assert np.array_equal(kc.C[0, :32], C)
+    assert (kc.labels[0] == lab).all()
+
+
+def test_multistage_zero_tau_falls_back():
+    """tau = 0 absorbs nothing (d < 0 never holds): every stage re-clusters all
+    L tokens with m0 centres until |C| >= N_max, then F is set."""
+    cfg = synth.CONFIGS[1]
+    _, K, _ = synth.make_layer(cfg, heads=[0])
+    p = orc.Params(Cq=4, m0=32, n_max=100, tau_mode=orc.TAU_ABSOLUTE, tau_value=0.0,
+                   topk=4, iters_k=2)
+    kc = orc.cluster_k_multistage(K[0], p)
+    assert kc.F[0] == 1 and kc.n_k[0] == 128 and kc.stages[0] == 4
+    assert (kc.removed_stage[0] == -1).all()
+
+
+def test_multistage_nmax_below_m0_falls_back_after_stage0():
+    cfg = synth.CONFIGS[1]
+    _, K, _ = synth.make_layer(cfg, heads=[1])
+    p = orc.Params(Cq=4, m0=32, n_max=16, tau_mode=orc.TAU_MEAN_FACTOR, tau_value=0.5,
+                   topk=4, iters_k=3)
+    kc = orc.cluster_k_multistage(K[0], p)
+    assert kc.n_k[0] == 32 and kc.F[0] == 1 and kc.stages[0] == 1
+
+
+def test_single_query_clusters_when_cq_equals_l():
+    """Cq = L: the seeded init takes every token (strata of width 1) and each
+    distinct query stays alone in its cluster."""
+    rng = np.random.default_rng(8)
+    Q = bf(rng.standard_normal((1, 64, 16)))
+    p = orc.Params(Cq=64, m0=1, n_max=2, tau_mode=0, tau_value=1.0, topk=1, iters_q=3)
+    lab, C, cnt = orc.cluster_q(Q, p)
+    assert (lab[0] == np.arange(64)).all() and (cnt == 1).all()
+
+
+# ----------------------------------------------------------------- stats
+
+def test_key_stats_against_numpy():
+    cfg = synth.CONFIGS[1]
+    _, K, _ = synth.make_layer(cfg)
+    p = orc.Params.from_layer_config(cfg)
+    kc = orc.cluster_k_multistage(K[0], p)
+    st = orc.key_stats(K[0], kc)
+    for h in range(cfg.H):
+        X = synth.bf16_bits_to_f32(K[0, h]).astype(np.float64)
+        lab = kc.labels[h]
+        assert st.counts[h].sum() == cfg.L
+        sse_tot = 0.0
+        for c in range(int(kc.n_k[h])):
+            m = lab == c
+            assert st.counts[h, c] == m.sum()
+            if m.any():
+                assert np.array_equal(st.kmax[h, c], X[m].max(0).astype(np.float32))
+                assert np.array_equal(st.kmin[h, c], X[m].min(0).astype(np.float32))
+                s = ((X[m] - kc.C[h, c].astype(np.float64)) ** 2).sum()
+                assert abs(st.sse[h, c] - s) <= 1e-4 * max(s, 1e-3)
+                sse_tot += s
+        assert abs(st.mse[h] - sse_tot / cfg.L) <= 1e-4 * sse_tot / cfg.L
+        assert st.comp[h] == np.float32(1.0) / st.mse[h]
+
+
+# ----------------------------------------------------------------- Eq. (1)
+
+def test_quest_hand_example():
+    g = _golden("quest_attention_hand.json")["quest"]
+    S = orc.quest(np.array([g["q"]], np.float32), np.array([g["kmax"]], np.float32),
+                  np.array([g["kmin"]], np.float32), np.array([2], np.int32))
+    assert S[0, 0] == g["quest"]
+    # Eq. (2) as printed (k+ / k- of the bounds) is not Eq. (1)
+    q = np.array(g["q"], np.float64)
+    e2 = np.maximum(q, 0) @ np.maximum(g["kmax"], 0) + np.minimum(q, 0) @ np.minimum(g["kmin"], 0)
+    assert e2 == g["eq2_as_printed_value"] != g["quest"]
+
+
+def test_quest_is_upper_bound_and_tensor_form():
+    """Check (c): Quest(q, K_c) >= q.k for every member k (raw and normalised
+    q), equality for single-member clusters, and Eq. (1) equals the
+    two-product form q+.Kmax + q-.Kmin."""
+    cfg = synth.CONFIGS[1]
+    Q, K, _ = synth.make_layer(cfg, heads=[0])
+    p = orc.Params.from_layer_config(cfg)
+    kc = orc.cluster_k_multistage(K[0], p)
+    st = orc.key_stats(K[0], kc)
+    nk = int(kc.n_k[0])
+    X = synth.bf16_bits_to_f32(K[0, 0]).astype(np.float64)
+    inv, xh = orc.qnorm(Q[0, 0][:200])
+    for qs in (synth.bf16_bits_to_f32(Q[0, 0][:200]), xh):
+        S = orc.quest(qs, st.kmax[0, :nk], st.kmin[0, :nk], st.counts[0, :nk])
+        dots = qs.astype(np.float64) @ X.T
+        for c in range(nk):
+            m = kc.labels[0] == c
+            if not m.any():
+                assert np.isneginf(S[:, c]).all()
+                continue
+            mx = dots[:, m].max(1)
+            assert (S[:, c] >= mx - 1e-4 * (np.abs(mx) + 1)).all()
+        q = qs.astype(np.float64)
+        two = np.maximum(q, 0) @ st.kmax[0, :nk].T.astype(np.float64) + \
+            np.minimum(q, 0) @ st.kmin[0, :nk].T.astype(np.float64)
+        ne = st.counts[0, :nk] > 0
+        assert np.allclose(S[:, ne], two[:, ne], rtol=1e-5, atol=1e-4)
+    # single-member cluster: the bound is attained
+    k1 = X[:1].astype(np.float32)
+    q1 = synth.bf16_bits_to_f32(Q[0, 0][:50])
+    S1 = orc.quest(q1, k1, k1, np.array([1], np.int32))
+    assert np.allclose(S1[:, 0], q1.astype(np.float64) @ k1[0].astype(np.float64), rtol=1e-5, atol=1e-5)
+
+
+def test_topk_bruteforce_with_ties_and_empties():
+    rng = np.random.default_rng(9)
+    S = rng.integers(0, 6, size=(20, 30)).astype(np.float32)
+    S[:, 7] = -np.inf
+    k = 9
+    sel = orc.topk(S, k)
+    for a in range(20):
+        order = sorted(range(30), key=lambda c: (-S[a, c], c))[:k]
+        assert sel[a].tolist() == sorted(order)
+        assert 7 not in sel[a]
+
+
+def test_topk_count_rule():
+    assert orc.topk_count(8, 100, 100) == 8
+    assert orc.topk_count(-100, 500, 500) == 50
+    assert orc.topk_count(-100, 501, 501) == 51      # ceil
+    assert orc.topk_count(-50, 10, 10) == 1
+    assert orc.topk_count(64, 100, 20) == 20          # clamp to non-empty
+    assert orc.topk_count(-1, 3, 3) == 1              # at least one
+
+
+# ----------------------------------------------------------------- attention
+
+def test_attention_hand_example():
+    g = _golden("quest_attention_hand.json")["attention"]
+    Q = bf([g["q"]])
+    K = bf(g["keys"])
+    V = bf(g["values"])
+    o = orc.attention_rows(Q, K, V, np.zeros(1, np.int32), np.zeros(2, np.int32), None, True,
+                           [0], scale=g["scale"])
+    assert np.allclose(o[0], g["out"], atol=1e-15)
+
+
+def test_dense_attention_equals_torch_sdpa():
+    import torch
+    rng = np.random.default_rng(10)
+    L, d = 300, 64
+    Q, K, V = (bf(rng.standard_normal((L, d))) for _ in range(3))
+    o = orc.attention_rows(Q, K, V, np.zeros(L, np.int32), np.zeros(L, np.int32), None, True,
+                           np.arange(L))
+    t = [torch.from_numpy(synth.bf16_bits_to_f32(x).astype(np.float64))[None, None] for x in (Q, K, V)]
+    ref = torch.nn.functional.scaled_dot_product_attention(*t)[0, 0].numpy()
+    assert np.abs(o - ref).max() < 1e-12
+
+
+def test_all_selected_equals_dense_and_error_split():
+    """Check (a): selecting every non-empty key cluster gives dense attention.
+    Check (d): o - o_S = (1 - w_S)(o_Sbar - o_S) (ClusterAttention Sec. 1.2,
+    Eq. (3)-(4)) with S the keys of the selected clusters."""
+    cfg = synth.CONFIGS[1]
+    Q, K, V = synth.make_layer(cfg, heads=[0])
+    Q, K, V = Q[0, 0], K[0, 0], V[0, 0]
+    p = orc.Params.from_layer_config(cfg)
+    r = orc.layer(Q[None], K[None], V[None], p, attention=False)
+    nk = int(r.kc.n_k[0])
+    lq, lk = r.labels_q[0], r.kc.labels[0]
+    rows = np.arange(0, cfg.L, 97)
+    allsel = np.tile(np.arange(nk, dtype=np.int32), (cfg.Cq, 1))
+    o_all = orc.attention_rows(Q, K, V, lq, lk, allsel, False, rows)
+    o_dense = orc.attention_rows(Q, K, V, lq, lk, None, True, rows)
+    assert np.abs(o_all - o_dense).max() < 1e-12
+    sel = r.sel[0]
+    o_S = orc.attention_rows(Q, K, V, lq, lk, sel, False, rows)
+    Vf = synth.bf16_bits_to_f32(V).astype(np.float64)
+    for n, i in enumerate(rows):
+        w = orc.dense_weights(Q[i], K)
+        inS = np.isin(lk, sel[lq[i]])
+        wS = w[inS].sum()
+        comp = [c for c in range(nk) if c not in set(sel[lq[i]].tolist())]
+        o_Sbar = orc.attention_rows(Q, K, V, lq, lk, np.array([comp] * cfg.Cq, np.int32), False,
+                                    [i])[0] if comp else np.zeros(cfg.d)
+        lhs = o_dense[n] - o_S[n]
+        rhs = (1 - wS) * (o_Sbar - o_S[n])
+        assert np.abs(lhs - rhs).max() < 1e-5
+        # and o itself is the weighted combination (Eq. (3))
+        assert np.abs(o_dense[n] - (w[:, None] * Vf).sum(0)).max() < 1e-10
