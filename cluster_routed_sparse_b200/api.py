@@ -1,0 +1,146 @@
+"""Python binding of libac over torch tensors (device memory and streams only).
+
+Every call forwards torch data pointers and the current CUDA stream to the C
+ABI in include/ac.h; all arithmetic of the layer runs in libac's kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import ACConfig, ACStageTimes, ACAttnCounters, check
+
+_TORCH_DTYPES = {"<f4": torch.float32, "<i4": torch.int32, "|u1": torch.uint8, "<i2": torch.int16}
+
+
+class _CudaArray:
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _bits(t):
+    """bf16 tensor -> pointer to its uint16 bit patterns."""
+    if t.dtype != torch.bfloat16:
+        raise TypeError("Q, K, V, O must be torch.bfloat16")
+    return _ptr(t)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+class SparseLayer:
+    """One cluster-routed sparse attention layer context for [B, H, L, d] inputs.
+
+    Hyper-parameters follow ac_config in include/ac.h.  The context owns its
+    workspace and the warm-start state carried across denoising steps."""
+
+    def __init__(self, B: int, H: int, L: int, d: int, *, Cq: int, m0: int, n_max: int,
+                 tau_mode: int, tau_value: float, topk: int, iters_q: int = 10,
+                 iters_k: int = 10, iters_warm: int = 2, seed: int = 1234, scale: float = 0.0):
+        self.lib = _lib.load()
+        self.B, self.H, self.L, self.d = B, H, L, d
+        self.cfg = ACConfig(Cq, m0, n_max, tau_mode, float(tau_value), topk, iters_q, iters_k,
+                            iters_warm, 0, seed & (2**64 - 1), float(scale), 0)
+        self.Cq, self.Ccap = Cq, n_max + m0
+        h = ctypes.c_void_p()
+        check(self.lib.ac_create(ctypes.byref(self.cfg), B, H, L, d, ctypes.byref(h)))
+        self.ctx = h
+
+    @classmethod
+    def from_config(cls, cfg, seed: int = 1234, B=None, H=None, L=None):
+        """Build from a synth.LayerConfig (shape overrides allowed)."""
+        return cls(B or cfg.B, H or cfg.H, L or cfg.L, cfg.d, Cq=cfg.Cq, m0=cfg.m0, n_max=cfg.n_max,
+                   tau_mode=cfg.tau_mode, tau_value=cfg.tau_value, topk=cfg.topk,
+                   iters_q=cfg.iters_q, iters_k=cfg.iters_k, iters_warm=cfg.iters_warm, seed=seed)
+
+    # ------------------------------------------------------------------ calls
+    def cluster_q(self, Q, init=None, iters: int = -1, labels=None, centroids=None):
+        check(self.lib.ac_cluster_q(self.ctx, _bits(Q), _ptr(init), iters, _ptr(labels),
+                                    _ptr(centroids), _stream()), self.ctx)
+
+    def cluster_k(self, K, warm_centroids=None, warm_n_k=None, warm_dense=None, labels=None,
+                  centroids=None, n_k=None, dense=None, comp=None):
+        check(self.lib.ac_cluster_k_multistage(
+            self.ctx, _bits(K), _ptr(warm_centroids), _ptr(warm_n_k), _ptr(warm_dense),
+            _ptr(labels), _ptr(centroids), _ptr(n_k), _ptr(dense), _ptr(comp), _stream()), self.ctx)
+
+    def score_select(self, topk: int = 0, sel=None, k=None):
+        check(self.lib.ac_score_select(self.ctx, topk, _ptr(sel), _ptr(k), _stream()), self.ctx)
+
+    def sparse_attn(self, Q, K, V, O=None):
+        if O is None:
+            O = torch.empty_like(Q)
+        check(self.lib.ac_sparse_attn(self.ctx, _bits(Q), _bits(K), _bits(V), _bits(O), _stream()),
+              self.ctx)
+        return O
+
+    def forward(self, Q, K, V, O=None, warm: bool = False, times: bool = False):
+        if O is None:
+            O = torch.empty_like(Q)
+        t = ACStageTimes() if times else None
+        check(self.lib.ac_layer_forward(self.ctx, _bits(Q), _bits(K), _bits(V), _bits(O),
+                                        1 if warm else 0, ctypes.byref(t) if t is not None else None,
+                                        _stream()), self.ctx)
+        return (O, t.as_dict()) if times else O
+
+    def forward_host(self, hQ, hK, hV, hO, warm: bool = False):
+        """Host (ideally pinned) bf16 tensors in and out; copies inside the call."""
+        check(self.lib.ac_layer_forward_host(self.ctx, _bits(hQ), _bits(hK), _bits(hV), _bits(hO),
+                                             1 if warm else 0, _stream()), self.ctx)
+        return hO
+
+    def synchronize(self):
+        check(self.lib.ac_synchronize(self.ctx, _stream()), self.ctx)
+
+    def tensor(self, which: int) -> torch.Tensor:
+        """Device view of an intermediate tensor (ac_get_tensor); valid until the next call."""
+        p = ctypes.c_void_p()
+        shape = (ctypes.c_int64 * 4)()
+        check(self.lib.ac_get_tensor(self.ctx, which, ctypes.byref(p), shape), self.ctx)
+        typ = _lib.TENSOR_TYPES[which]
+        dims = [int(x) for x in shape[:4]]
+        while len(dims) > 1 and dims[-1] == 1:
+            dims.pop()
+        t = torch.as_tensor(_CudaArray(p.value, dims, typ), device="cuda")
+        if which in (_lib.AC_T_KMAX, _lib.AC_T_KMIN):
+            t = t.view(torch.bfloat16)
+        return t
+
+    def counters(self) -> dict:
+        c = ACAttnCounters()
+        check(self.lib.ac_get_attn_counters(self.ctx, ctypes.byref(c)), self.ctx)
+        return {f: int(getattr(c, f)) for f, _ in c._fields_}
+
+    def export_state(self) -> bytes:
+        n = ctypes.c_int64(0)
+        check(self.lib.ac_state_export(self.ctx, None, ctypes.byref(n)), self.ctx)
+        buf = ctypes.create_string_buffer(n.value)
+        check(self.lib.ac_state_export(self.ctx, buf, ctypes.byref(n)), self.ctx)
+        return buf.raw
+
+    def import_state(self, data: bytes):
+        buf = ctypes.create_string_buffer(data, len(data))
+        check(self.lib.ac_state_import(self.ctx, buf, len(data)), self.ctx)
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            self.lib.ac_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,700 @@
+// ac_api.cu -- the C ABI of libac: context, workspace, and the host control
+// flow of the cluster-routed sparse layer (AdaCluster, arXiv 2604.18348,
+// Algorithm 3, with Algorithm 1 for the keys).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "ac_device.cuh"
+#include "ac_internal.h"
+
+using namespace ac;
+
+namespace {
+
+const char *g_static_msg = "";
+
+ac_status fail(ac_ctx *c, ac_status st, const char *what) {
+    if (c) c->msg = what;
+    return st;
+}
+
+ac_status cuda_fail(ac_ctx *c, cudaError_t e, const char *what) {
+    if (c) {
+        char buf[512];
+        snprintf(buf, sizeof(buf), "%s: %s", what, cudaGetErrorString(e));
+        c->msg = buf;
+    }
+    return AC_ERR_CUDA;
+}
+
+#define CK(call, what)                                   \
+    do {                                                 \
+        cudaError_t e_ = (call);                         \
+        if (e_ != cudaSuccess) return cuda_fail(c, e_, what); \
+    } while (0)
+
+// Cluster count of stage t > 0 of Algorithm 1 ("re-cluster these outlier tokens
+// with a few number of new clusters"): proportional to what is left, so that
+// the mean cluster size stays L/m0.
+int stage_clusters(int m0, int64_t nU, int64_t L, int t) {
+    if (t == 0) return (int)std::min<int64_t>(m0, nU);
+    int64_t m = (m0 * nU + L - 1) / L;
+    m = std::max<int64_t>(1, std::min<int64_t>(m, nU));
+    return (int)m;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+ac_status make_tmap(ac_ctx *c, CUtensorMap *tm, void *base, int64_t rows, int d, int box_rows) {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+            return fail(c, AC_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(c, AC_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    return AC_OK;
+}
+
+template <class T>
+cudaError_t dalloc(T **p, size_t n) {
+    return cudaMalloc(reinterpret_cast<void **>(p), std::max<size_t>(n, 1) * sizeof(T));
+}
+
+// Read back the device error word, clear it, and turn it into a status.
+ac_status check_dev_err(ac_ctx *c, cudaStream_t s) {
+    CK(cudaMemcpyAsync(c->h_err, c->err, sizeof(uint32_t), cudaMemcpyDeviceToHost, s), "error word");
+    CK(cudaStreamSynchronize(s), "stream sync");
+    uint32_t e = *c->h_err;
+    if (e) {
+        CK(cudaMemsetAsync(c->err, 0, sizeof(uint32_t), s), "error word reset");
+        if (e & DEV_ERR_TIMEOUT) return fail(c, AC_ERR_TIMEOUT, "a bounded in-kernel wait expired");
+        if (e & DEV_ERR_NONFINITE) return fail(c, AC_ERR_NONFINITE, "non-finite value in an input");
+        return fail(c, AC_ERR_CUDA, "kernel bounds check failed");
+    }
+    return AC_OK;
+}
+
+// ---------------------------------------------------------------- k-means pieces
+// T Lloyd iterations (assign, sort, update) then a final assignment + sort.
+struct Lloyd {
+    AssignArgs as;
+    SortArgs so;
+    UpdateArgs up;
+};
+
+cudaError_t run_lloyd(Lloyd &k, int T, bool final_sort, cudaStream_t s) {
+    cudaError_t e;
+    for (int t = 0; t < T; ++t) {
+        if ((e = launch_assign_exact(k.as, s)) != cudaSuccess) return e;
+        if ((e = launch_counting_sort(k.so, s)) != cudaSuccess) return e;
+        if ((e = launch_update(k.up, s)) != cudaSuccess) return e;
+    }
+    if ((e = launch_assign_exact(k.as, s)) != cudaSuccess) return e;
+    if (final_sort && (e = launch_counting_sort(k.so, s)) != cudaSuccess) return e;
+    return cudaSuccess;
+}
+
+// Algorithm 3 line 3 on the context's buffers.
+ac_status cluster_q_impl(ac_ctx *c, const bf16 *Q, const float *init, int iters, cudaStream_t s) {
+    const int64_t L = c->L;
+    CK(launch_qnorm(Q, c->inv_q, (int64_t)c->BH * L, c->d, c->err, s), "qnorm");
+    if (init) {
+        if (init != c->cent_q)
+            CK(cudaMemcpyAsync(c->cent_q, init, sizeof(float) * c->BH * c->Cq * c->d, cudaMemcpyDeviceToDevice, s),
+               "init copy");
+    } else {
+        SeedArgs sa{Q, c->inv_q, L, nullptr, nullptr, c->L, c->cent_q, (int64_t)c->Cq * c->d, nullptr,
+                    nullptr, c->Cq, c->Cq, c->cfg.seed, 0, c->BH, c->d};
+        CK(launch_seed(sa, s), "seed q");
+    }
+    Lloyd k;
+    k.as = AssignArgs{Q, c->inv_q, L, nullptr, nullptr, c->L, c->cent_q, (int64_t)c->Cq * c->d, nullptr,
+                      nullptr, c->Cq, c->labels_q, nullptr, c->BH, c->d};
+    k.so = SortArgs{c->labels_q, L, nullptr, c->L, nullptr, c->Cq, c->Cq, c->perm_q, c->offs_q, c->Cq + 1,
+                    c->counts_q, c->Cq, c->BH};
+    k.up = UpdateArgs{Q, c->inv_q, L, nullptr, c->perm_q, c->offs_q, c->Cq + 1, c->cent_q,
+                      (int64_t)c->Cq * c->d, nullptr, nullptr, c->Cq, c->BH, c->d, c->Cq};
+    CK(run_lloyd(k, iters, true, s), "q lloyd");
+    c->have_q = true;
+    return AC_OK;
+}
+
+// Algorithm 1, step 0 (all units batched; one readback of |U| per stage).
+// The loop state lives in host vectors; the pinned staging buffers are only
+// rewritten after a stream synchronisation, so no pending copy reads them.
+ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
+    const int BH = c->BH, L = c->L, d = c->d, m0 = c->cfg.m0;
+    const int64_t cstride = (int64_t)c->Ccap * d;
+    CK(launch_iota_rows(c->u_idx, c->u_cnt, BH, L, s), "iota");
+    CK(cudaMemsetAsync(c->removed_stage, 0xFF, sizeof(int) * BH * (size_t)L, s), "removed init");
+    CK(cudaMemsetAsync(c->tau_acc, 0, sizeof(unsigned long long), s), "tau acc");
+    std::vector<int> done(BH, 0), stages(BH, 0), nk(BH, 0), m(BH, 0), ucnt(BH, L);
+    std::vector<uint8_t> dense(BH, 0);
+    for (int t = 0;; ++t) {
+        if (t > 0) {
+            CK(cudaMemcpyAsync(c->h_u_cnt, c->u_cnt, sizeof(int) * BH, cudaMemcpyDeviceToHost, s), "u_cnt");
+            CK(cudaStreamSynchronize(s), "stage sync");
+            for (int h = 0; h < BH; ++h) {
+                ucnt[h] = c->h_u_cnt[h];
+                nk[h] += m[h];  // line 19 of the previous stage
+            }
+        }
+        bool any = false;
+        int max_m = 0;
+        for (int h = 0; h < BH; ++h) {
+            m[h] = 0;
+            if (done[h]) continue;
+            if (ucnt[h] == 0) {            // line 6: U is empty
+                done[h] = 1;
+                stages[h] = t;
+                continue;
+            }
+            if (nk[h] >= c->cfg.n_max) {  // lines 7-9
+                dense[h] = 1;
+                done[h] = 1;
+                stages[h] = t;
+                continue;
+            }
+            m[h] = stage_clusters(m0, ucnt[h], L, t);  // line 11
+            max_m = std::max(max_m, m[h]);
+            any = true;
+        }
+        if (!any) break;
+        for (int h = 0; h < BH; ++h) {
+            c->h_st_m[h] = m[h];
+            c->h_n_k[h] = nk[h];
+        }
+        CK(cudaMemcpyAsync(c->st_m, c->h_st_m, sizeof(int) * BH, cudaMemcpyHostToDevice, s), "st_m");
+        CK(cudaMemcpyAsync(c->n_k, c->h_n_k, sizeof(int) * BH, cudaMemcpyHostToDevice, s), "n_k");
+        // line 12: KMeans(U, m_t), stage centres appended after the n_k existing ones
+        SeedArgs sa{K, nullptr, L, c->u_idx, c->u_cnt, 0, c->cent_k, cstride, c->n_k, c->st_m, 0, max_m,
+                    c->cfg.seed, 1 + t, BH, d};
+        CK(launch_seed(sa, s), "seed k");
+        Lloyd k;
+        k.as = AssignArgs{K, nullptr, L, c->u_idx, c->u_cnt, 0, c->cent_k, cstride, c->n_k, c->st_m, 0,
+                          c->st_labels, c->dmin_k, BH, d};
+        k.so = SortArgs{c->st_labels, L, c->u_cnt, 0, c->st_m, 0, max_m, c->st_perm, c->st_offs, m0 + 1, nullptr,
+                        0, BH};
+        k.up = UpdateArgs{K, nullptr, L, c->u_idx, c->st_perm, c->st_offs, m0 + 1, c->cent_k, cstride, c->n_k,
+                          c->st_m, 0, BH, d, max_m};
+        CK(run_lloyd(k, c->cfg.iters_k, false, s), "k stage lloyd");
+        // line 14: d_i = ||k_i - c(k_i)||
+        CK(launch_stage_dist(c->dmin_k, c->st_dist, c->u_cnt, c->st_m, L, BH, t == 0 ? c->tau_acc : nullptr, s),
+           "stage dist");
+        if (t == 0) {
+            const int64_t n_total = (int64_t)BH * L;
+            if (c->cfg.tau_mode == AC_TAU_MEAN_FACTOR) {
+                CK(launch_tau_mean(c->tau_acc, nullptr, n_total, c->cfg.tau_value, c->tau, s), "tau mean");
+            } else if (c->cfg.tau_mode == AC_TAU_PERCENTILE) {
+                CK(launch_tau_percentile(c->st_dist, c->st_m, L, BH, n_total, (int)c->cfg.tau_value, c->radix,
+                                         c->tau, s),
+                   "tau percentile");
+            } else {
+                CK(cudaMemcpyAsync(c->tau, &c->cfg.tau_value, sizeof(float), cudaMemcpyHostToDevice, s), "tau");
+            }
+        }
+        // lines 13-18: drop the keys within tau of their centre from U
+        CK(launch_remove(c->st_dist, c->tau, c->u_idx, c->u_idx2, c->u_cnt, c->st_m, c->removed_stage, t, L, BH, s),
+           "remove");
+        std::swap(c->u_idx, c->u_idx2);
+    }
+    for (int h = 0; h < BH; ++h) {
+        c->h_n_k[h] = nk[h];
+        c->h_dense[h] = dense[h];
+        c->h_st_m[h] = stages[h];
+    }
+    CK(cudaMemcpyAsync(c->n_k, c->h_n_k, sizeof(int) * BH, cudaMemcpyHostToDevice, s), "n_k");
+    CK(cudaMemcpyAsync(c->dense, c->h_dense, BH, cudaMemcpyHostToDevice, s), "dense");
+    CK(cudaMemcpyAsync(c->stages, c->h_st_m, sizeof(int) * BH, cudaMemcpyHostToDevice, s), "stages");
+    CK(cudaStreamSynchronize(s), "stage end sync");  // the staging buffers are reused by the next call
+    // line 22: every key to its closest centre among all of C
+    AssignArgs fa{K, nullptr, L, nullptr, nullptr, L, c->cent_k, cstride, nullptr, c->n_k, 0, c->labels_k,
+                  c->dmin_k, BH, d};
+    CK(launch_assign_exact(fa, s), "final assign");
+    return AC_OK;
+}
+
+// Warm-started step (Sec. 3.2.2 "Efficient initialization"): Lloyd over all
+// keys from the previous centres, cluster counts fixed, dense units skipped.
+__global__ void k_warm_counts(const int *n_k, const uint8_t *dense, int *ncent, int BH) {
+    int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h < BH) ncent[h] = dense[h] ? 0 : n_k[h];
+}
+
+ac_status cluster_k_warm(ac_ctx *c, const bf16 *K, cudaStream_t s) {
+    const int BH = c->BH, L = c->L, d = c->d;
+    const int64_t cstride = (int64_t)c->Ccap * d;
+    k_warm_counts<<<(BH + 127) / 128, 128, 0, s>>>(c->n_k, c->dense, c->st_m, BH);
+    CK(cudaGetLastError(), "warm counts");
+    Lloyd k;
+    k.as = AssignArgs{K, nullptr, L, nullptr, nullptr, L, c->cent_k, cstride, nullptr, c->st_m, 0, c->labels_k,
+                      c->dmin_k, BH, d};
+    k.so = SortArgs{c->labels_k, L, nullptr, L, c->n_k, 0, c->Ccap, c->perm_k, c->offs_k, c->Ccap + 1, c->counts_k,
+                    c->Ccap, BH};
+    k.up = UpdateArgs{K, nullptr, L, nullptr, c->perm_k, c->offs_k, c->Ccap + 1, c->cent_k, cstride, nullptr,
+                      c->st_m, 0, BH, d, c->Ccap};
+    CK(run_lloyd(k, c->cfg.iters_warm, false, s), "warm lloyd");
+    return AC_OK;
+}
+
+// Cluster-order permutation of the keys and the per-cluster statistics.
+ac_status key_stats_impl(ac_ctx *c, const bf16 *K, cudaStream_t s) {
+    SortArgs so{c->labels_k, c->L, nullptr, c->L, c->n_k, 0, c->Ccap, c->perm_k, c->offs_k, c->Ccap + 1,
+                c->counts_k, c->Ccap, c->BH};
+    CK(launch_counting_sort(so, s), "k sort");
+    StatsArgs st{K, c->L, c->perm_k, c->offs_k, c->Ccap + 1, c->dmin_k, c->n_k, c->Ccap, c->d, c->BH,
+                 c->counts_k, c->kmax, c->kmin, c->sse, c->mse, c->comp};
+    CK(launch_key_stats(st, s), "k stats");
+    c->have_k = true;
+    return AC_OK;
+}
+
+ac_status score_select_impl(ac_ctx *c, int topk, cudaStream_t s) {
+    SelectArgs a{c->cent_q, c->kmax, c->kmin, c->counts_k, c->n_k, c->dense, c->offs_k, c->counts_q,
+                 c->Cq, c->Ccap, c->d, c->BH, c->L, topk != 0 ? topk : c->cfg.topk,
+                 c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix};
+    CK(launch_score_select(a, s), "score select");
+    return AC_OK;
+}
+
+ac_status sparse_attn_impl(ac_ctx *c, const bf16 *Q, const bf16 *K, const bf16 *V, bf16 *O, cudaStream_t s) {
+    CK(launch_permute_rows(Q, c->perm_q, c->Qp, c->L, c->d, c->BH, s), "permute q");
+    CK(launch_permute_rows(K, c->perm_k, c->Kp, c->L, c->d, c->BH, s), "permute k");
+    CK(launch_permute_rows(V, c->perm_k, c->Vp, c->L, c->d, c->BH, s), "permute v");
+    CK(cudaMemsetAsync(c->counters, 0, 4 * sizeof(unsigned long long), s), "counters");
+    AttnArgs a{&c->tm_q, &c->tm_k, &c->tm_v, O, c->perm_q, c->offs_q, c->counts_q, c->tile_prefix, c->ranges,
+               c->nboxes, c->ksel, c->dense, c->L, c->Cq, c->Ccap, c->BH, c->d,
+               (float)(c->scale * 1.4426950408889634), c->err, c->counters};
+    CK(launch_sparse_attn(a, s), "sparse attention");
+    return AC_OK;
+}
+
+void free_all(ac_ctx *c) {
+    void *dev[] = {c->inv_q, c->labels_q, c->cent_q, c->counts_q, c->perm_q, c->offs_q, c->labels_k, c->dmin_k,
+                   c->cent_k, c->n_k, c->dense, c->stages, c->removed_stage, c->tau, c->tau_acc, c->counts_k,
+                   c->perm_k, c->offs_k, c->kmax, c->kmin, c->sse, c->mse, c->comp, c->u_idx, c->u_idx2,
+                   c->u_cnt, c->st_m, c->st_labels, c->st_dist, c->st_perm, c->st_offs, c->st_counts, c->radix,
+                   c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->Qp, c->Kp, c->Vp,
+                   c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err};
+    for (void *p : dev)
+        if (p) cudaFree(p);
+    void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err};
+    for (void *p : host)
+        if (p) cudaFreeHost(p);
+    for (auto &e : c->ev)
+        if (e) cudaEventDestroy(e);
+}
+
+}  // namespace
+
+// ======================================================================== ABI
+
+extern "C" {
+
+const char *ac_last_error_string(const ac_ctx *ctx) { return ctx ? ctx->msg.c_str() : g_static_msg; }
+
+ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32_t d, ac_ctx **out) {
+    if (!cfg || !out) return AC_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (B < 1 || H < 1 || L < 1) return AC_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return AC_ERR_UNSUPPORTED;
+    if (cfg->Cq < 1 || cfg->Cq > L || cfg->m0 < 1 || cfg->m0 > L || cfg->n_max < 1 || cfg->iters_q < 0 ||
+        cfg->iters_k < 0 || cfg->iters_warm < 0 || cfg->tau_mode < 0 || cfg->tau_mode > 2 || cfg->topk == 0 ||
+        cfg->reserved0 != 0 || cfg->reserved1 != 0 || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
+        return AC_ERR_INVALID_ARG;
+    if ((int64_t)B * H * L >= (int64_t)1 << 31) return AC_ERR_INVALID_ARG;
+    if (cfg->tau_mode == AC_TAU_PERCENTILE && (cfg->tau_value < 1.f || cfg->tau_value > 1000.f))
+        return AC_ERR_INVALID_ARG;
+    if ((int64_t)cfg->n_max + cfg->m0 > 16384) return AC_ERR_INVALID_ARG;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return AC_ERR_UNSUPPORTED;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return AC_ERR_UNSUPPORTED;
+    if (prop.major != 10) return AC_ERR_UNSUPPORTED;
+
+    ac_ctx *c = new (std::nothrow) ac_ctx();
+    if (!c) return AC_ERR_WORKSPACE;
+    c->cfg = *cfg;
+    c->B = B;
+    c->H = H;
+    c->L = L;
+    c->d = d;
+    c->BH = B * H;
+    c->Cq = cfg->Cq;
+    c->Ccap = cfg->n_max + cfg->m0;
+    c->device = dev;
+    c->scale = cfg->scale > 0.f ? cfg->scale : 1.0f / std::sqrt((float)d);
+
+    const size_t BH = c->BH, Lz = L, dz = d, Cq = c->Cq, Cc = c->Ccap, m0 = cfg->m0;
+    bool okm = true;
+    auto A = [&](cudaError_t e) { okm = okm && e == cudaSuccess; };
+    A(dalloc(&c->inv_q, BH * Lz));
+    A(dalloc(&c->labels_q, BH * Lz));
+    A(dalloc(&c->cent_q, BH * Cq * dz));
+    A(dalloc(&c->counts_q, BH * Cq));
+    A(dalloc(&c->perm_q, BH * Lz));
+    A(dalloc(&c->offs_q, BH * (Cq + 1)));
+    A(dalloc(&c->labels_k, BH * Lz));
+    A(dalloc(&c->dmin_k, BH * Lz));
+    A(dalloc(&c->cent_k, BH * Cc * dz));
+    A(dalloc(&c->n_k, BH));
+    A(dalloc(&c->dense, BH));
+    A(dalloc(&c->stages, BH));
+    A(dalloc(&c->removed_stage, BH * Lz));
+    A(dalloc(&c->tau, 1));
+    A(dalloc(&c->tau_acc, 1));
+    A(dalloc(&c->counts_k, BH * Cc));
+    A(dalloc(&c->perm_k, BH * Lz));
+    A(dalloc(&c->offs_k, BH * (Cc + 1)));
+    A(dalloc(&c->kmax, BH * Cc * dz));
+    A(dalloc(&c->kmin, BH * Cc * dz));
+    A(dalloc(&c->sse, BH * Cc));
+    A(dalloc(&c->mse, BH));
+    A(dalloc(&c->comp, BH));
+    A(dalloc(&c->u_idx, BH * Lz));
+    A(dalloc(&c->u_idx2, BH * Lz));
+    A(dalloc(&c->u_cnt, BH));
+    A(dalloc(&c->st_m, BH));
+    A(dalloc(&c->st_labels, BH * Lz));
+    A(dalloc(&c->st_dist, BH * Lz));
+    A(dalloc(&c->st_perm, BH * Lz));
+    A(dalloc(&c->st_offs, BH * (m0 + 1)));
+    A(dalloc(&c->st_counts, BH * m0));
+    A(dalloc(&c->radix, 260));
+    A(dalloc(&c->score, BH * Cq * Cc));
+    A(dalloc(&c->sel, BH * Cq * Cc));
+    A(dalloc(&c->ksel, BH));
+    A(dalloc(&c->ranges, BH * Cq * Cc));
+    A(dalloc(&c->nboxes, BH * Cq));
+    A(dalloc(&c->tile_prefix, BH * Cq + 1));
+    A(dalloc(&c->Qp, BH * Lz * dz));
+    A(dalloc(&c->Kp, BH * Lz * dz));
+    A(dalloc(&c->Vp, BH * Lz * dz));
+    A(dalloc(&c->counters, 4));
+    A(dalloc(&c->err, 1));
+    A(cudaMallocHost(&c->h_u_cnt, BH * sizeof(int)));
+    A(cudaMallocHost(&c->h_st_m, BH * sizeof(int)));
+    A(cudaMallocHost(&c->h_n_k, BH * sizeof(int)));
+    A(cudaMallocHost(&c->h_dense, BH));
+    A(cudaMallocHost(&c->h_err, sizeof(uint32_t)));
+    for (auto &e : c->ev) A(cudaEventCreate(&e));
+    if (!okm) {
+        free_all(c);
+        delete c;
+        cudaGetLastError();
+        return AC_ERR_WORKSPACE;
+    }
+    if (cudaMemset(c->err, 0, sizeof(uint32_t)) != cudaSuccess ||
+        cudaMemset(c->dense, 0, BH) != cudaSuccess || cudaMemset(c->n_k, 0, BH * sizeof(int)) != cudaSuccess) {
+        free_all(c);
+        delete c;
+        return AC_ERR_CUDA;
+    }
+    const int64_t rows = (int64_t)BH * L;
+    if (make_tmap(c, &c->tm_q, c->Qp, rows, d, 128) != AC_OK || make_tmap(c, &c->tm_k, c->Kp, rows, d, 8) != AC_OK ||
+        make_tmap(c, &c->tm_v, c->Vp, rows, d, 8) != AC_OK) {
+        free_all(c);
+        delete c;
+        return AC_ERR_CUDA;
+    }
+    *out = c;
+    return AC_OK;
+}
+
+ac_status ac_destroy(ac_ctx *c) {
+    if (!c) return AC_ERR_INVALID_ARG;
+    cudaDeviceSynchronize();
+    free_all(c);
+    delete c;
+    return AC_OK;
+}
+
+ac_status ac_cluster_q(ac_ctx *c, const uint16_t *Q, const float *init, int32_t iters, int32_t *labels_out,
+                       float *cent_out, void *stream) {
+    if (!c || !Q) return fail(c, AC_ERR_INVALID_ARG, "ac_cluster_q: NULL argument");
+    cudaStream_t s = (cudaStream_t)stream;
+    const int T = iters >= 0 ? iters : (init ? c->cfg.iters_warm : c->cfg.iters_q);
+    ac_status st = cluster_q_impl(c, reinterpret_cast<const bf16 *>(Q), init, T, s);
+    if (st != AC_OK) return st;
+    if (labels_out)
+        CK(cudaMemcpyAsync(labels_out, c->labels_q, sizeof(int) * (size_t)c->BH * c->L, cudaMemcpyDeviceToDevice, s),
+           "labels out");
+    if (cent_out)
+        CK(cudaMemcpyAsync(cent_out, c->cent_q, sizeof(float) * (size_t)c->BH * c->Cq * c->d,
+                           cudaMemcpyDeviceToDevice, s),
+           "centres out");
+    return check_dev_err(c, s);
+}
+
+ac_status ac_cluster_k_multistage(ac_ctx *c, const uint16_t *K, const float *warm_cent, const int32_t *warm_n_k,
+                                  const uint8_t *warm_dense, int32_t *labels_out, float *cent_out, int32_t *n_k_out,
+                                  uint8_t *dense_out, float *comp_out, void *stream) {
+    if (!c || !K) return fail(c, AC_ERR_INVALID_ARG, "ac_cluster_k_multistage: NULL argument");
+    if ((warm_cent == nullptr) != (warm_n_k == nullptr))
+        return fail(c, AC_ERR_INVALID_ARG, "warm start needs both centres and counts");
+    cudaStream_t s = (cudaStream_t)stream;
+    const bf16 *Kb = reinterpret_cast<const bf16 *>(K);
+    const size_t BH = c->BH;
+    ac_status st;
+    if (warm_cent) {
+        if (warm_cent != c->cent_k)
+            CK(cudaMemcpyAsync(c->cent_k, warm_cent, sizeof(float) * BH * c->Ccap * c->d, cudaMemcpyDeviceToDevice, s),
+               "warm centres");
+        if (warm_n_k != c->n_k)
+            CK(cudaMemcpyAsync(c->n_k, warm_n_k, sizeof(int) * BH, cudaMemcpyDeviceToDevice, s), "warm counts");
+        if (warm_dense) {
+            if (warm_dense != c->dense)
+                CK(cudaMemcpyAsync(c->dense, warm_dense, BH, cudaMemcpyDeviceToDevice, s), "warm dense");
+        } else {
+            CK(cudaMemsetAsync(c->dense, 0, BH, s), "warm dense");
+        }
+        st = cluster_k_warm(c, Kb, s);
+    } else {
+        st = cluster_k_step0(c, Kb, s);
+    }
+    if (st != AC_OK) return st;
+    if ((st = key_stats_impl(c, Kb, s)) != AC_OK) return st;
+    if (labels_out) CK(cudaMemcpyAsync(labels_out, c->labels_k, sizeof(int) * BH * c->L, cudaMemcpyDeviceToDevice, s), "out");
+    if (cent_out)
+        CK(cudaMemcpyAsync(cent_out, c->cent_k, sizeof(float) * BH * c->Ccap * c->d, cudaMemcpyDeviceToDevice, s), "out");
+    if (n_k_out) CK(cudaMemcpyAsync(n_k_out, c->n_k, sizeof(int) * BH, cudaMemcpyDeviceToDevice, s), "out");
+    if (dense_out) CK(cudaMemcpyAsync(dense_out, c->dense, BH, cudaMemcpyDeviceToDevice, s), "out");
+    if (comp_out) CK(cudaMemcpyAsync(comp_out, c->comp, sizeof(float) * BH, cudaMemcpyDeviceToDevice, s), "out");
+    c->have_state = c->have_q;
+    return check_dev_err(c, s);
+}
+
+ac_status ac_score_select(ac_ctx *c, int32_t topk, int32_t *sel_out, int32_t *k_out, void *stream) {
+    if (!c) return AC_ERR_INVALID_ARG;
+    if (!c->have_q || !c->have_k) return fail(c, AC_ERR_STATE, "ac_score_select before clustering");
+    cudaStream_t s = (cudaStream_t)stream;
+    ac_status st = score_select_impl(c, topk, s);
+    if (st != AC_OK) return st;
+    if (sel_out)
+        CK(cudaMemcpyAsync(sel_out, c->sel, sizeof(int) * (size_t)c->BH * c->Cq * c->Ccap, cudaMemcpyDeviceToDevice,
+                           s),
+           "sel out");
+    if (k_out) CK(cudaMemcpyAsync(k_out, c->ksel, sizeof(int) * (size_t)c->BH, cudaMemcpyDeviceToDevice, s), "k out");
+    return AC_OK;
+}
+
+ac_status ac_sparse_attn(ac_ctx *c, const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O,
+                         void *stream) {
+    if (!c || !Q || !K || !V || !O) return fail(c, AC_ERR_INVALID_ARG, "ac_sparse_attn: NULL argument");
+    if (!c->have_q || !c->have_k) return fail(c, AC_ERR_STATE, "ac_sparse_attn before clustering");
+    return sparse_attn_impl(c, reinterpret_cast<const bf16 *>(Q), reinterpret_cast<const bf16 *>(K),
+                            reinterpret_cast<const bf16 *>(V), reinterpret_cast<bf16 *>(O), (cudaStream_t)stream);
+}
+
+ac_status ac_layer_forward(ac_ctx *c, const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O,
+                           int32_t warm, ac_stage_times *times, void *stream) {
+    if (!c || !Q || !K || !V || !O) return fail(c, AC_ERR_INVALID_ARG, "ac_layer_forward: NULL argument");
+    if (warm && !c->have_state) return fail(c, AC_ERR_STATE, "warm step before any step 0");
+    cudaStream_t s = (cudaStream_t)stream;
+    const bf16 *Qb = reinterpret_cast<const bf16 *>(Q), *Kb = reinterpret_cast<const bf16 *>(K),
+               *Vb = reinterpret_cast<const bf16 *>(V);
+    ac_status st;
+    if (times) CK(cudaEventRecord(c->ev[0], s), "event");
+    st = cluster_q_impl(c, Qb, warm ? c->cent_q : nullptr, warm ? c->cfg.iters_warm : c->cfg.iters_q, s);
+    if (st != AC_OK) return st;
+    if (times) CK(cudaEventRecord(c->ev[1], s), "event");
+    st = warm ? cluster_k_warm(c, Kb, s) : cluster_k_step0(c, Kb, s);
+    if (st != AC_OK) return st;
+    if (times) CK(cudaEventRecord(c->ev[2], s), "event");
+    if ((st = key_stats_impl(c, Kb, s)) != AC_OK) return st;
+    if (times) CK(cudaEventRecord(c->ev[3], s), "event");
+    if ((st = score_select_impl(c, 0, s)) != AC_OK) return st;
+    if (times) CK(cudaEventRecord(c->ev[4], s), "event");
+    if ((st = sparse_attn_impl(c, Qb, Kb, Vb, reinterpret_cast<bf16 *>(O), s)) != AC_OK) return st;
+    if (times) CK(cudaEventRecord(c->ev[5], s), "event");
+    c->have_state = true;
+    if (times) {
+        CK(cudaEventSynchronize(c->ev[5]), "event sync");
+        float ms[5];
+        for (int i = 0; i < 5; ++i) CK(cudaEventElapsedTime(&ms[i], c->ev[i], c->ev[i + 1]), "elapsed");
+        times->q_cluster_ms = ms[0];
+        times->k_cluster_ms = ms[1];
+        times->stats_sort_ms = ms[2];
+        times->score_select_ms = ms[3];
+        times->attention_ms = ms[4];
+        CK(cudaEventElapsedTime(&times->total_ms, c->ev[0], c->ev[5]), "elapsed");
+        return check_dev_err(c, s);
+    }
+    return AC_OK;
+}
+
+ac_status ac_layer_forward_host(ac_ctx *c, const uint16_t *hQ, const uint16_t *hK, const uint16_t *hV,
+                                uint16_t *hO, int32_t warm, void *stream) {
+    if (!c || !hQ || !hK || !hV || !hO) return fail(c, AC_ERR_INVALID_ARG, "ac_layer_forward_host: NULL argument");
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t n = (size_t)c->BH * c->L * c->d;
+    if (!c->hbufQ) {
+        if (dalloc(&c->hbufQ, n) != cudaSuccess || dalloc(&c->hbufK, n) != cudaSuccess ||
+            dalloc(&c->hbufV, n) != cudaSuccess || dalloc(&c->hbufO, n) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(c, AC_ERR_WORKSPACE, "host-buffer staging allocation failed");
+        }
+    }
+    CK(cudaMemcpyAsync(c->hbufQ, hQ, n * 2, cudaMemcpyHostToDevice, s), "h2d Q");
+    CK(cudaMemcpyAsync(c->hbufK, hK, n * 2, cudaMemcpyHostToDevice, s), "h2d K");
+    CK(cudaMemcpyAsync(c->hbufV, hV, n * 2, cudaMemcpyHostToDevice, s), "h2d V");
+    ac_status st = ac_layer_forward(c, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, warm, nullptr, stream);
+    if (st != AC_OK) return st;
+    CK(cudaMemcpyAsync(hO, c->hbufO, n * 2, cudaMemcpyDeviceToHost, s), "d2h O");
+    return check_dev_err(c, s);
+}
+
+ac_status ac_get_tensor(ac_ctx *c, int32_t which, void **ptr, int64_t shape[4]) {
+    if (!c || !ptr || !shape) return AC_ERR_INVALID_ARG;
+    const int64_t BH = c->BH, L = c->L, d = c->d, Cq = c->Cq, Cc = c->Ccap;
+    int64_t s0 = 1, s1 = 1, s2 = 1;
+    void *p = nullptr;
+    switch (which) {
+        case AC_T_INV_NORM_Q: p = c->inv_q; s0 = BH; s1 = L; break;
+        case AC_T_LABELS_Q: p = c->labels_q; s0 = BH; s1 = L; break;
+        case AC_T_CENT_Q: p = c->cent_q; s0 = BH; s1 = Cq; s2 = d; break;
+        case AC_T_COUNTS_Q: p = c->counts_q; s0 = BH; s1 = Cq; break;
+        case AC_T_PERM_Q: p = c->perm_q; s0 = BH; s1 = L; break;
+        case AC_T_OFFS_Q: p = c->offs_q; s0 = BH; s1 = Cq + 1; break;
+        case AC_T_LABELS_K: p = c->labels_k; s0 = BH; s1 = L; break;
+        case AC_T_DMIN_K: p = c->dmin_k; s0 = BH; s1 = L; break;
+        case AC_T_CENT_K: p = c->cent_k; s0 = BH; s1 = Cc; s2 = d; break;
+        case AC_T_N_K: p = c->n_k; s0 = BH; break;
+        case AC_T_DENSE: p = c->dense; s0 = BH; break;
+        case AC_T_COUNTS_K: p = c->counts_k; s0 = BH; s1 = Cc; break;
+        case AC_T_KMAX: p = c->kmax; s0 = BH; s1 = Cc; s2 = d; break;
+        case AC_T_KMIN: p = c->kmin; s0 = BH; s1 = Cc; s2 = d; break;
+        case AC_T_SSE: p = c->sse; s0 = BH; s1 = Cc; break;
+        case AC_T_COMP: p = c->comp; s0 = BH; break;
+        case AC_T_PERM_K: p = c->perm_k; s0 = BH; s1 = L; break;
+        case AC_T_OFFS_K: p = c->offs_k; s0 = BH; s1 = Cc + 1; break;
+        case AC_T_SCORE: p = c->score; s0 = BH; s1 = Cq; s2 = Cc; break;
+        case AC_T_SEL: p = c->sel; s0 = BH; s1 = Cq; s2 = Cc; break;
+        case AC_T_KSEL: p = c->ksel; s0 = BH; break;
+        case AC_T_TAU: p = c->tau; s0 = 1; break;
+        case AC_T_STAGES: p = c->stages; s0 = BH; break;
+        case AC_T_REMOVED_STAGE: p = c->removed_stage; s0 = BH; s1 = L; break;
+        case AC_T_MSE: p = c->mse; s0 = BH; break;
+        default: return fail(c, AC_ERR_INVALID_ARG, "unknown tensor id");
+    }
+    *ptr = p;
+    shape[0] = s0;
+    shape[1] = s1;
+    shape[2] = s2;
+    shape[3] = 1;
+    return AC_OK;
+}
+
+ac_status ac_synchronize(ac_ctx *c, void *stream) {
+    if (!c) return AC_ERR_INVALID_ARG;
+    return check_dev_err(c, (cudaStream_t)stream);
+}
+
+ac_status ac_get_attn_counters(ac_ctx *c, ac_attn_counters *out) {
+    if (!c || !out) return AC_ERR_INVALID_ARG;
+    unsigned long long h[4];
+    CK(cudaDeviceSynchronize(), "sync");
+    CK(cudaMemcpy(h, c->counters, sizeof(h), cudaMemcpyDeviceToHost), "counters");
+    std::vector<uint8_t> dn(c->BH);
+    CK(cudaMemcpy(dn.data(), c->dense, c->BH, cudaMemcpyDeviceToHost), "dense");
+    out->kept_pairs = (int64_t)h[0];
+    out->computed_pairs = (int64_t)h[1];
+    out->tiles = (int64_t)h[2];
+    out->dense_heads = 0;
+    for (uint8_t v : dn) out->dense_heads += v ? 1 : 0;
+    return AC_OK;
+}
+
+// State layout: magic, B, H, L, d, Cq, Ccap, then cent_q, cent_k, n_k, dense,
+// labels_k, dmin_k.
+ac_status ac_state_export(ac_ctx *c, void *host_buf, int64_t *bytes) {
+    if (!c || !bytes) return AC_ERR_INVALID_ARG;
+    const size_t BH = c->BH;
+    const size_t sz_q = BH * c->Cq * c->d * 4, sz_k = BH * c->Ccap * c->d * 4, sz_n = BH * 4, sz_f = BH,
+                 sz_l = BH * c->L * 4;
+    const size_t total = 8 * 8 + sz_q + sz_k + sz_n + sz_f + 2 * sz_l;
+    if (!host_buf) {
+        *bytes = (int64_t)total;
+        return AC_OK;
+    }
+    if (*bytes < (int64_t)total) return fail(c, AC_ERR_INVALID_ARG, "state buffer too small");
+    if (!c->have_state) return fail(c, AC_ERR_STATE, "no state to export");
+    CK(cudaDeviceSynchronize(), "sync");
+    int64_t *hd = reinterpret_cast<int64_t *>(host_buf);
+    hd[0] = 0x41435354415445LL;
+    hd[1] = c->B;
+    hd[2] = c->H;
+    hd[3] = c->L;
+    hd[4] = c->d;
+    hd[5] = c->Cq;
+    hd[6] = c->Ccap;
+    hd[7] = 0;
+    uint8_t *p = reinterpret_cast<uint8_t *>(host_buf) + 64;
+    CK(cudaMemcpy(p, c->cent_q, sz_q, cudaMemcpyDeviceToHost), "export");
+    p += sz_q;
+    CK(cudaMemcpy(p, c->cent_k, sz_k, cudaMemcpyDeviceToHost), "export");
+    p += sz_k;
+    CK(cudaMemcpy(p, c->n_k, sz_n, cudaMemcpyDeviceToHost), "export");
+    p += sz_n;
+    CK(cudaMemcpy(p, c->dense, sz_f, cudaMemcpyDeviceToHost), "export");
+    p += sz_f;
+    CK(cudaMemcpy(p, c->labels_k, sz_l, cudaMemcpyDeviceToHost), "export");
+    p += sz_l;
+    CK(cudaMemcpy(p, c->dmin_k, sz_l, cudaMemcpyDeviceToHost), "export");
+    *bytes = (int64_t)total;
+    return AC_OK;
+}
+
+ac_status ac_state_import(ac_ctx *c, const void *host_buf, int64_t bytes) {
+    if (!c || !host_buf) return AC_ERR_INVALID_ARG;
+    int64_t need = 0;
+    ac_state_export(c, nullptr, &need);
+    if (bytes < need) return fail(c, AC_ERR_INVALID_ARG, "state buffer too small");
+    const int64_t *hd = reinterpret_cast<const int64_t *>(host_buf);
+    if (hd[0] != 0x41435354415445LL || hd[1] != c->B || hd[2] != c->H || hd[3] != c->L || hd[4] != c->d ||
+        hd[5] != c->Cq || hd[6] != c->Ccap)
+        return fail(c, AC_ERR_INVALID_ARG, "state does not match this context");
+    const size_t BH = c->BH;
+    const size_t sz_q = BH * c->Cq * c->d * 4, sz_k = BH * c->Ccap * c->d * 4, sz_n = BH * 4, sz_f = BH,
+                 sz_l = BH * c->L * 4;
+    CK(cudaDeviceSynchronize(), "sync");
+    const uint8_t *p = reinterpret_cast<const uint8_t *>(host_buf) + 64;
+    CK(cudaMemcpy(c->cent_q, p, sz_q, cudaMemcpyHostToDevice), "import");
+    p += sz_q;
+    CK(cudaMemcpy(c->cent_k, p, sz_k, cudaMemcpyHostToDevice), "import");
+    p += sz_k;
+    CK(cudaMemcpy(c->n_k, p, sz_n, cudaMemcpyHostToDevice), "import");
+    p += sz_n;
+    CK(cudaMemcpy(c->dense, p, sz_f, cudaMemcpyHostToDevice), "import");
+    p += sz_f;
+    CK(cudaMemcpy(c->labels_k, p, sz_l, cudaMemcpyHostToDevice), "import");
+    p += sz_l;
+    CK(cudaMemcpy(c->dmin_k, p, sz_l, cudaMemcpyHostToDevice), "import");
+    c->have_state = true;
+    c->have_q = true;
+    c->have_k = true;
+    return AC_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,197 @@
+// ac_internal.h -- context layout and kernel launchers of libac (host side).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "ac.h"
+
+typedef __nv_bfloat16 bf16;
+
+struct ac_ctx {
+    ac_config cfg;
+    int B, H, L, d, BH, Cq, Ccap;
+    int device;
+    float scale;
+
+    // ---- query clustering (Algorithm 3 line 3)
+    float *inv_q;      // [BH, L]
+    int *labels_q;     // [BH, L]
+    float *cent_q;     // [BH, Cq, d]
+    int *counts_q;     // [BH, Cq]
+    int *perm_q;       // [BH, L]
+    int *offs_q;       // [BH, Cq+1]
+
+    // ---- key clustering (Algorithm 1)
+    int *labels_k;     // [BH, L]
+    float *dmin_k;     // [BH, L]
+    float *cent_k;     // [BH, Ccap, d]
+    int *n_k;          // [BH]
+    uint8_t *dense;    // [BH]
+    int *stages;       // [BH]
+    int *removed_stage;  // [BH, L]
+    float *tau;        // [1]
+    unsigned long long *tau_acc;  // [1] fixed-point sum of stage-0 distances
+    int *counts_k;     // [BH, Ccap]
+    int *perm_k;       // [BH, L]
+    int *offs_k;       // [BH, Ccap+1]
+    bf16 *kmax, *kmin; // [BH, Ccap, d]
+    float *sse;        // [BH, Ccap]
+    float *mse, *comp; // [BH]
+
+    // ---- multi-stage scratch
+    int *u_idx;        // [BH, L]  unabsorbed keys, ascending
+    int *u_idx2;       // [BH, L]
+    int *u_cnt;        // [BH]
+    int *st_m;         // [BH]     clusters of the current stage (0: idle head)
+    int *st_labels;    // [BH, L]
+    float *st_dist;    // [BH, L]
+    int *st_perm;      // [BH, L]
+    int *st_offs;      // [BH, m0+1]
+    int *st_counts;    // [BH, m0]
+    uint32_t *radix;   // [256 + 4] percentile selection scratch
+
+    // ---- selection (Algorithm 3 line 9)
+    float *score;      // [BH, Cq, Ccap]
+    int *sel;          // [BH, Cq, Ccap]
+    int *ksel;         // [BH]
+    int2 *ranges;      // [BH, Cq, Ccap]  (start row in cluster order, count)
+    int *nboxes;       // [BH*Cq]         8-row key boxes per query cluster
+    int *tile_prefix;  // [BH*Cq+1]       128-query tiles, exclusive prefix
+
+    // ---- attention
+    bf16 *Qp, *Kp, *Vp;  // [BH, L, d] cluster-order copies
+    unsigned long long *counters;  // [4] kept pairs, computed pairs, tiles, dense heads
+    CUtensorMap tm_q, tm_k, tm_v;
+
+    // ---- host-buffer forward
+    uint16_t *hbufQ, *hbufK, *hbufV, *hbufO;  // device staging of the host entry point
+
+    uint32_t *err;      // device error word
+    int *h_u_cnt;       // pinned host mirrors
+    int *h_st_m;
+    int *h_n_k;
+    uint8_t *h_dense;
+    uint32_t *h_err;
+
+    bool have_q, have_k, have_state;
+    std::string msg;
+    cudaEvent_t ev[8];
+};
+
+// ---------------------------------------------------------------- launchers
+// All launchers enqueue on `s` and return the launch status.
+namespace ac {
+
+cudaError_t launch_qnorm(const bf16 *Q, float *inv, int64_t rows, int d, uint32_t *err, cudaStream_t s);
+
+// Exact assignment: for every row of every unit h (rows given by an index
+// list or 0..n-1), label = argmin over the unit's centres of the fp32
+// squared distance summed in dimension order; ties to the lowest index.
+struct AssignArgs {
+    const bf16 *X;        // [BH, L, d]
+    const float *inv;     // [BH, L] or null (then rows are not normalised)
+    int64_t L;
+    const int *rows;      // [BH, L] row indices or null
+    const int *nrows;     // [BH] or null (then nrows_const)
+    int nrows_const;
+    const float *C;       // [BH, cstride] centres
+    int64_t cstride;      // floats per unit
+    const int *coff;      // [BH] first centre of the unit (in centres) or null
+    const int *ncent;     // [BH] or null (then ncent_const)
+    int ncent_const;
+    int *labels;          // [BH, L]
+    float *dmin;          // [BH, L] or null
+    int BH, d;
+};
+cudaError_t launch_assign_exact(const AssignArgs &a, cudaStream_t s);
+
+// Stable counting sort of labels per unit: perm[h, pos] = row position (or
+// rows[pos]'s index when rows given, see below), offs[h, 0..m], counts[h, 0..m).
+struct SortArgs {
+    const int *labels;    // [BH, L]
+    int64_t L;
+    const int *nrows;     // [BH] or null
+    int nrows_const;
+    const int *nlab;      // [BH] or null
+    int nlab_const;
+    int max_lab;          // upper bound of nlab over units
+    int *perm;            // [BH, L]
+    int *offs;            // [BH, offs_stride]
+    int offs_stride;
+    int *counts;          // [BH, counts_stride] or null
+    int counts_stride;
+    int BH;
+};
+cudaError_t launch_counting_sort(const SortArgs &a, cudaStream_t s);
+
+// Centre update: C[h, coff+c] = mean of the members of cluster c, summed in
+// ascending order; empty clusters keep their centre.
+struct UpdateArgs {
+    const bf16 *X; const float *inv; int64_t L;
+    const int *rows;      // [BH, L] or null
+    const int *perm; const int *offs; int offs_stride;
+    float *C; int64_t cstride; const int *coff;
+    const int *ncent; int ncent_const;
+    int BH, d, max_cent;
+};
+cudaError_t launch_update(const UpdateArgs &a, cudaStream_t s);
+
+// Seeded initial centres: C[h, coff + j] = X[rows[h, pick_j]] (normalised
+// when inv is given), j < m[h], pick_j from stratum j of n[h] members.
+struct SeedArgs {
+    const bf16 *X; const float *inv; int64_t L;
+    const int *rows; const int *nrows; int nrows_const;
+    float *C; int64_t cstride; const int *coff;
+    const int *m; int m_const; int max_m;
+    uint64_t seed; int tag; int BH, d;
+};
+cudaError_t launch_seed(const SeedArgs &a, cudaStream_t s);
+
+// Multi-stage helpers.
+cudaError_t launch_iota_rows(int *u_idx, int *u_cnt, int BH, int L, cudaStream_t s);
+cudaError_t launch_stage_dist(const float *dmin, float *dist, const int *u_cnt, const int *st_m,
+                              int64_t L, int BH, unsigned long long *tau_acc, cudaStream_t s);
+cudaError_t launch_tau_mean(const unsigned long long *tau_acc, const int *u_cnt0_total_unused,
+                            int64_t n_total, float factor, float *tau, cudaStream_t s);
+cudaError_t launch_tau_percentile(const float *dist, const int *st_m, int64_t L, int BH,
+                                  int64_t n_total, int permille, uint32_t *radix, float *tau,
+                                  cudaStream_t s);
+cudaError_t launch_remove(const float *dist, const float *tau, int *u_idx, int *u_idx2, int *u_cnt,
+                          const int *st_m, int *removed_stage, int stage, int64_t L, int BH,
+                          cudaStream_t s);
+
+struct StatsArgs {
+    const bf16 *K; int64_t L; const int *perm; const int *offs; int offs_stride;
+    const float *dmin; const int *n_k; int Ccap; int d; int BH;
+    int *counts; bf16 *kmax; bf16 *kmin; float *sse; float *mse; float *comp;
+};
+cudaError_t launch_key_stats(const StatsArgs &a, cudaStream_t s);
+
+cudaError_t launch_permute_rows(const bf16 *X, const int *perm, bf16 *Xp, int64_t L, int d, int BH,
+                                cudaStream_t s);
+
+struct SelectArgs {
+    const float *cent_q; const bf16 *kmax; const bf16 *kmin; const int *counts_k;
+    const int *n_k; const uint8_t *dense; const int *offs_k; const int *counts_q;
+    int Cq, Ccap, d, BH, L, topk;
+    float *score; int *sel; int *ksel; int2 *ranges; int *nboxes; int *tile_prefix;
+};
+cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s);
+
+struct AttnArgs {
+    const CUtensorMap *tm_q, *tm_k, *tm_v;
+    bf16 *O; const int *perm_q; const int *offs_q; const int *counts_q;
+    const int *tile_prefix; const int2 *ranges; const int *nboxes; const int *ksel;
+    const uint8_t *dense; int L, Cq, Ccap, BH, d;
+    float scale_log2;
+    uint32_t *err; unsigned long long *counters;
+};
+cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s);
+int attn_max_tiles(int L, int Cq, int BH);
+
+}  // namespace ac

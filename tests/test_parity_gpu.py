@@ -1,0 +1,183 @@
+"""GPU parity: the CUDA layer (through the C ABI) against the CPU oracle.
+
+Labels, permutations, stage bookkeeping and selections are compared
+bit-exactly, centres within fp32 relative 1e-4, and the attention output
+within max abs 2e-2 / relative L2 5e-3 of the fp64 oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from _gpu_common import (assert_attention, compare_layer, dev, gpu_state, heavy_tail_layer, host_f32,
+                         make_layer_ctx, run_gpu_layer)
+from oracle import oracle as orc
+from cluster_routed_sparse_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _params(cfg, seed=1234, **kw):
+    p = orc.Params.from_layer_config(cfg, seed=seed)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def _flat(x):
+    B, H, L, d = x.shape
+    return x.reshape(B * H, L, d)
+
+
+def test_tiny_layer_step0_end_to_end():
+    cfg = synth.CONFIGS[1]
+    Q, K, V = synth.make_layer(cfg)
+    p = _params(cfg)
+    r = orc.layer(_flat(Q), _flat(K), _flat(V), p)
+    lay, O, gs = run_gpu_layer(Q, K, V, p)
+    compare_layer(gs, r, p, O)
+    lay.close()
+
+
+def test_tiny_layer_warm_chain():
+    """Step 0 then two warm-started steps on perturbed tokens (Sec. 3.2.2)."""
+    cfg = synth.CONFIGS[1]
+    p = _params(cfg)
+    lay = None
+    prev = None
+    for step in range(3):
+        Q, K, V = synth.make_layer(cfg, step=step)
+        r = orc.layer(_flat(Q), _flat(K), _flat(V), p, warm_from=prev)
+        lay, O, gs = run_gpu_layer(Q, K, V, p, lay=lay, warm=step > 0)
+        compare_layer(gs, r, p, O, check_step0=step == 0)
+        prev = r
+    lay.close()
+
+
+@pytest.mark.parametrize("shape,kw", [
+    ((1, 2, 1000, 64), dict(Cq=7, m0=10, n_max=40, tau_mode=1, tau_value=1.0, topk=-300)),
+    ((1, 2, 2048, 128), dict(Cq=16, m0=16, n_max=64, tau_mode=2, tau_value=900.0, topk=4)),
+    ((2, 2, 1500, 64), dict(Cq=9, m0=12, n_max=48, tau_mode=1, tau_value=1.5, topk=-100)),
+    ((1, 1, 333, 128), dict(Cq=3, m0=5, n_max=20, tau_mode=1, tau_value=1.2, topk=2)),
+])
+def test_ragged_shapes(shape, kw):
+    B, H, Lq, d = shape
+    cfg = synth.LayerConfig("ragged", B, H, Lq, d, key_components=30, iters_q=4, iters_k=4, **kw)
+    Q, K, V = synth.make_layer(cfg)
+    p = _params(cfg, seed=99)
+    r = orc.layer(_flat(Q), _flat(K), _flat(V), p)
+    lay, O, gs = run_gpu_layer(Q, K, V, p)
+    compare_layer(gs, r, p, O)
+    lay.close()
+
+
+def test_heavy_tailed_clusters():
+    """Dirichlet(0.3) component weights: many clusters under 8 keys, so most
+    key boxes are partly masked."""
+    cfg = heavy_tail_layer()
+    Q, K, V = synth.make_layer(cfg)
+    p = _params(cfg, seed=7)
+    r = orc.layer(_flat(Q), _flat(K), _flat(V), p)
+    lay, O, gs = run_gpu_layer(Q, K, V, p)
+    compare_layer(gs, r, p, O)
+    assert (r.st.counts[:, :int(r.kc.n_k.min())] < 8).sum() > 0
+    lay.close()
+
+
+def test_dense_fallback_heads():
+    """tau = 0 absorbs nothing: every head reaches N_max and attends densely
+    (Algorithm 1 lines 7-9, Algorithm 3 line 6)."""
+    cfg = synth.LayerConfig("dense", 1, 2, 1200, 64, Cq=5, m0=8, n_max=20, tau_mode=0, tau_value=0.0,
+                            topk=2, key_components=20, iters_q=3, iters_k=2)
+    Q, K, V = synth.make_layer(cfg)
+    p = _params(cfg)
+    r = orc.layer(_flat(Q), _flat(K), _flat(V), p)
+    assert r.kc.F.all()
+    lay, O, gs = run_gpu_layer(Q, K, V, p)
+    compare_layer(gs, r, p, O)
+    lay.close()
+
+
+def test_all_clusters_selected_is_dense_attention():
+    cfg = synth.LayerConfig("allsel", 1, 2, 1536, 128, Cq=6, m0=12, n_max=40, tau_mode=1,
+                            tau_value=1.0, topk=10000, key_components=25, iters_q=3, iters_k=3)
+    Q, K, V = synth.make_layer(cfg)
+    p = _params(cfg)
+    lay, O, gs = run_gpu_layer(Q, K, V, p)
+    for h in range(2):
+        ref = orc.attention_rows(Q[0, h], K[0, h], V[0, h], gs["labels_q"][h], gs["labels_k"][h],
+                                 None, True, np.arange(cfg.L))
+        assert_attention(O[h], ref, f"head {h}")
+    lay.close()
+
+
+@pytest.mark.parametrize("Lq", [1, 5, 9])
+def test_tiny_sequences(Lq):
+    cfg = synth.LayerConfig("tiny", 1, 1, Lq, 64, Cq=min(2, Lq), m0=min(3, Lq), n_max=4, tau_mode=1,
+                            tau_value=1.0, topk=1, key_components=2, iters_q=2, iters_k=2)
+    Q, K, V = synth.make_layer(cfg)
+    p = _params(cfg)
+    r = orc.layer(_flat(Q), _flat(K), _flat(V), p)
+    lay, O, gs = run_gpu_layer(Q, K, V, p)
+    compare_layer(gs, r, p, O)
+    lay.close()
+
+
+def test_host_entry_point_matches_device_forward():
+    cfg = synth.CONFIGS[1]
+    Q, K, V = synth.make_layer(cfg)
+    p = _params(cfg)
+    lay, O, _ = run_gpu_layer(Q, K, V, p)
+    lay2 = make_layer_ctx(p, *Q.shape)
+    hQ, hK, hV = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (Q, K, V))
+    hO = torch.empty_like(hQ).pin_memory()
+    lay2.forward_host(hQ, hK, hV, hO)
+    assert np.array_equal(hO.view(torch.int16).numpy().reshape(O.shape),
+                          torch.from_numpy(O).to(torch.bfloat16).view(torch.int16).numpy())
+    lay.close()
+    lay2.close()
+
+
+def test_state_resume_is_bit_exact():
+    """Checkpoint/resume across denoising steps: exporting the warm-start state
+    after step 0 and importing it into a fresh context gives the same warm step."""
+    cfg = synth.CONFIGS[1]
+    p = _params(cfg)
+    Q0, K0, V0 = synth.make_layer(cfg, step=0)
+    Q1, K1, V1 = synth.make_layer(cfg, step=1)
+    a, _, _ = run_gpu_layer(Q0, K0, V0, p)
+    blob = a.export_state()
+    _, Oa, ga = run_gpu_layer(Q1, K1, V1, p, lay=a, warm=True)
+    b = make_layer_ctx(p, *Q0.shape)
+    b.import_state(blob)
+    _, Ob, gb = run_gpu_layer(Q1, K1, V1, p, lay=b, warm=True)
+    assert np.array_equal(Oa, Ob)
+    for key in ("labels_q", "labels_k", "cent_q", "cent_k", "sel"):
+        assert np.array_equal(ga[key], gb[key]), key
+    a.close()
+    b.close()
+
+
+def test_warm_step_before_step0_is_a_state_error():
+    cfg = synth.CONFIGS[1]
+    p = _params(cfg)
+    lay = make_layer_ctx(p, 1, 2, cfg.L, cfg.d)
+    Q, K, V = (dev(x) for x in synth.make_layer(cfg))
+    from cluster_routed_sparse_b200._lib import ACError, AC_ERR_STATE
+    with pytest.raises(ACError) as e:
+        lay.forward(Q, K, V, warm=True)
+    assert e.value.status == AC_ERR_STATE
+    lay.close()
+
+
+def test_nonfinite_input_is_reported():
+    cfg = synth.CONFIGS[1]
+    p = _params(cfg)
+    Q, K, V = synth.make_layer(cfg)
+    Q = Q.copy()
+    Q[0, 0, 17, 3] = 0x7FC0  # bf16 NaN
+    lay = make_layer_ctx(p, *Q.shape)
+    from cluster_routed_sparse_b200._lib import ACError, AC_ERR_NONFINITE
+    with pytest.raises(ACError) as e:
+        lay.cluster_q(dev(Q))
+    assert e.value.status == AC_ERR_NONFINITE
+    lay.close()
