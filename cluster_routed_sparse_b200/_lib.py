@@ -35,6 +35,16 @@ TENSOR_TYPES = {
 }
 
 
+# rank of each tensor id (ac_get_tensor reports unused trailing extents as 1)
+TENSOR_RANKS = {
+    AC_T_INV_NORM_Q: 2, AC_T_LABELS_Q: 2, AC_T_CENT_Q: 3, AC_T_COUNTS_Q: 2, AC_T_PERM_Q: 2,
+    AC_T_OFFS_Q: 2, AC_T_LABELS_K: 2, AC_T_DMIN_K: 2, AC_T_CENT_K: 3, AC_T_N_K: 1, AC_T_DENSE: 1,
+    AC_T_COUNTS_K: 2, AC_T_KMAX: 3, AC_T_KMIN: 3, AC_T_SSE: 2, AC_T_COMP: 1, AC_T_PERM_K: 2,
+    AC_T_OFFS_K: 2, AC_T_SCORE: 3, AC_T_SEL: 3, AC_T_KSEL: 1, AC_T_TAU: 1, AC_T_STAGES: 1,
+    AC_T_REMOVED_STAGE: 2, AC_T_MSE: 1,
+}
+
+
 class ACConfig(ctypes.Structure):
     _fields_ = [("Cq", ctypes.c_int32), ("m0", ctypes.c_int32), ("n_max", ctypes.c_int32),
                 ("tau_mode", ctypes.c_int32), ("tau_value", ctypes.c_float), ("topk", ctypes.c_int32),
@@ -46,7 +56,8 @@ class ACConfig(ctypes.Structure):
 class ACStageTimes(ctypes.Structure):
     _fields_ = [("q_cluster_ms", ctypes.c_float), ("k_cluster_ms", ctypes.c_float),
                 ("stats_sort_ms", ctypes.c_float), ("score_select_ms", ctypes.c_float),
-                ("attention_ms", ctypes.c_float), ("total_ms", ctypes.c_float)]
+                ("attention_ms", ctypes.c_float), ("attn_kernel_ms", ctypes.c_float),
+                ("total_ms", ctypes.c_float)]
 
     def as_dict(self):
         return {f: float(getattr(self, f)) for f, _ in self._fields_}
@@ -73,6 +84,7 @@ SIGNATURES = {
     "ac_synchronize": (_I, [_P, _P]),
     "ac_get_tensor": (_I, [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int64)]),
     "ac_get_attn_counters": (_I, [_P, ctypes.POINTER(ACAttnCounters)]),
+    "ac_get_launch_count": (_I, [ctypes.POINTER(ctypes.c_int64)]),
     "ac_state_export": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int64)]),
     "ac_state_import": (_I, [_P, _P, ctypes.c_int64]),
 }

@@ -110,13 +110,17 @@ class SparseLayer:
         shape = (ctypes.c_int64 * 4)()
         check(self.lib.ac_get_tensor(self.ctx, which, ctypes.byref(p), shape), self.ctx)
         typ = _lib.TENSOR_TYPES[which]
-        dims = [int(x) for x in shape[:4]]
-        while len(dims) > 1 and dims[-1] == 1:
-            dims.pop()
+        dims = [int(x) for x in shape[:_lib.TENSOR_RANKS[which]]]
         t = torch.as_tensor(_CudaArray(p.value, dims, typ), device="cuda")
         if which in (_lib.AC_T_KMAX, _lib.AC_T_KMIN):
             t = t.view(torch.bfloat16)
         return t
+
+    def launch_count(self) -> int:
+        """Kernels libac has launched in this process so far."""
+        n = ctypes.c_int64(0)
+        check(self.lib.ac_get_launch_count(ctypes.byref(n)), self.ctx)
+        return int(n.value)
 
     def counters(self) -> dict:
         c = ACAttnCounters()

@@ -16,6 +16,8 @@
 
 using namespace ac;
 
+std::atomic<long long> ac::g_launches{0};
+
 namespace {
 
 const char *g_static_msg = "";
@@ -245,6 +247,7 @@ ac_status cluster_k_warm(ac_ctx *c, const bf16 *K, cudaStream_t s) {
     const int BH = c->BH, L = c->L, d = c->d;
     const int64_t cstride = (int64_t)c->Ccap * d;
     k_warm_counts<<<(BH + 127) / 128, 128, 0, s>>>(c->n_k, c->dense, c->st_m, BH);
+    AC_NOTE_LAUNCH();
     CK(cudaGetLastError(), "warm counts");
     Lloyd k;
     k.as = AssignArgs{K, nullptr, L, nullptr, nullptr, L, c->cent_k, cstride, nullptr, c->st_m, 0, c->labels_k,
@@ -285,7 +288,9 @@ ac_status sparse_attn_impl(ac_ctx *c, const bf16 *Q, const bf16 *K, const bf16 *
     AttnArgs a{&c->tm_q, &c->tm_k, &c->tm_v, O, c->perm_q, c->offs_q, c->counts_q, c->tile_prefix, c->ranges,
                c->nboxes, c->ksel, c->dense, c->L, c->Cq, c->Ccap, c->BH, c->d,
                (float)(c->scale * 1.4426950408889634), c->err, c->counters};
+    if (c->timing) CK(cudaEventRecord(c->ev[6], s), "event");
     CK(launch_sparse_attn(a, s), "sparse attention");
+    if (c->timing) CK(cudaEventRecord(c->ev[7], s), "event");
     return AC_OK;
 }
 
@@ -515,6 +520,7 @@ ac_status ac_layer_forward(ac_ctx *c, const uint16_t *Q, const uint16_t *K, cons
     const bf16 *Qb = reinterpret_cast<const bf16 *>(Q), *Kb = reinterpret_cast<const bf16 *>(K),
                *Vb = reinterpret_cast<const bf16 *>(V);
     ac_status st;
+    c->timing = times != nullptr;
     if (times) CK(cudaEventRecord(c->ev[0], s), "event");
     st = cluster_q_impl(c, Qb, warm ? c->cent_q : nullptr, warm ? c->cfg.iters_warm : c->cfg.iters_q, s);
     if (st != AC_OK) return st;
@@ -538,7 +544,9 @@ ac_status ac_layer_forward(ac_ctx *c, const uint16_t *Q, const uint16_t *K, cons
         times->stats_sort_ms = ms[2];
         times->score_select_ms = ms[3];
         times->attention_ms = ms[4];
+        CK(cudaEventElapsedTime(&times->attn_kernel_ms, c->ev[6], c->ev[7]), "elapsed");
         CK(cudaEventElapsedTime(&times->total_ms, c->ev[0], c->ev[5]), "elapsed");
+        c->timing = false;
         return check_dev_err(c, s);
     }
     return AC_OK;
@@ -603,6 +611,12 @@ ac_status ac_get_tensor(ac_ctx *c, int32_t which, void **ptr, int64_t shape[4]) 
     shape[1] = s1;
     shape[2] = s2;
     shape[3] = 1;
+    return AC_OK;
+}
+
+ac_status ac_get_launch_count(int64_t *out) {
+    if (!out) return AC_ERR_INVALID_ARG;
+    *out = (int64_t)g_launches.load(std::memory_order_relaxed);
     return AC_OK;
 }
 

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <string>
 
 #include "ac.h"
@@ -79,6 +80,7 @@ struct ac_ctx {
     uint32_t *h_err;
 
     bool have_q, have_k, have_state;
+    bool timing;        // record events around the attention kernel
     std::string msg;
     cudaEvent_t ev[8];
 };
@@ -86,6 +88,10 @@ struct ac_ctx {
 // ---------------------------------------------------------------- launchers
 // All launchers enqueue on `s` and return the launch status.
 namespace ac {
+
+// Kernels launched by this library in this process.
+extern std::atomic<long long> g_launches;
+#define AC_NOTE_LAUNCH() ::ac::g_launches.fetch_add(1, std::memory_order_relaxed)
 
 cudaError_t launch_qnorm(const bf16 *Q, float *inv, int64_t rows, int d, uint32_t *err, cudaStream_t s);
 

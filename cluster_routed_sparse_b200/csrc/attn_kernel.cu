@@ -411,11 +411,13 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s) {
                                  (int)Layout<128>::SMEM);
         if (e != cudaSuccess) return e;
         k_sparse_attn<128><<<grid, NTHREADS, Layout<128>::SMEM, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, p);
+        AC_NOTE_LAUNCH();
     } else {
         e = cudaFuncSetAttribute(k_sparse_attn<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)Layout<64>::SMEM);
         if (e != cudaSuccess) return e;
         k_sparse_attn<64><<<grid, NTHREADS, Layout<64>::SMEM, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, p);
+        AC_NOTE_LAUNCH();
     }
     return cudaGetLastError();
 }

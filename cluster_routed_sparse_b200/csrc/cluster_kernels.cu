@@ -39,6 +39,7 @@ __global__ void k_qnorm(const bf16 *__restrict__ Q, float *__restrict__ inv, int
 
 cudaError_t launch_qnorm(const bf16 *Q, float *inv, int64_t rows, int d, uint32_t *err, cudaStream_t s) {
     k_qnorm<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(Q, inv, rows, d, err);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 
@@ -128,6 +129,7 @@ cudaError_t launch_assign_exact(const AssignArgs &a, cudaStream_t s) {
         if (norm) k_assign_exact<64, true><<<grid, 128, 0, s>>>(a);
         else k_assign_exact<64, false><<<grid, 128, 0, s>>>(a);
     }
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 
@@ -205,6 +207,7 @@ cudaError_t launch_counting_sort(const SortArgs &a, cudaStream_t s) {
                                          (int)(smem < 48 * 1024 ? 48 * 1024 : smem));
     if (e != cudaSuccess) return e;
     k_counting_sort<<<a.BH, SORT_WARPS * 32, smem, s>>>(a);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 
@@ -257,6 +260,7 @@ cudaError_t launch_update(const UpdateArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)a.max_cent, (unsigned)a.BH);
     if (a.inv) k_update<true><<<grid, a.d, 0, s>>>(a);
     else k_update<false><<<grid, a.d, 0, s>>>(a);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 
@@ -284,6 +288,7 @@ cudaError_t launch_seed(const SeedArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)((a.max_m + 7) / 8), (unsigned)a.BH);
     if (grid.x == 0) return cudaSuccess;
     k_seed<<<grid, block, 0, s>>>(a);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 
@@ -297,6 +302,7 @@ __global__ void k_iota_rows(int *u_idx, int *u_cnt, int L) {
 
 cudaError_t launch_iota_rows(int *u_idx, int *u_cnt, int BH, int L, cudaStream_t s) {
     k_iota_rows<<<dim3((L + 255) / 256, BH), 256, 0, s>>>(u_idx, u_cnt, L);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 
@@ -324,6 +330,7 @@ __global__ void k_stage_dist(const float *__restrict__ dmin, float *__restrict__
 cudaError_t launch_stage_dist(const float *dmin, float *dist, const int *u_cnt, const int *st_m,
                               int64_t L, int BH, unsigned long long *tau_acc, cudaStream_t s) {
     k_stage_dist<<<dim3((unsigned)((L + 255) / 256), BH), 256, 0, s>>>(dmin, dist, u_cnt, st_m, L, tau_acc);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 
@@ -336,6 +343,7 @@ __global__ void k_tau_mean(const unsigned long long *acc, int64_t n, float facto
 cudaError_t launch_tau_mean(const unsigned long long *tau_acc, const int *, int64_t n_total, float factor,
                             float *tau, cudaStream_t s) {
     k_tau_mean<<<1, 1, 0, s>>>(tau_acc, n_total, factor, tau);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 
@@ -390,10 +398,13 @@ cudaError_t launch_tau_percentile(const float *dist, const int *st_m, int64_t L,
     if (idx < 0) idx = 0;
     if (idx > n_total - 1) idx = n_total - 1;
     k_radix_init<<<1, 256, 0, s>>>(radix, (uint32_t)idx);
+    AC_NOTE_LAUNCH();
     for (int p = 0; p < 4; ++p) {
         int shift = 24 - 8 * p;
         k_radix_hist<<<dim3(64, BH), 256, 0, s>>>(dist, st_m, L, radix, shift);
+        AC_NOTE_LAUNCH();
         k_radix_pick<<<1, 32, 0, s>>>(radix, shift, tau, p == 3);
+        AC_NOTE_LAUNCH();
     }
     return cudaGetLastError();
 }
@@ -436,6 +447,7 @@ __global__ void __launch_bounds__(1024) k_remove(const float *__restrict__ dist,
 cudaError_t launch_remove(const float *dist, const float *tau, int *u_idx, int *u_idx2, int *u_cnt,
                           const int *st_m, int *removed_stage, int stage, int64_t L, int BH, cudaStream_t s) {
     k_remove<<<BH, 1024, 0, s>>>(dist, tau, u_idx, u_idx2, u_cnt, st_m, removed_stage, stage, L);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 
@@ -494,9 +506,11 @@ __global__ void k_head_comp(StatsArgs a) {
 
 cudaError_t launch_key_stats(const StatsArgs &a, cudaStream_t s) {
     k_key_stats<<<dim3(a.Ccap, a.BH), a.d, 0, s>>>(a);
+    AC_NOTE_LAUNCH();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_head_comp<<<(a.BH + 127) / 128, 128, 0, s>>>(a);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 
@@ -519,6 +533,7 @@ cudaError_t launch_permute_rows(const bf16 *X, const int *perm, bf16 *Xp, int64_
     const int64_t rows = (int64_t)BH * L;
     const int64_t threads = rows * (d / 8);
     k_permute_rows<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(X, perm, Xp, L, d, rows);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 

@@ -136,9 +136,11 @@ cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s) {
                                          (int)(smem < 48 * 1024 ? 48 * 1024 : smem));
     if (e != cudaSuccess) return e;
     k_score_select<<<a.BH * a.Cq, SEL_THREADS, smem, s>>>(a);
+    AC_NOTE_LAUNCH();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_tile_prefix<<<1, 1024, 0, s>>>(a.counts_q, a.BH * a.Cq, a.tile_prefix);
+    AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
 

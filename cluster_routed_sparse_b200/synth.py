@@ -165,3 +165,23 @@ def make_layer(cfg: LayerConfig, step: int = 0, heads=None):
             hh = h + b * cfg.H
             Q[b, i], K[b, i], V[b, i] = make_head(cfg, hh, step)
     return Q, K, V
+
+
+def _make_head_job(args):
+    cfg, head, step = args
+    return head, make_head(cfg, head, step)
+
+
+def make_layer_parallel(cfg: LayerConfig, step: int = 0, procs: int | None = None):
+    """make_layer for B = 1 with heads generated in a spawn-started process pool
+    (bit-identical to make_layer; start it before the parent touches CUDA)."""
+    import multiprocessing as mp
+    import os
+    assert cfg.B == 1
+    procs = procs or min(32, os.cpu_count() or 1)
+    shape = (1, cfg.H, cfg.L, cfg.d)
+    Q, K, V = (np.empty(shape, np.uint16) for _ in range(3))
+    with mp.get_context("spawn").Pool(procs) as pool:
+        for h, (q, k, v) in pool.imap_unordered(_make_head_job, [(cfg, h, step) for h in range(cfg.H)]):
+            Q[0, h], K[0, h], V[0, h] = q, k, v
+    return Q, K, V

@@ -95,6 +95,7 @@ typedef struct ac_stage_times {
     float stats_sort_ms;    /* key stats and cluster-order permutations          */
     float score_select_ms;  /* Quest scores + top-k + key ranges                  */
     float attention_ms;     /* gathers into cluster order + sparse attention      */
+    float attn_kernel_ms;   /* the sparse attention kernel alone                  */
     float total_ms;
 } ac_stage_times;
 
@@ -230,6 +231,9 @@ typedef struct ac_attn_counters {
 } ac_attn_counters;
 
 AC_API ac_status ac_get_attn_counters(ac_ctx *ctx, ac_attn_counters *out);
+
+/* Number of kernels libac has launched in this process so far (all contexts). */
+AC_API ac_status ac_get_launch_count(int64_t *out);
 
 /* Warm-start state (query centres, key centres, cluster counts, dense flags)
  * to and from host memory, for checkpoint / resume across denoising steps.
