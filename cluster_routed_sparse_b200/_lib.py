@@ -49,7 +49,7 @@ class ACConfig(ctypes.Structure):
     _fields_ = [("Cq", ctypes.c_int32), ("m0", ctypes.c_int32), ("n_max", ctypes.c_int32),
                 ("tau_mode", ctypes.c_int32), ("tau_value", ctypes.c_float), ("topk", ctypes.c_int32),
                 ("iters_q", ctypes.c_int32), ("iters_k", ctypes.c_int32), ("iters_warm", ctypes.c_int32),
-                ("reserved0", ctypes.c_int32), ("seed", ctypes.c_uint64), ("scale", ctypes.c_float),
+                ("stage_rule", ctypes.c_int32), ("seed", ctypes.c_uint64), ("scale", ctypes.c_float),
                 ("reserved1", ctypes.c_int32)]
 
 

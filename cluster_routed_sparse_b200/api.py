@@ -48,11 +48,12 @@ class SparseLayer:
 
     def __init__(self, B: int, H: int, L: int, d: int, *, Cq: int, m0: int, n_max: int,
                  tau_mode: int, tau_value: float, topk: int, iters_q: int = 10,
-                 iters_k: int = 10, iters_warm: int = 2, seed: int = 1234, scale: float = 0.0):
+                 iters_k: int = 10, iters_warm: int = 2, seed: int = 1234, scale: float = 0.0,
+                 stage_rule: int = 0):
         self.lib = _lib.load()
         self.B, self.H, self.L, self.d = B, H, L, d
         self.cfg = ACConfig(Cq, m0, n_max, tau_mode, float(tau_value), topk, iters_q, iters_k,
-                            iters_warm, 0, seed & (2**64 - 1), float(scale), 0)
+                            iters_warm, stage_rule, seed & (2**64 - 1), float(scale), 0)
         self.Cq, self.Ccap = Cq, n_max + m0
         h = ctypes.c_void_p()
         check(self.lib.ac_create(ctypes.byref(self.cfg), B, H, L, d, ctypes.byref(h)))
@@ -63,7 +64,8 @@ class SparseLayer:
         """Build from a synth.LayerConfig (shape overrides allowed)."""
         return cls(B or cfg.B, H or cfg.H, L or cfg.L, cfg.d, Cq=cfg.Cq, m0=cfg.m0, n_max=cfg.n_max,
                    tau_mode=cfg.tau_mode, tau_value=cfg.tau_value, topk=cfg.topk,
-                   iters_q=cfg.iters_q, iters_k=cfg.iters_k, iters_warm=cfg.iters_warm, seed=seed)
+                   iters_q=cfg.iters_q, iters_k=cfg.iters_k, iters_warm=cfg.iters_warm, seed=seed,
+                   stage_rule=cfg.stage_rule)
 
     # ------------------------------------------------------------------ calls
     def cluster_q(self, Q, init=None, iters: int = -1, labels=None, centroids=None):

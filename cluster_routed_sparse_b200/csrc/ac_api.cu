@@ -42,11 +42,11 @@ ac_status cuda_fail(ac_ctx *c, cudaError_t e, const char *what) {
         if (e_ != cudaSuccess) return cuda_fail(c, e_, what); \
     } while (0)
 
-// Cluster count of stage t > 0 of Algorithm 1 ("re-cluster these outlier tokens
-// with a few number of new clusters"): proportional to what is left, so that
-// the mean cluster size stays L/m0.
-int stage_clusters(int m0, int64_t nU, int64_t L, int t) {
-    if (t == 0) return (int)std::min<int64_t>(m0, nU);
+// Cluster count m_t of stage t (Algorithm 1 line 11, "choose a moderate
+// cluster number"): rule 0 makes the stage-0 choice every stage, min(m0, |U|);
+// rule 1 keeps the mean cluster size at L/m0, ceil(m0 |U| / L).
+int stage_clusters(int m0, int64_t nU, int64_t L, int t, int rule) {
+    if (t == 0 || rule == 0) return (int)std::min<int64_t>(m0, nU);
     int64_t m = (m0 * nU + L - 1) / L;
     m = std::max<int64_t>(1, std::min<int64_t>(m, nU));
     return (int)m;
@@ -177,7 +177,7 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
                 stages[h] = t;
                 continue;
             }
-            m[h] = stage_clusters(m0, ucnt[h], L, t);  // line 11
+            m[h] = stage_clusters(m0, ucnt[h], L, t, c->cfg.stage_rule);  // line 11
             max_m = std::max(max_m, m[h]);
             any = true;
         }
@@ -325,7 +325,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     if (d != 64 && d != 128) return AC_ERR_UNSUPPORTED;
     if (cfg->Cq < 1 || cfg->Cq > L || cfg->m0 < 1 || cfg->m0 > L || cfg->n_max < 1 || cfg->iters_q < 0 ||
         cfg->iters_k < 0 || cfg->iters_warm < 0 || cfg->tau_mode < 0 || cfg->tau_mode > 2 || cfg->topk == 0 ||
-        cfg->reserved0 != 0 || cfg->reserved1 != 0 || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
+        cfg->stage_rule < 0 || cfg->stage_rule > 1 || cfg->reserved1 != 0 || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
         return AC_ERR_INVALID_ARG;
     if ((int64_t)B * H * L >= (int64_t)1 << 31) return AC_ERR_INVALID_ARG;
     if (cfg->tau_mode == AC_TAU_PERCENTILE && (cfg->tau_value < 1.f || cfg->tau_value > 1000.f))

@@ -55,6 +55,7 @@ class LayerConfig:
     q_directions: int = 16
     steps: int = 1                   # simulated denoising steps
     seed: int = 20260000
+    stage_rule: int = 0              # m_t of stages t > 0: 0 = min(m0, |U|), 1 = proportional
 
 
 TAU_ABSOLUTE, TAU_MEAN_FACTOR, TAU_PERCENTILE = 0, 1, 2

@@ -79,7 +79,10 @@ typedef struct ac_config {
     int32_t iters_q;     /* Lloyd iterations of the query k-means (step 0)        */
     int32_t iters_k;     /* Lloyd iterations of each key stage (step 0)           */
     int32_t iters_warm;  /* Lloyd iterations of a warm-started step              */
-    int32_t reserved0;   /* must be 0                                             */
+    int32_t stage_rule;  /* cluster count m_t of stages t > 0 of Algorithm 1
+                            (line 11, "a moderate cluster number"):
+                            0: m_t = min(m0, |U|) (same choice every stage);
+                            1: m_t = min(|U|, max(1, ceil(m0 |U| / L)))           */
     uint64_t seed;       /* seeds the initial centres of step 0                   */
     float scale;         /* softmax scale; 0 selects 1/sqrt(d)                    */
     int32_t reserved1;   /* must be 0                                             */

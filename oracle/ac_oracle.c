@@ -49,7 +49,7 @@ typedef struct or_cfg {
     int iters_q;     /* Lloyd iterations for queries */
     int iters_k;     /* Lloyd iterations per key stage */
     int iters_warm;  /* Lloyd iterations in a warm-started step */
-    int pad_;
+    int stage_rule;  /* cluster count of stages t > 0, see or_stage_clusters */
     uint64_t seed;
 } or_cfg;
 
@@ -303,12 +303,16 @@ float or_tau(const float *dist, int64_t n, int mode, float value)
 /* Algorithm 1: MultiStageClustering                                    */
 /* ------------------------------------------------------------------ */
 
-/* Cluster count of stage t > 0.  The pages say only "a few number of new
- * clusters" (Sec. 3.2.2).  Reading: proportional to what is left, so that the
- * mean cluster size stays L/m0: m_t = min(|U|, max(1, ceil(m0 |U| / L))). */
-int32_t or_stage_clusters(int32_t m0, int64_t nU, int64_t L, int t)
+/* Cluster count m_t of stage t (Algorithm 1 line 11, "choose a moderate
+ * cluster number m_t"; the prose of Sec. 3.2.2 re-clusters the outliers "with
+ * a few number of new clusters").  Readings:
+ *   rule 0 (default): every stage makes the same moderate choice as stage 0,
+ *     m_t = min(m0, |U|);
+ *   rule 1: proportional to what is left, so that the mean cluster size stays
+ *     L/m0: m_t = min(|U|, max(1, ceil(m0 |U| / L))). */
+int32_t or_stage_clusters(int32_t m0, int64_t nU, int64_t L, int t, int rule)
 {
-    if (t == 0) return (int32_t)(m0 < nU ? m0 : nU);
+    if (t == 0 || rule == 0) return (int32_t)(m0 < nU ? m0 : nU);
     int64_t m = (m0 * nU + L - 1) / L;
     if (m < 1) m = 1;
     if (m > nU) m = nU;
@@ -367,7 +371,7 @@ int or_cluster_k_multistage(const uint16_t *K, int BH, int L, int d, const or_cf
         for (int64_t i = 0; i < (int64_t)L * d; ++i) Kf[i] = bf2f(K[(int64_t)h * L * d + i]);
         int64_t *uidx = (int64_t *)malloc((size_t)L * sizeof(int64_t));
         for (int64_t i = 0; i < L; ++i) uidx[i] = i;
-        int32_t m = or_stage_clusters(cfg->m0, L, L, 0);
+        int32_t m = or_stage_clusters(cfg->m0, L, L, 0, cfg->stage_rule);
         ms_stage(Kf, d, uidx, L, m, cfg, h, 0, C + (int64_t)h * Ccap * d, dist0 + (int64_t)h * L);
         n_k[h] = m;
         free(Kf);
@@ -408,7 +412,7 @@ int or_cluster_k_multistage(const uint16_t *K, int BH, int L, int d, const or_cf
                 f = 1;
                 break;
             }
-            int32_t m = or_stage_clusters(cfg->m0, nU, L, t);        /* line 11 */
+            int32_t m = or_stage_clusters(cfg->m0, nU, L, t, cfg->stage_rule); /* line 11 */
             ms_stage(Kf, d, uidx, nU, m, cfg, h, t, Ch + (int64_t)nc * d, dist); /* line 12, 14 */
             int64_t keep = 0;
             for (int64_t j = 0; j < nU; ++j) {                     /* lines 13-18 */

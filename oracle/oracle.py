@@ -46,7 +46,7 @@ class _Cfg(ctypes.Structure):
     _fields_ = [("Cq", ctypes.c_int), ("m0", ctypes.c_int), ("n_max", ctypes.c_int),
                 ("tau_mode", ctypes.c_int), ("tau_value", ctypes.c_float),
                 ("topk", ctypes.c_int), ("iters_q", ctypes.c_int), ("iters_k", ctypes.c_int),
-                ("iters_warm", ctypes.c_int), ("pad_", ctypes.c_int),
+                ("iters_warm", ctypes.c_int), ("stage_rule", ctypes.c_int),
                 ("seed", ctypes.c_uint64)]
 
 
@@ -65,7 +65,8 @@ def lib():
         _lib.or_topk_count.restype = ctypes.c_int32
         _lib.or_topk_count.argtypes = [ctypes.c_int32] * 3
         _lib.or_stage_clusters.restype = ctypes.c_int32
-        _lib.or_stage_clusters.argtypes = [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
+        _lib.or_stage_clusters.argtypes = [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                           ctypes.c_int]
         _lib.or_cluster_k_multistage.restype = ctypes.c_int
     return _lib
 
@@ -91,6 +92,7 @@ class Params:
     iters_k: int = 10
     iters_warm: int = 2
     seed: int = 1234
+    stage_rule: int = 0
 
     @property
     def ccap(self) -> int:
@@ -98,13 +100,13 @@ class Params:
 
     def c(self) -> _Cfg:
         return _Cfg(self.Cq, self.m0, self.n_max, self.tau_mode, float(self.tau_value),
-                    self.topk, self.iters_q, self.iters_k, self.iters_warm, 0,
+                    self.topk, self.iters_q, self.iters_k, self.iters_warm, self.stage_rule,
                     ctypes.c_uint64(self.seed & (2**64 - 1)))
 
     @staticmethod
     def from_layer_config(cfg, seed: int = 1234) -> "Params":
         return Params(cfg.Cq, cfg.m0, cfg.n_max, cfg.tau_mode, cfg.tau_value, cfg.topk,
-                      cfg.iters_q, cfg.iters_k, cfg.iters_warm, seed)
+                      cfg.iters_q, cfg.iters_k, cfg.iters_warm, seed, cfg.stage_rule)
 
 
 # ---------------------------------------------------------------- single steps
@@ -177,8 +179,8 @@ def tau(dist: np.ndarray, mode: int, value: float) -> float:
                               ctypes.c_float(value)))
 
 
-def stage_clusters(m0: int, nU: int, L: int, t: int) -> int:
-    return int(lib().or_stage_clusters(m0, nU, L, t))
+def stage_clusters(m0: int, nU: int, L: int, t: int, rule: int = 0) -> int:
+    return int(lib().or_stage_clusters(m0, nU, L, t, rule))
 
 
 def topk_count(topk: int, nk: int, nonempty: int) -> int:

@@ -31,7 +31,7 @@ def host_f32(t: torch.Tensor) -> np.ndarray:
 def make_layer_ctx(p: orc.Params, B, H, Lq, d) -> SparseLayer:
     return SparseLayer(B, H, Lq, d, Cq=p.Cq, m0=p.m0, n_max=p.n_max, tau_mode=p.tau_mode,
                        tau_value=p.tau_value, topk=p.topk, iters_q=p.iters_q, iters_k=p.iters_k,
-                       iters_warm=p.iters_warm, seed=p.seed)
+                       iters_warm=p.iters_warm, seed=p.seed, stage_rule=p.stage_rule)
 
 
 def gpu_state(lay: SparseLayer) -> dict:
@@ -53,7 +53,10 @@ def gpu_state(lay: SparseLayer) -> dict:
 def rel_err(a, b):
     a = np.asarray(a, np.float64)
     b = np.asarray(b, np.float64)
-    return np.abs(a - b) / np.maximum(np.abs(b), 1e-30)
+    same = a == b  # includes equal infinities (Comp = 1/0 when every key sits on its centre)
+    with np.errstate(invalid="ignore"):
+        r = np.abs(a - b) / np.maximum(np.abs(b), 1e-30)
+    return np.where(same, 0.0, r)
 
 
 def assert_centres(gpu, ora, what):

@@ -35,7 +35,7 @@ def _check_state(cfg, Q, K, V, O, gs, p, step0: bool):
             rs = gs["removed_stage"][h]
             tot, nU = 0, L
             for t in range(int(gs["stages"][h])):
-                m = orc.stage_clusters(cfg.m0, nU, L, t)
+                m = orc.stage_clusters(cfg.m0, nU, L, t, p.stage_rule)
                 tot += m
                 nU -= int((rs == t).sum())
             assert tot == nk

@@ -191,13 +191,13 @@ def test_tau_rules_by_hand():
 
 # ----------------------------------------------------------------- Algorithm 1
 
-@pytest.mark.parametrize("case", [0, 1])
+@pytest.mark.parametrize("case", [0, 1, 2])
 def test_multistage_hand_example(case):
     g = _golden("multistage_hand.json")
     c = g["cases"][case]
     K16 = bf(np.array(g["keys"], np.float32))[None]
     p = orc.Params(Cq=1, m0=g["m0"], n_max=c["n_max"], tau_mode=orc.TAU_ABSOLUTE,
-                   tau_value=c["tau"], topk=1, iters_k=g["iters"])
+                   tau_value=c["tau"], topk=1, iters_k=g["iters"], stage_rule=c["stage_rule"])
     kc = orc.cluster_k_multistage(K16, p)
     assert kc.n_k[0] == c["n_k"] and kc.F[0] == c["F"] and kc.stages[0] == c["stages"]
     assert kc.labels[0].tolist() == c["labels"]
@@ -227,7 +227,7 @@ def test_multistage_invariants_tiny_config():
         # n_k is the sum of the stage sizes m_t
         tot, nU = 0, L
         for t in range(int(kc.stages[h])):
-            m = orc.stage_clusters(cfg.m0, nU, L, t)
+            m = orc.stage_clusters(cfg.m0, nU, L, t, p.stage_rule)
             tot += m
             nU -= int((rs == t).sum())
         assert tot == nk

@@ -151,8 +151,11 @@ def test_state_resume_is_bit_exact():
     b.import_state(blob)
     _, Ob, gb = run_gpu_layer(Q1, K1, V1, p, lay=b, warm=True)
     assert np.array_equal(Oa, Ob)
-    for key in ("labels_q", "labels_k", "cent_q", "cent_k", "sel"):
+    for key in ("labels_q", "labels_k", "cent_q", "cent_k", "ksel"):
         assert np.array_equal(ga[key], gb[key]), key
+    for h in range(ga["ksel"].shape[0]):
+        k = int(ga["ksel"][h])
+        assert np.array_equal(ga["sel"][h, :, :k], gb["sel"][h, :, :k])
     a.close()
     b.close()
 
