@@ -40,6 +40,16 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
+def cluster_q_noalloc(Q, Cq: int, labels, centroids, iters: int = 10, seed: int = 1234, init=None):
+    """ac_cluster_q_noalloc: angular k-means of Q [B, H, L, d] (bf16, CUDA) into
+    caller-provided labels [B, H, L] int32 and centroids [B, H, Cq, d] fp32,
+    with no device allocation inside the library (see include/ac.h)."""
+    lib = _lib.load()
+    B, H, L, d = Q.shape
+    check(lib.ac_cluster_q_noalloc(_bits(Q), B * H, L, d, Cq, iters, seed & (2**64 - 1), _ptr(init),
+                                   _ptr(labels), _ptr(centroids), _stream()))
+
+
 class SparseLayer:
     """One cluster-routed sparse attention layer context for [B, H, L, d] inputs.
 

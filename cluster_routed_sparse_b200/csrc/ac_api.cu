@@ -20,7 +20,7 @@ std::atomic<long long> ac::g_launches{0};
 
 namespace {
 
-const char *g_static_msg = "";
+thread_local std::string g_static_msg;
 
 ac_status fail(ac_ctx *c, ac_status st, const char *what) {
     if (c) c->msg = what;
@@ -312,11 +312,13 @@ void free_all(ac_ctx *c) {
 
 }  // namespace
 
+void ac::set_static_error(const char *msg) { g_static_msg = msg; }
+
 // ======================================================================== ABI
 
 extern "C" {
 
-const char *ac_last_error_string(const ac_ctx *ctx) { return ctx ? ctx->msg.c_str() : g_static_msg; }
+const char *ac_last_error_string(const ac_ctx *ctx) { return ctx ? ctx->msg.c_str() : g_static_msg.c_str(); }
 
 ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32_t d, ac_ctx **out) {
     if (!cfg || !out) return AC_ERR_INVALID_ARG;

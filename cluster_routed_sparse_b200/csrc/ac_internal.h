@@ -93,6 +93,9 @@ namespace ac {
 extern std::atomic<long long> g_launches;
 #define AC_NOTE_LAUNCH() ::ac::g_launches.fetch_add(1, std::memory_order_relaxed)
 
+// Message returned by ac_last_error_string(NULL) (per thread).
+void set_static_error(const char *msg);
+
 cudaError_t launch_qnorm(const bf16 *Q, float *inv, int64_t rows, int d, uint32_t *err, cudaStream_t s);
 
 // Exact assignment: for every row of every unit h (rows given by an index

@@ -112,7 +112,8 @@ AC_API ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L
 /* Free the context and its workspace (synchronises the device first). */
 AC_API ac_status ac_destroy(ac_ctx *ctx);
 
-/* Last error message of the context (static storage for ctx == NULL). */
+/* Last error message of the context; with ctx == NULL, the last error of a
+ * context-free call (ac_cluster_q_noalloc) in this thread. */
 AC_API const char *ac_last_error_string(const ac_ctx *ctx);
 
 /* Algorithm 3 line 3, Sec. 3.1 / App. A.2: L2-normalise every query (fp32)
@@ -234,6 +235,30 @@ typedef struct ac_attn_counters {
 } ac_attn_counters;
 
 AC_API ac_status ac_get_attn_counters(ac_ctx *ctx, ac_attn_counters *out);
+
+/* The query clustering of ac_cluster_q (normalise, then Lloyd k-means with
+ * Cq centres) without a context and without allocating device memory.  The
+ * paper has no counterpart of this entry point; it exists for callers that
+ * cannot call cudaMalloc while they run: a plugin's enqueue callback inside an
+ * inference engine, a server that must not grow its footprint while serving,
+ * or a process whose device memory belongs to another allocator.
+ *  - Q: device [BH, L, d] bf16 (d in {64, 128}).  init_centroids: nullable
+ *    device [BH, Cq, d] fp32 (NULL: seeded from the queries with `seed`, as
+ *    ac_cluster_q does).  iters >= 0 Lloyd iterations, then a final assignment.
+ *  - Outputs (device, required): labels_out [BH, L] int32; centroids_out
+ *    [BH, Cq, d] fp32, also used as the working centres (updated in place).
+ *  - Limits: BH*L <= 1048576 and BH*(Cq+1) <= 65536, else AC_ERR_INVALID_ARG
+ *    before any work.  The scratch (norms, permutation, offsets, counts) is one
+ *    8.5 MiB __device__ array that every GPU which loads libac holds until the
+ *    process exits; nothing is allocated per call.
+ *  - The first call on a device looks the array's address up
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call shares the one array: calls that overlap on the GPU (two
+ *    streams, two threads) race and corrupt each other's results.  Serialise
+ *    them.  Asynchronous on `stream`; no NaN check (no error word to read). */
+AC_API ac_status ac_cluster_q_noalloc(const uint16_t *Q, int32_t BH, int32_t L, int32_t d, int32_t Cq,
+                                      int32_t iters, uint64_t seed, const float *init_centroids,
+                                      int32_t *labels_out, float *centroids_out, void *stream);
 
 /* Number of kernels libac has launched in this process so far (all contexts). */
 AC_API ac_status ac_get_launch_count(int64_t *out);
