@@ -40,9 +40,8 @@ NOISE_STD = 0.02
 
 # ---------------------------------------------------------------- inputs
 def _gen_head(args):
-    cfg_id, head = args
+    cfg, head = args
     from cluster_routed_sparse_b200 import synth
-    cfg = synth.CONFIGS[cfg_id]
     g = synth
     q = g._head_queries_f32(cfg, head)
     k = g._head_keys_f32(cfg, head)
@@ -50,15 +49,13 @@ def _gen_head(args):
     return head, q, k, v
 
 
-def generate_step0_f32(cfg_id: int, heads, procs: int):
+def generate_step0_f32(cfg, heads, procs: int):
     """fp32 step-0 tokens of the listed heads, generated in a spawn pool."""
     import multiprocessing as mp
-    from cluster_routed_sparse_b200 import synth
-    cfg = synth.CONFIGS[cfg_id]
     out = np.empty((3, len(heads), cfg.L, cfg.d), np.float32)
     ctx = mp.get_context("spawn")
     with ctx.Pool(procs) as pool:
-        for h, q, k, v in pool.imap_unordered(_gen_head, [(cfg_id, h) for h in heads]):
+        for h, q, k, v in pool.imap_unordered(_gen_head, [(cfg, h) for h in heads]):
             i = heads.index(h)
             out[0, i], out[1, i], out[2, i] = q, k, v
     return out
@@ -208,6 +205,8 @@ def main():
     ap.add_argument("--no-sdpa", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--procs", type=int, default=min(32, os.cpu_count() or 1))
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only the first N heads (profiling of a smaller case; not a bench line)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -216,10 +215,13 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     from cluster_routed_sparse_b200 import synth
+    import dataclasses
     cfg = synth.CONFIGS[CONFIG_ID]
+    if args.heads:
+        cfg = dataclasses.replace(cfg, H=args.heads)
 
     # inputs first (spawn pool, before any CUDA call); each rank its own layer
-    x0 = generate_step0_f32(CONFIG_ID, list(range(cfg.H)), max(1, args.procs // max(1, world)))
+    x0 = generate_step0_f32(cfg, list(range(cfg.H)), max(1, args.procs // max(1, world)))
 
     import torch
     import torch.distributed as dist
@@ -380,11 +382,14 @@ def time_e2e(lay, steps_in, cfg, dense_flops_layer, world, dist):
     torch.cuda.synchronize()
     lay.forward_host(*host[0], hO, warm=False)  # warm-up of the staging buffers
     torch.cuda.synchronize()
-    t0 = time.perf_counter()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
     for s in range(N_DENOISE):
         lay.forward_host(*host[s], hO, warm=s > 0)
+    e1.record(stream)
     torch.cuda.synchronize()
-    ms = (time.perf_counter() - t0) * 1e3
+    ms = e0.elapsed_time(e1)
     if dist is not None:
         t = torch.tensor([ms], device="cuda", dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -392,7 +397,7 @@ def time_e2e(lay, steps_in, cfg, dense_flops_layer, world, dist):
     nbytes = cfg.B * cfg.H * cfg.L * cfg.d * 2
     return {"value": world * N_DENOISE * dense_flops_layer / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": 3 * nbytes * N_DENOISE, "d2h_bytes_per_step": nbytes * N_DENOISE,
-            "ms_per_step": ms, "clock": "host wall clock around synchronous calls"}
+            "ms_per_step": ms, "clock": "CUDA events around the ten host-buffer calls"}
 
 
 if __name__ == "__main__":

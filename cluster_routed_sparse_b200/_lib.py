@@ -65,7 +65,8 @@ class ACStageTimes(ctypes.Structure):
 
 class ACAttnCounters(ctypes.Structure):
     _fields_ = [("kept_pairs", ctypes.c_int64), ("computed_pairs", ctypes.c_int64),
-                ("tiles", ctypes.c_int64), ("dense_heads", ctypes.c_int64)]
+                ("tiles", ctypes.c_int64), ("dense_heads", ctypes.c_int64),
+                ("wait_failure", ctypes.c_int64)]
 
 
 # every function that include/ac.h declares, with its ctypes signature

@@ -284,7 +284,7 @@ ac_status sparse_attn_impl(ac_ctx *c, const bf16 *Q, const bf16 *K, const bf16 *
     CK(launch_permute_rows(Q, c->perm_q, c->Qp, c->L, c->d, c->BH, s), "permute q");
     CK(launch_permute_rows(K, c->perm_k, c->Kp, c->L, c->d, c->BH, s), "permute k");
     CK(launch_permute_rows(V, c->perm_k, c->Vp, c->L, c->d, c->BH, s), "permute v");
-    CK(cudaMemsetAsync(c->counters, 0, 4 * sizeof(unsigned long long), s), "counters");
+    CK(cudaMemsetAsync(c->counters, 0, 8 * sizeof(unsigned long long), s), "counters");
     AttnArgs a{&c->tm_q, &c->tm_k, &c->tm_v, O, c->perm_q, c->offs_q, c->counts_q, c->tile_prefix, c->ranges,
                c->nboxes, c->ksel, c->dense, c->L, c->Cq, c->Ccap, c->BH, c->d,
                (float)(c->scale * 1.4426950408889634), c->err, c->counters};
@@ -398,7 +398,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->Qp, BH * Lz * dz));
     A(dalloc(&c->Kp, BH * Lz * dz));
     A(dalloc(&c->Vp, BH * Lz * dz));
-    A(dalloc(&c->counters, 4));
+    A(dalloc(&c->counters, 8));
     A(dalloc(&c->err, 1));
     A(cudaMallocHost(&c->h_u_cnt, BH * sizeof(int)));
     A(cudaMallocHost(&c->h_st_m, BH * sizeof(int)));
@@ -629,7 +629,7 @@ ac_status ac_synchronize(ac_ctx *c, void *stream) {
 
 ac_status ac_get_attn_counters(ac_ctx *c, ac_attn_counters *out) {
     if (!c || !out) return AC_ERR_INVALID_ARG;
-    unsigned long long h[4];
+    unsigned long long h[8];
     CK(cudaDeviceSynchronize(), "sync");
     CK(cudaMemcpy(h, c->counters, sizeof(h), cudaMemcpyDeviceToHost), "counters");
     std::vector<uint8_t> dn(c->BH);
@@ -637,6 +637,7 @@ ac_status ac_get_attn_counters(ac_ctx *c, ac_attn_counters *out) {
     out->kept_pairs = (int64_t)h[0];
     out->computed_pairs = (int64_t)h[1];
     out->tiles = (int64_t)h[2];
+    out->wait_failure = (int64_t)h[4];
     out->dense_heads = 0;
     for (uint8_t v : dn) out->dense_heads += v ? 1 : 0;
     return AC_OK;

@@ -62,11 +62,11 @@ struct ac_ctx {
     int *ksel;         // [BH]
     int2 *ranges;      // [BH, Cq, Ccap]  (start row in cluster order, count)
     int *nboxes;       // [BH*Cq]         8-row key boxes per query cluster
-    int *tile_prefix;  // [BH*Cq+1]       128-query tiles, exclusive prefix
+    int *tile_prefix;  // [BH*Cq+1]       attention items (pairs of 128-query tiles), exclusive prefix
 
     // ---- attention
     bf16 *Qp, *Kp, *Vp;  // [BH, L, d] cluster-order copies
-    unsigned long long *counters;  // [4] kept pairs, computed pairs, tiles, dense heads
+    unsigned long long *counters;  // [8] kept pairs, computed pairs, items, -, first wait failure
     CUtensorMap tm_q, tm_k, tm_v;
 
     // ---- host-buffer forward

@@ -3,21 +3,30 @@
 //
 // Inputs are the cluster-order copies Qp, Kp, Vp ([BH*L, d] bf16): the queries
 // of one query cluster are contiguous, and so are the keys of one key cluster.
-// One CTA handles one 128-query tile of one query cluster.  Its key set is the
-// list of row ranges of the selected key clusters (one range of all L keys for
-// a dense unit), walked in 8-row boxes; 16 boxes form a 128-column key tile.
-// Columns of a box past the end of its cluster are masked, so a cluster wastes
-// at most 7 columns.
+// One CTA handles two consecutive 128-query tiles of one query cluster, which
+// share every K/V tile.  The key set is the list of row ranges of the selected
+// key clusters (one range of all L keys for a dense unit), walked in 8-row
+// boxes; 16 boxes form a 128-column key tile.  Columns of a box past the end of
+// its cluster are masked, so a cluster wastes at most 7 columns.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t
-//   warp 4     TMA producer (Q tile once; K and V boxes per key tile)
-//   warp 5     TMEM allocator and the single-thread tcgen05.mma issuer
-// Pipeline per key tile j (S and O double-buffered in TMEM, K/V in 2 stages):
-//   S_j = Q K_j^T  -> softmax_j (P_j to smem)  -> O_j = P_j V_j
-// with S_{j+1} issued before PV_j, so the tensor core runs while the softmax
-// warps work.  The softmax warps keep the output row in registers:
-//   acc = acc * 2^(m_{j-1} - m_j) + O_j.
+// Warp roles (384 threads, three warpgroups):
+//   warps 0-3 / 4-7  softmax + epilogue of query tile 0 / 1; thread t owns
+//                    query row t = TMEM lane t
+//   warp 8           TMA producer: Q tiles once; per key tile the K and V
+//                    boxes and the tile's column-validity masks
+//   warp 9           TMEM allocator and the single-thread tcgen05.mma issuer
+//   warps 10-11      idle
+// Registers: launched at 168 per thread (65536 / 384, rounded down to 8); the
+// third warpgroup drops to 72 and the two softmax warpgroups rise to 200:
+// 2 * 128 * 200 + 128 * 72 = 60416 <= 384 * 168 = 64512.
+// Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1.  The softmax writes P
+// (bf16) over the first half of its S columns and the PV product reads A = P
+// from tensor memory, so S, P and O never touch shared memory.  O accumulates
+// in TMEM across key tiles; its rows are rescaled only when the running row
+// maximum grows by more than 8 (log2 units), so P <= 2^8 stays exact in fp32
+// sums and representable in bf16.
+// MMA order per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): while one
+// softmax warpgroup works on its S, the tensor core runs the other's products.
 // Every mbarrier wait is bounded; on timeout the CTA records an error, drains
 // what it issued and frees its TMEM.
 #include "ac_device.cuh"
@@ -30,34 +39,34 @@ constexpr int BM = 128;       // query rows per tile
 constexpr int BN = 128;       // key columns per tile
 constexpr int NS = 2;         // K/V pipeline stages
 constexpr int BOXES = BN / 8; // 8-row boxes per key tile
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 384;
+constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 72;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= NTHREADS * 168, "register split exceeds the launch");
+constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
 struct Layout {
     static constexpr int HALVES = D / 64;  // 128-byte (64 x bf16) column halves
-    static constexpr uint32_t Q_BYTES = HALVES * BM * 128;
+    static constexpr uint32_t Q_TILE = HALVES * BM * 128;
     static constexpr uint32_t KV_BYTES = HALVES * BN * 128;
-    static constexpr uint32_t P_BYTES = 2 * BM * 128;  // 128 keys = 2 halves
-    static constexpr uint32_t OFF_Q = 0;
-    static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+    static constexpr uint32_t OFF_Q = 0;                        // two query tiles
+    static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_TILE;
     static constexpr uint32_t OFF_V = OFF_K + NS * KV_BYTES;
-    static constexpr uint32_t OFF_P = OFF_V + NS * KV_BYTES;
-    static constexpr uint32_t OFF_BAR = OFF_P + 2 * P_BYTES;
+    static constexpr uint32_t OFF_MASK = OFF_V + NS * KV_BYTES;  // [NS][4] uint32
+    static constexpr uint32_t OFF_BAR = OFF_MASK + 64;
     static constexpr uint32_t BYTES = OFF_BAR + 256;
     static constexpr uint32_t SMEM = BYTES + 1024;  // 1024-byte alignment slack
 };
 
 enum {
-    B_KVF = 0,   // [2] K/V stage filled (TMA tx)
-    B_KVE = 2,   // [2] K/V stage free (MMA commit)
-    B_QF = 4,    // Q tile filled
-    B_SF = 5,    // [2] S buffer written (MMA commit)
-    B_SE = 7,    // [2] S buffer read (128 softmax threads)
-    B_PF = 9,    // [2] P buffer written (128 softmax threads)
-    B_OF = 11,   // [2] O buffer written (MMA commit)
-    B_OE = 13,   // [2] O buffer read (128 softmax threads)
-    B_DONE = 15, // all MMAs complete
-    NBAR = 16
+    B_KVF = 0,   // [NS] K/V stage filled (TMA tx) -- also publishes the masks
+    B_KVE = 2,   // [NS] K/V stage free (MMA commit after both PV products)
+    B_QF = 4,    // query tiles filled
+    B_SF = 5,    // [2] S_i written (MMA commit)
+    B_PF = 7,    // [2] P_i written (+ O_i rescaled) by the 128 softmax threads
+    B_OF = 9,    // [2] last PV_i complete (MMA commit)
+    B_DONE = 11, // every MMA complete
+    NBAR = 12
 };
 
 struct KeyWalker {
@@ -99,24 +108,14 @@ struct AttnParams {
     unsigned long long *counters;
 };
 
-// acc = acc * a + O_jj (row of this thread), then release the O buffer.
-template <int D>
-__device__ __forceinline__ bool accumulate_o(float (&acc)[D], uint32_t tmem_row, uint32_t bar_full,
-                                             uint32_t bar_empty, int jj, float a) {
-    if (!mbar_wait(bar_full, (jj >> 1) & 1)) return false;
-    tc_fence_after();
-    const uint32_t tO = tmem_row + 256 + (jj & 1) * 128;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + c * 32, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[c * 32 + i] = acc[c * 32 + i] * a + __uint_as_float(r[i]);
+__device__ __forceinline__ void record_wait_failure(const AttnParams &p, int role, int bidx, int j, int par) {
+    set_err(p.err, DEV_ERR_TIMEOUT);
+    if (p.counters) {
+        const unsigned long long code =
+            1ull << 60 | (unsigned long long)role << 24 | (unsigned long long)bidx << 16 |
+            (unsigned long long)(j & 0x7FFF) << 1 | (unsigned long long)(par & 1);
+        atomicCAS(&p.counters[4], 0ull, code);
     }
-    tc_fence_before();
-    mbar_arrive(bar_empty);
-    return true;
 }
 
 template <int D>
@@ -130,7 +129,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // ---- work item: (unit h, query cluster qc, 128-row tile)
+    // ---- work item: (unit h, query cluster qc, pair of 128-row tiles)
     const int nhq = p.BH * p.Cq;
     const int item = blockIdx.x;
     if (item >= p.tile_prefix[nhq]) return;
@@ -141,9 +140,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         else hi = mid;
     }
     const int hq = lo, h = hq / p.Cq, qc = hq % p.Cq;
-    const int tile = item - p.tile_prefix[hq];
-    const int row0 = p.offs_q[(int64_t)h * (p.Cq + 1) + qc] + tile * BM;
-    const int nvalid = min(BM, p.counts_q[hq] - tile * BM);
+    const int pair = item - p.tile_prefix[hq];
+    const int row0 = p.offs_q[(int64_t)h * (p.Cq + 1) + qc] + pair * 2 * BM;
+    const int rest = p.counts_q[hq] - pair * 2 * BM;
+    const int valid0 = min(BM, rest), valid1 = min(BM, rest - BM);
+    const bool has1 = valid1 > 0;
     const int64_t unit_row = (int64_t)h * p.L;
     const int n_tiles = (p.nboxes[hq] + BOXES - 1) / BOXES;
     const int2 *rg = p.ranges + (int64_t)hq * p.Ccap;
@@ -151,23 +152,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     const uint32_t bar0 = sbase + LY::OFF_BAR;
 #define BAR(i) (bar0 + 8u * (uint32_t)(i))
+    // Bounded wait; the first wait to give up anywhere records
+    // (role << 24 | barrier << 16 | tile << 1 | parity) in counters[4].
+#define WAIT(role, bidx, jj, par)                                                                     \
+    (mbar_wait_or_abort(BAR(bidx), (par), p.err) ||                                                   \
+     (record_wait_failure(p, (role), (bidx), (jj), (par)), false))
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + LY::OFF_BAR + 8 * NBAR);
+    uint32_t *masks = reinterpret_cast<uint32_t *>(sm + LY::OFF_MASK);
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NS; ++i) {
             mbar_init(BAR(B_KVF + i), 1);
             mbar_init(BAR(B_KVE + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(BAR(B_SF + i), 1);
-            mbar_init(BAR(B_SE + i), BM);
             mbar_init(BAR(B_PF + i), BM);
             mbar_init(BAR(B_OF + i), 1);
-            mbar_init(BAR(B_OE + i), BM);
         }
         mbar_init(BAR(B_QF), 1);
         mbar_init(BAR(B_DONE), 1);
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
     }
@@ -177,29 +184,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
 
-    if (warp == 4) {
+    if (warp >= 8) {
+      reg_dealloc<kRegsOther>();
+      if (warp == 8) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(BAR(B_QF), LY::Q_BYTES);
-            for (int hf = 0; hf < LY::HALVES; ++hf)
-                tma_load_2d(sbase + LY::OFF_Q + hf * BM * 128, &tm_q, hf * 64, (int)(unit_row + row0),
-                            BAR(B_QF));
+            mbar_arrive_expect_tx(BAR(B_QF), 2 * LY::Q_TILE);
+            for (int t = 0; t < 2; ++t)
+                for (int hf = 0; hf < LY::HALVES; ++hf)
+                    tma_load_2d(sbase + LY::OFF_Q + t * LY::Q_TILE + hf * BM * 128, &tm_q, hf * 64,
+                                (int)(unit_row + row0 + t * BM), BAR(B_QF));
             KeyWalker w;
             w.init(rg, nr);
             int issued = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int s = j % NS;
-                if (j >= NS && !mbar_wait(BAR(B_KVE + s), ((j / NS) - 1) & 1)) {
+                if (j >= NS && !WAIT(1, B_KVE + s, j, ((j / NS) - 1) & 1)) {
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(BAR(B_KVF + s), 2 * LY::KV_BYTES);
-                const uint32_t kd = sbase + LY::OFF_K + s * LY::KV_BYTES;
-                const uint32_t vd = sbase + LY::OFF_V + s * LY::KV_BYTES;
+                // pass 1: validity masks of the 16 boxes; pass 2: their loads
+                KeyWalker w2 = w;
+                uint32_t vm[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
                 for (int b = 0; b < BOXES; ++b) {
                     int st, c;
                     w.next(st, c);
+                    vm[b >> 2] |= (c >= 8 ? 0xFFu : ((1u << c) - 1u)) << ((b & 3) * 8);
+                }
+                *reinterpret_cast<uint4 *>(masks + 4 * s) = make_uint4(vm[0], vm[1], vm[2], vm[3]);
+                mbar_arrive_expect_tx(BAR(B_KVF + s), 2 * LY::KV_BYTES);  // releases the masks
+                const uint32_t kd = sbase + LY::OFF_K + s * LY::KV_BYTES;
+                const uint32_t vd = sbase + LY::OFF_V + s * LY::KV_BYTES;
+#pragma unroll 1
+                for (int b = 0; b < BOXES; ++b) {
+                    int st, c;
+                    w2.next(st, c);
                     const int row = (int)(unit_row + st);
+#pragma unroll
                     for (int hf = 0; hf < LY::HALVES; ++hf) {
                         tma_load_2d(kd + hf * BN * 128 + b * 1024, &tm_k, hf * 64, row, BAR(B_KVF + s));
                         tma_load_2d(vd + hf * BN * 128 + b * 1024, &tm_v, hf * 64, row, BAR(B_KVF + s));
@@ -209,174 +231,208 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             // Loads still in flight must land before the CTA exits.
             for (int j = issued - NS < 0 ? 0 : issued - NS; j < issued; ++j)
-                if (!mbar_wait(BAR(B_KVF + (j % NS)), (j / NS) & 1)) ok = false;
-            if (!mbar_wait(BAR(B_QF), 0)) ok = false;
+                if (!WAIT(2, B_KVF + (j % NS), j, (j / NS) & 1)) ok = false;
+            if (!WAIT(2, B_QF, 0, 0)) ok = false;
             if (!ok) set_err(p.err, DEV_ERR_TIMEOUT);
         }
         __syncwarp();
-    } else if (warp == 5) {
+      } else if (warp == 9) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t IQK = idesc_bf16_f32(BM, BN, false);
             constexpr uint32_t IPV = idesc_bf16_f32(BM, D, true);
-            const uint32_t qa = sbase + LY::OFF_Q;
-            if (!mbar_wait(BAR(B_QF), 0)) ok = false;
-            tc_fence_after();
-            auto issue_s = [&](int j) -> bool {
-                const int s = j % NS, b = j & 1;
-                if (!mbar_wait(BAR(B_KVF + s), (j / NS) & 1)) return false;
-                if (j >= 2 && !mbar_wait(BAR(B_SE + b), ((j >> 1) - 1) & 1)) return false;
-                tc_fence_after();
-                const uint32_t ka = sbase + LY::OFF_K + s * LY::KV_BYTES;
+            auto issue_s = [&](int i, int j) {
+                const uint32_t qa = sbase + LY::OFF_Q + i * LY::Q_TILE;
+                const uint32_t ka = sbase + LY::OFF_K + (j % NS) * LY::KV_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                    tc_mma_bf16(tmem + b * BN, sdesc_sw128(qa + off, 16, 1024),
-                                sdesc_sw128(ka + off, 16, 1024), IQK, kk > 0 ? 1u : 0u);
+                    tc_mma_bf16(tmem + i * BN, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
+                                IQK, kk > 0 ? 1u : 0u);
                 }
-                tc_commit(BAR(B_SF + b));
-                return true;
+                tc_commit(BAR(B_SF + i));
             };
-            if (ok && n_tiles > 0) ok = issue_s(0);
+            auto issue_pv = [&](int i, int j) {
+                const uint32_t va = sbase + LY::OFF_V + (j % NS) * LY::KV_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    tc_mma_bf16_ts(tmem + 256 + i * 128, tmem + i * BN + kk * 8,
+                                   sdesc_sw128(va + kk * 16 * 128, BN * 128, 1024), IPV,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+            };
+            if (!WAIT(3, B_QF, 0, 0)) ok = false;
+            if (ok && n_tiles > 0) {
+                if (!WAIT(3, B_KVF, 0, 0)) ok = false;
+                tc_fence_after();
+                if (ok) {
+                    issue_s(0, 0);
+                    if (has1) issue_s(1, 0);
+                }
+            }
             for (int j = 0; j < n_tiles && ok; ++j) {
-                if (j + 1 < n_tiles && !issue_s(j + 1)) {
-                    ok = false;
-                    break;
-                }
-                const int s = j % NS, b = j & 1;
-                if (!mbar_wait(BAR(B_PF + b), (j >> 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                if (j >= 2 && !mbar_wait(BAR(B_OE + b), ((j >> 1) - 1) & 1)) {
+                const bool more = j + 1 < n_tiles;
+                if (!WAIT(3, B_PF + 0, j, j & 1)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t pa = sbase + LY::OFF_P + b * LY::P_BYTES;
-                const uint32_t va = sbase + LY::OFF_V + s * LY::KV_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                    const uint32_t boff = kk * 16 * 128;
-                    tc_mma_bf16(tmem + 256 + b * 128, sdesc_sw128(pa + aoff, 16, 1024),
-                                sdesc_sw128(va + boff, BN * 128, 1024), IPV, kk > 0 ? 1u : 0u);
+                issue_pv(0, j);
+                if (!more) tc_commit(BAR(B_OF + 0));
+                if (more) {
+                    if (!WAIT(3, B_KVF + ((j + 1) % NS), j + 1, ((j + 1) / NS) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_s(0, j + 1);
                 }
-                tc_commit(BAR(B_OF + b));
-                tc_commit(BAR(B_KVE + s));
+                if (has1) {
+                    if (!WAIT(3, B_PF + 1, j, j & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_pv(1, j);
+                    if (!more) tc_commit(BAR(B_OF + 1));
+                    if (more) issue_s(1, j + 1);
+                }
+                tc_commit(BAR(B_KVE + (j % NS)));
             }
             tc_commit(BAR(B_DONE));
-            if (!mbar_wait(BAR(B_DONE), 0)) ok = false;
+            if (!WAIT(4, B_DONE, 0, 0)) ok = false;
             if (!ok) set_err(p.err, DEV_ERR_TIMEOUT);
         }
         __syncwarp();
+      }
     } else {
+        reg_alloc<kRegsSoftmax>();
         // ------------------------------------------------ softmax + epilogue
-        const int row = tid;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const float sl2 = p.scale_log2;
-        float m_run = -INFINITY, l_run = 0.f, alpha_prev = 0.f;
-        float acc[D];
-#pragma unroll
-        for (int k = 0; k < D; ++k) acc[k] = 0.f;
-        long long kept_cols = 0;
-
-        KeyWalker w;
-        w.init(rg, nr);
-        for (int j = 0; j < n_tiles; ++j) {
-            uint32_t vm[4] = {0u, 0u, 0u, 0u};
-#pragma unroll 1
-            for (int bx = 0; bx < BOXES; ++bx) {
-                int st, c;
-                w.next(st, c);
-                const uint32_t bits = c >= 8 ? 0xFFu : ((1u << c) - 1u);
-                vm[bx >> 2] |= bits << ((bx & 3) * 8);
-            }
-            kept_cols += __popc(vm[0]) + __popc(vm[1]) + __popc(vm[2]) + __popc(vm[3]);
-            const int b = j & 1;
-            if (!mbar_wait(BAR(B_SF + b), (j >> 1) & 1)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t tS = tmem + lane_off + b * BN;
-            float tmax = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tS + c * 32, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if ((vm[c] >> i) & 1u) tmax = fmaxf(tmax, __uint_as_float(r[i]));
-            }
-            const float m_new = fmaxf(m_run, tmax * sl2);
-            const float alpha = ex2_approx(m_run - m_new);
-            float rs = 0.f;
-            uint8_t *pb = sm + LY::OFF_P + b * LY::P_BYTES;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tS + c * 32, r);
-                tmem_ld_wait();
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float p0 = ((vm[c] >> i) & 1u) ? ex2_approx(__uint_as_float(r[i]) * sl2 - m_new) : 0.f;
-                    const float p1 =
-                        ((vm[c] >> (i + 1)) & 1u) ? ex2_approx(__uint_as_float(r[i + 1]) * sl2 - m_new) : 0.f;
-                    rs += p0 + p1;
-                    pk[i >> 1] = pack_bf16x2(p0, p1);
+        const int wg = warp >> 2;  // query tile
+        const int row = tid & 127;
+        const int valid = wg == 0 ? valid0 : valid1;
+        if (wg == 0 || has1) {
+            const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+            const uint32_t tS = tmem + lane_off + wg * BN;
+            const uint32_t tO = tmem + lane_off + 256 + wg * 128;
+            const float sl2 = p.scale_log2;
+            float m_run = -INFINITY, l_run = 0.f;
+            long long kept_cols = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int s = j % NS;
+                // Wait outcomes are combined across the warp: the TMEM loads and
+                // stores below are warp-collective, so a warp leaves together.
+                if (!__all_sync(0xFFFFFFFFu, WAIT(5 + wg, B_KVF + s, j, (j / NS) & 1))) {
+                    ok = false;
+                    break;
                 }
-                // keys [32c, 32c+32): half c>>1, 16-byte chunks (c&1)*4 .. +3, 128B swizzle
-                uint8_t *rowp = pb + (c >> 1) * (BM * 128) + row * 128;
+                const uint4 mk = *reinterpret_cast<const uint4 *>(masks + 4 * s);
+                const uint32_t vm[4] = {mk.x, mk.y, mk.z, mk.w};
+                kept_cols += __popc(vm[0]) + __popc(vm[1]) + __popc(vm[2]) + __popc(vm[3]);
+                if (!__all_sync(0xFFFFFFFFu, WAIT(5 + wg, B_SF + wg, j, j & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t r[4][32];
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int chunk = (((c & 1) * 4) + q4) ^ (row & 7);
-                    *reinterpret_cast<uint4 *>(rowp + chunk * 16) =
-                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, r[c]);
+                tmem_ld_wait();
+                float tmax = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if ((vm[c] >> i) & 1u) tmax = fmaxf(tmax, __uint_as_float(r[c][i]));
+                const float m_new = fmaxf(m_run, tmax * sl2);
+                // The rescale touches TMEM with warp-collective (.sync.aligned)
+                // loads and stores, so the decision must be uniform across the
+                // warp: if any row's maximum grew by more than 2^8, every row of
+                // the warp moves to its new maximum (factor 1 where it did not grow).
+                if (__any_sync(0xFFFFFFFFu, j == 0 || m_new > m_run + kRescaleLog2)) {
+                    if (j > 0) {
+                        // O_i and l are rescaled to the new maximum (PV_i(j-1) is
+                        // complete: S_i(j) was issued after it).
+                        const float alpha = m_new > m_run ? ex2_approx(m_run - m_new) : 1.f;
+                        l_run *= alpha;
+#pragma unroll 1
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(tO + c * 32, o);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                            tmem_st32(tO + c * 32, o);
+                        }
+                        tmem_st_wait();
+                    }
+                    m_run = m_new;
+                }
+                float rs = 0.f;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c = half * 2 + cc;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            const float p0 =
+                                ((vm[c] >> i) & 1u) ? ex2_approx(__uint_as_float(r[c][i]) * sl2 - m_run) : 0.f;
+                            const float p1 = ((vm[c] >> (i + 1)) & 1u)
+                                                 ? ex2_approx(__uint_as_float(r[c][i + 1]) * sl2 - m_run)
+                                                 : 0.f;
+                            rs += p0 + p1;
+                            pk[cc * 16 + (i >> 1)] = pack_bf16x2(p0, p1);
+                        }
+                    }
+                    tmem_st32(tS + half * 32, pk);  // P columns [32*half, 32*half+32)
+                }
+                tmem_st_wait();
+                l_run += rs;
+                tc_fence_before();
+                mbar_arrive(BAR(B_PF + wg));
+            }
+            if (ok && n_tiles > 0) {
+                if (!__all_sync(0xFFFFFFFFu, WAIT(7 + wg, B_OF + wg, n_tiles, 0))) ok = false;
+            }
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok) {
+                set_err(p.err, DEV_ERR_TIMEOUT);
+            } else {
+                tc_fence_after();
+                const float il = n_tiles > 0 ? 1.f / l_run : 0.f;
+                const bool store = row < valid;
+                const int tok = store ? p.perm_q[unit_row + row0 + wg * BM + row] : 0;
+                uint4 *dst = reinterpret_cast<uint4 *>(p.O + (unit_row + tok) * D);
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + c * 32, o);
+                    tmem_ld_wait();
+                    if (store) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float *f = reinterpret_cast<const float *>(o + 8 * q);
+                            dst[c * 4 + q] = make_uint4(pack_bf16x2(f[0] * il, f[1] * il),
+                                                        pack_bf16x2(f[2] * il, f[3] * il),
+                                                        pack_bf16x2(f[4] * il, f[5] * il),
+                                                        pack_bf16x2(f[6] * il, f[7] * il));
+                        }
+                    }
                 }
             }
-            tc_fence_before();
-            mbar_arrive(BAR(B_SE + b));
-            fence_proxy_async_smem();
-            mbar_arrive(BAR(B_PF + b));
-            l_run = l_run * alpha + rs;
-            m_run = m_new;
-            if (j >= 1 && !accumulate_o<D>(acc, tmem + lane_off, BAR(B_OF + ((j - 1) & 1)),
-                                           BAR(B_OE + ((j - 1) & 1)), j - 1, alpha_prev)) {
-                ok = false;
-                break;
+            if (row == 0 && p.counters) {
+                atomicAdd(&p.counters[0], (unsigned long long)((long long)valid * kept_cols));
+                atomicAdd(&p.counters[1], (unsigned long long)((long long)BM * BN * n_tiles));
+                atomicAdd(&p.counters[2], 1ull);
             }
-            alpha_prev = alpha;
-        }
-        if (ok && n_tiles > 0 &&
-            !accumulate_o<D>(acc, tmem + lane_off, BAR(B_OF + ((n_tiles - 1) & 1)), BAR(B_OE + ((n_tiles - 1) & 1)),
-                             n_tiles - 1, alpha_prev))
-            ok = false;
-        if (!ok) {
-            set_err(p.err, DEV_ERR_TIMEOUT);
-        } else if (row < nvalid) {
-            const float il = n_tiles > 0 ? 1.f / l_run : 0.f;
-            const int tok = p.perm_q[unit_row + row0 + row];
-            uint4 *dst = reinterpret_cast<uint4 *>(p.O + (unit_row + tok) * D);
-#pragma unroll
-            for (int k8 = 0; k8 < D / 8; ++k8)
-                dst[k8] = make_uint4(pack_bf16x2(acc[8 * k8] * il, acc[8 * k8 + 1] * il),
-                                     pack_bf16x2(acc[8 * k8 + 2] * il, acc[8 * k8 + 3] * il),
-                                     pack_bf16x2(acc[8 * k8 + 4] * il, acc[8 * k8 + 5] * il),
-                                     pack_bf16x2(acc[8 * k8 + 6] * il, acc[8 * k8 + 7] * il));
-        }
-        if (tid == 0 && p.counters) {
-            atomicAdd(&p.counters[0], (unsigned long long)((long long)nvalid * kept_cols));
-            atomicAdd(&p.counters[1], (unsigned long long)((long long)BM * BN * n_tiles));
-            atomicAdd(&p.counters[2], 1ull);
         }
     }
+#undef WAIT
 #undef BAR
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -384,7 +440,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 }  // namespace
 
-int attn_max_tiles(int L, int Cq, int BH) { return BH * ((L + BM - 1) / BM + Cq); }
+int attn_max_tiles(int L, int Cq, int BH) { return BH * ((L + 2 * BM - 1) / (2 * BM) + Cq); }
 
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s) {
     AttnParams p;

@@ -109,7 +109,8 @@ __global__ void __launch_bounds__(SEL_THREADS) k_score_select(SelectArgs a) {
     }
 }
 
-// Exclusive prefix of the number of 128-query tiles of every (unit, query cluster).
+// Exclusive prefix of the number of attention work items of every (unit, query
+// cluster): one item per pair of 128-query tiles.
 __global__ void __launch_bounds__(1024) k_tile_prefix(const int *counts_q, int n, int *prefix) {
     typedef cub::BlockScan<int, 1024> Scan;
     __shared__ typename Scan::TempStorage tmp;
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(1024) k_tile_prefix(const int *counts_q, int n
     __syncthreads();
     for (int i0 = 0; i0 < n; i0 += 1024) {
         const int i = i0 + threadIdx.x;
-        const int t = i < n ? (counts_q[i] + 127) / 128 : 0;
+        const int t = i < n ? (counts_q[i] + 255) / 256 : 0;
         int p, tot;
         Scan(tmp).ExclusiveSum(t, p, tot);
         const int base = base_s;

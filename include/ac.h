@@ -226,12 +226,15 @@ AC_API ac_status ac_get_tensor(ac_ctx *ctx, int32_t which, void **dev_ptr, int64
 
 /* Work counters of the last ac_sparse_attn (synchronises the device):
  * kept key tokens summed over queries, the same in computed (padded) tile
- * columns, and the number of 128-query tiles. */
+ * columns, the number of work items (pairs of 128-query tiles), dense units,
+ * and the location of the first in-kernel wait that gave up (0 if none). */
 typedef struct ac_attn_counters {
     int64_t kept_pairs;       /* sum over queries of |K*|                        */
     int64_t computed_pairs;   /* sum over tiles of 128 x computed key columns   */
     int64_t tiles;
     int64_t dense_heads;
+    int64_t wait_failure;     /* 0, or where the first bounded wait gave up:
+                                 1<<60 | role<<24 | barrier<<16 | tile<<1 | parity */
 } ac_attn_counters;
 
 AC_API ac_status ac_get_attn_counters(ac_ctx *ctx, ac_attn_counters *out);
