@@ -77,6 +77,31 @@ ac_status make_tmap(ac_ctx *c, CUtensorMap *tm, void *base, int64_t rows, int d,
     return AC_OK;
 }
 
+// K and V boxes: 8 rows x all d columns in one copy, laid out in shared memory
+// as [column half][8 rows][64 columns] (dims: column, row, half; the half
+// stride is 128 bytes, the row stride d*2 bytes), 128-byte swizzle.
+ac_status make_tmap_kv(ac_ctx *c, CUtensorMap *tm, void *base, int64_t rows, int d) {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+            return fail(c, AC_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    const int halves = d / 64;
+    cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)halves};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, 128};
+    cuuint32_t box[3] = {64, 8, (cuuint32_t)halves};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(c, AC_ERR_CUDA, "cuTensorMapEncodeTiled (K/V boxes) failed");
+    return AC_OK;
+}
+
 template <class T>
 cudaError_t dalloc(T **p, size_t n) {
     return cudaMalloc(reinterpret_cast<void **>(p), std::max<size_t>(n, 1) * sizeof(T));
@@ -419,8 +444,8 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
         return AC_ERR_CUDA;
     }
     const int64_t rows = (int64_t)BH * L;
-    if (make_tmap(c, &c->tm_q, c->Qp, rows, d, 128) != AC_OK || make_tmap(c, &c->tm_k, c->Kp, rows, d, 8) != AC_OK ||
-        make_tmap(c, &c->tm_v, c->Vp, rows, d, 8) != AC_OK) {
+    if (make_tmap(c, &c->tm_q, c->Qp, rows, d, 128) != AC_OK || make_tmap_kv(c, &c->tm_k, c->Kp, rows, d) != AC_OK ||
+        make_tmap_kv(c, &c->tm_v, c->Vp, rows, d) != AC_OK) {
         free_all(c);
         delete c;
         return AC_ERR_CUDA;

@@ -43,17 +43,22 @@ constexpr int NTHREADS = 384;
 constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= NTHREADS * 168, "register split exceeds the launch");
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int RG_CACHE = 2048;  // key ranges kept in shared memory (more: read from global)
+// K/V tile layout in shared memory: 16 boxes, each [column half][8 rows][128 B]
+// (one 3-D TMA copy per box); an 8-row group is BOX_BYTES after the previous.
 
 template <int D>
 struct Layout {
     static constexpr int HALVES = D / 64;  // 128-byte (64 x bf16) column halves
     static constexpr uint32_t Q_TILE = HALVES * BM * 128;
     static constexpr uint32_t KV_BYTES = HALVES * BN * 128;
+    static constexpr uint32_t BOX_BYTES = HALVES * 1024;
     static constexpr uint32_t OFF_Q = 0;                        // two query tiles
     static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_TILE;
     static constexpr uint32_t OFF_V = OFF_K + NS * KV_BYTES;
     static constexpr uint32_t OFF_MASK = OFF_V + NS * KV_BYTES;  // [NS][4] uint32
-    static constexpr uint32_t OFF_BAR = OFF_MASK + 64;
+    static constexpr uint32_t OFF_RG = OFF_MASK + 64;            // [RG_CACHE] int2 key ranges
+    static constexpr uint32_t OFF_BAR = OFF_RG + RG_CACHE * 8;
     static constexpr uint32_t BYTES = OFF_BAR + 256;
     static constexpr uint32_t SMEM = BYTES + 1024;  // 1024-byte alignment slack
 };
@@ -188,6 +193,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       reg_dealloc<kRegsOther>();
       if (warp == 8) {
         // ------------------------------------------------ TMA producer
+        int2 *rg_s = reinterpret_cast<int2 *>(sm + LY::OFF_RG);
+        const bool rg_cached = nr <= RG_CACHE;
+        if (rg_cached)
+            for (int i = lane; i < nr; i += 32) rg_s[i] = rg[i];
+        __syncwarp();
         if (lane == 0) {
             mbar_arrive_expect_tx(BAR(B_QF), 2 * LY::Q_TILE);
             for (int t = 0; t < 2; ++t)
@@ -195,7 +205,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tma_load_2d(sbase + LY::OFF_Q + t * LY::Q_TILE + hf * BM * 128, &tm_q, hf * 64,
                                 (int)(unit_row + row0 + t * BM), BAR(B_QF));
             KeyWalker w;
-            w.init(rg, nr);
+            w.init(rg_cached ? rg_s : rg, nr);
             int issued = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int s = j % NS;
@@ -221,11 +231,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     int st, c;
                     w2.next(st, c);
                     const int row = (int)(unit_row + st);
-#pragma unroll
-                    for (int hf = 0; hf < LY::HALVES; ++hf) {
-                        tma_load_2d(kd + hf * BN * 128 + b * 1024, &tm_k, hf * 64, row, BAR(B_KVF + s));
-                        tma_load_2d(vd + hf * BN * 128 + b * 1024, &tm_v, hf * 64, row, BAR(B_KVF + s));
-                    }
+                    tma_load_3d(kd + b * LY::BOX_BYTES, &tm_k, 0, row, 0, BAR(B_KVF + s));
+                    tma_load_3d(vd + b * LY::BOX_BYTES, &tm_v, 0, row, 0, BAR(B_KVF + s));
                 }
                 ++issued;
             }
@@ -246,9 +253,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const uint32_t ka = sbase + LY::OFF_K + (j % NS) * LY::KV_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                    tc_mma_bf16(tmem + i * BN, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
-                                IQK, kk > 0 ? 1u : 0u);
+                    const uint32_t qoff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                    const uint32_t koff = (kk >> 2) * 1024 + (kk & 3) * 32;
+                    tc_mma_bf16(tmem + i * BN, sdesc_sw128(qa + qoff, 16, 1024),
+                                sdesc_sw128(ka + koff, 16, LY::BOX_BYTES), IQK, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(BAR(B_SF + i));
             };
@@ -257,7 +265,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
                     tc_mma_bf16_ts(tmem + 256 + i * 128, tmem + i * BN + kk * 8,
-                                   sdesc_sw128(va + kk * 16 * 128, BN * 128, 1024), IPV,
+                                   sdesc_sw128(va + kk * 2 * LY::BOX_BYTES, 1024, LY::BOX_BYTES), IPV,
                                    (j > 0 || kk > 0) ? 1u : 0u);
             };
             if (!WAIT(3, B_QF, 0, 0)) ok = false;
@@ -337,12 +345,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, r[c]);
                 tmem_ld_wait();
-                float tmax = -INFINITY;
+                // Masked columns become -inf (the masks are the same for every
+                // row, so the branch is warp-uniform; most chunks are full).
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (vm[c] != 0xFFFFFFFFu) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[c][i] = ((vm[c] >> i) & 1u) ? r[c][i] : 0xFF800000u;
+                    }
+                }
+                // Row maximum with 8 independent partial maxima.
+                float pm[8];
+#pragma unroll
+                for (int a = 0; a < 8; ++a) pm[a] = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if ((vm[c] >> i) & 1u) tmax = fmaxf(tmax, __uint_as_float(r[c][i]));
+                    for (int i = 0; i < 32; ++i) pm[i & 7] = fmaxf(pm[i & 7], __uint_as_float(r[c][i]));
+                const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                         fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
                 const float m_new = fmaxf(m_run, tmax * sl2);
                 // The rescale touches TMEM with warp-collective (.sync.aligned)
                 // loads and stores, so the decision must be uniform across the
@@ -367,7 +388,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     m_run = m_new;
                 }
-                float rs = 0.f;
+                // p = 2^(s * scale * log2(e) - m): one FMA and one ex2 per element;
+                // -inf columns give 0.  Row sum with 8 independent partial sums.
+                const float neg_m = -m_run;
+                float ps[8];
+#pragma unroll
+                for (int a = 0; a < 8; ++a) ps[a] = 0.f;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[32];
@@ -376,17 +402,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const int c = half * 2 + cc;
 #pragma unroll
                         for (int i = 0; i < 32; i += 2) {
-                            const float p0 =
-                                ((vm[c] >> i) & 1u) ? ex2_approx(__uint_as_float(r[c][i]) * sl2 - m_run) : 0.f;
-                            const float p1 = ((vm[c] >> (i + 1)) & 1u)
-                                                 ? ex2_approx(__uint_as_float(r[c][i + 1]) * sl2 - m_run)
-                                                 : 0.f;
-                            rs += p0 + p1;
+                            const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), sl2, neg_m));
+                            const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), sl2, neg_m));
+                            ps[i & 7] += p0;
+                            ps[(i + 1) & 7] += p1;
                             pk[cc * 16 + (i >> 1)] = pack_bf16x2(p0, p1);
                         }
                     }
                     tmem_st32(tS + half * 32, pk);  // P columns [32*half, 32*half+32)
                 }
+                const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 tmem_st_wait();
                 l_run += rs;
                 tc_fence_before();
