@@ -69,6 +69,12 @@ class ACAttnCounters(ctypes.Structure):
                 ("wait_failure", ctypes.c_int64)]
 
 
+class ACAssignCounters(ctypes.Structure):
+    _fields_ = [("tensor_passes", ctypes.c_int64), ("exact_passes", ctypes.c_int64),
+                ("rows", ctypes.c_int64), ("uncertain_rows", ctypes.c_int64),
+                ("full_rescore_rows", ctypes.c_int64)]
+
+
 # every function that include/ac.h declares, with its ctypes signature
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -86,6 +92,7 @@ SIGNATURES = {
     "ac_get_tensor": (_I, [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int64)]),
     "ac_get_attn_counters": (_I, [_P, ctypes.POINTER(ACAttnCounters)]),
     "ac_get_launch_count": (_I, [ctypes.POINTER(ctypes.c_int64)]),
+    "ac_get_assign_counters": (_I, [_P, ctypes.POINTER(ACAssignCounters), _I]),
     "ac_cluster_q_noalloc": (_I, [_P, _I, _I, _I, _I, _I, ctypes.c_uint64, _P, _P, _P, _P]),
     "ac_state_export": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int64)]),
     "ac_state_import": (_I, [_P, _P, ctypes.c_int64]),

@@ -139,6 +139,12 @@ class SparseLayer:
         check(self.lib.ac_get_attn_counters(self.ctx, ctypes.byref(c)), self.ctx)
         return {f: int(getattr(c, f)) for f, _ in c._fields_}
 
+    def assign_counters(self, reset: bool = False) -> dict:
+        """Tensor-core / exact assignment passes and rows rescored exactly."""
+        c = _lib.ACAssignCounters()
+        check(self.lib.ac_get_assign_counters(self.ctx, ctypes.byref(c), 1 if reset else 0), self.ctx)
+        return {f: int(getattr(c, f)) for f, _ in c._fields_}
+
     def export_state(self) -> bytes:
         n = ctypes.c_int64(0)
         check(self.lib.ac_state_export(self.ctx, None, ctypes.byref(n)), self.ctx)

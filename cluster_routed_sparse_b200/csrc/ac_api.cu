@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -114,8 +115,8 @@ ac_status check_dev_err(ac_ctx *c, cudaStream_t s) {
     uint32_t e = *c->h_err;
     if (e) {
         CK(cudaMemsetAsync(c->err, 0, sizeof(uint32_t), s), "error word reset");
-        if (e & DEV_ERR_TIMEOUT) return fail(c, AC_ERR_TIMEOUT, "a bounded in-kernel wait expired");
         if (e & DEV_ERR_NONFINITE) return fail(c, AC_ERR_NONFINITE, "non-finite value in an input");
+        if (e & DEV_ERR_TIMEOUT) return fail(c, AC_ERR_TIMEOUT, "a bounded in-kernel wait expired");
         return fail(c, AC_ERR_CUDA, "kernel bounds check failed");
     }
     return AC_OK;
@@ -127,18 +128,76 @@ struct Lloyd {
     AssignArgs as;
     SortArgs so;
     UpdateArgs up;
+    bool fast = false;  // assignment on the tensor cores (fa) instead of the exact kernel (as)
+    FastAssignArgs fa;
 };
 
-cudaError_t run_lloyd(Lloyd &k, int T, bool final_sort, cudaStream_t s) {
+// One assignment pass; dmin (where the caller asked for it) only when wanted.
+cudaError_t assign_pass(ac_ctx *c, const Lloyd &k, bool want_dmin, cudaStream_t s) {
+    if (k.fast) {
+        FastAssignArgs a = k.fa;
+        if (!want_dmin) a.dmin = nullptr;
+        ++c->n_fast;
+        c->n_fast_rows += (long long)a.BH * a.L;
+        return launch_assign_fast(a, s);
+    }
+    ++c->n_exact;
+    return launch_assign_exact(k.as, s);
+}
+
+cudaError_t run_lloyd(ac_ctx *c, Lloyd &k, int T, bool final_sort, cudaStream_t s) {
     cudaError_t e;
     for (int t = 0; t < T; ++t) {
-        if ((e = launch_assign_exact(k.as, s)) != cudaSuccess) return e;
+        if ((e = assign_pass(c, k, false, s)) != cudaSuccess) return e;
         if ((e = launch_counting_sort(k.so, s)) != cudaSuccess) return e;
         if ((e = launch_update(k.up, s)) != cudaSuccess) return e;
     }
-    if ((e = launch_assign_exact(k.as, s)) != cudaSuccess) return e;
+    if ((e = assign_pass(c, k, true, s)) != cudaSuccess) return e;
     if (final_sort && (e = launch_counting_sort(k.so, s)) != cudaSuccess) return e;
     return cudaSuccess;
+}
+
+// Tensor-core assignment of all rows 0..L-1 of every unit against the unit's
+// centres 0..m-1 at C + h * cstride (see assign_mma.cu).  Returns false (exact
+// kernel instead) when disabled or when the rows are not 16-byte aligned.
+bool make_fast(ac_ctx *c, Lloyd &k, const bf16 *X, bool queries, const float *C, int64_t cstride,
+               const int *ncent, int ncent_const, int *labels, float *dmin) {
+    if (!c->fast_assign || (reinterpret_cast<uintptr_t>(X) & 15u) != 0) return false;
+    CUtensorMap *tmx = queries ? &c->tm_xq : &c->tm_xk;
+    if (make_tmap(c, tmx, const_cast<bf16 *>(X), (int64_t)c->BH * c->L, c->d, 128) != AC_OK) return false;
+    FastAssignArgs &a = k.fa;
+    a.tm_x = tmx;
+    a.tm_c = queries ? &c->tm_chi_q : &c->tm_chi_k;
+    a.X = X;
+    a.inv = queries ? c->inv_q : nullptr;
+    a.rowsq = queries ? nullptr : c->rowsq_k;
+    a.L = c->L;
+    a.nrows = nullptr;
+    a.nrows_const = c->L;
+    a.C = C;
+    a.cstride = cstride;
+    a.ncent = ncent;
+    a.ncent_const = ncent_const;
+    a.Cpad = queries ? c->Cpad_q : c->Cpad_k;
+    a.CH = queries ? c->CH_q : c->CH_k;
+    a.Chi = queries ? c->chi_q : c->chi_k;
+    // Normalised queries sit in tight angular clusters (distances ~1e-2 of
+    // |x|^2): c_hi alone would leave most rows to the exact rescoring.
+    a.two_term = queries;
+    a.cn = c->cn;
+    a.hstat = c->hstat;
+    a.labels = labels;
+    a.dmin = dmin;
+    a.cand = c->cand;
+    a.amb_list = c->amb_list;
+    a.amb_count = c->amb_count;
+    a.stats = c->asg_stats;
+    a.err = c->err;
+    a.BH = c->BH;
+    a.d = c->d;
+    a.num_sms = c->num_sms;
+    k.fast = true;
+    return true;
 }
 
 // Algorithm 3 line 3 on the context's buffers.
@@ -161,7 +220,8 @@ ac_status cluster_q_impl(ac_ctx *c, const bf16 *Q, const float *init, int iters,
                     c->counts_q, c->Cq, c->BH};
     k.up = UpdateArgs{Q, c->inv_q, L, nullptr, c->perm_q, c->offs_q, c->Cq + 1, c->cent_q,
                       (int64_t)c->Cq * c->d, nullptr, nullptr, c->Cq, c->BH, c->d, c->Cq};
-    CK(run_lloyd(k, iters, true, s), "q lloyd");
+    make_fast(c, k, Q, true, c->cent_q, (int64_t)c->Cq * c->d, nullptr, c->Cq, c->labels_q, nullptr);
+    CK(run_lloyd(c, k, iters, true, s), "q lloyd");
     c->have_q = true;
     return AC_OK;
 }
@@ -172,6 +232,7 @@ ac_status cluster_q_impl(ac_ctx *c, const bf16 *Q, const float *init, int iters,
 ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
     const int BH = c->BH, L = c->L, d = c->d, m0 = c->cfg.m0;
     const int64_t cstride = (int64_t)c->Ccap * d;
+    if (c->fast_assign) CK(launch_row_sqnorm(K, (int64_t)BH * L, d, c->rowsq_k, s), "row norms");
     CK(launch_iota_rows(c->u_idx, c->u_cnt, BH, L, s), "iota");
     CK(cudaMemsetAsync(c->removed_stage, 0xFF, sizeof(int) * BH * (size_t)L, s), "removed init");
     CK(cudaMemsetAsync(c->tau_acc, 0, sizeof(unsigned long long), s), "tau acc");
@@ -224,7 +285,9 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
                         0, BH};
         k.up = UpdateArgs{K, nullptr, L, c->u_idx, c->st_perm, c->st_offs, m0 + 1, c->cent_k, cstride, c->n_k,
                           c->st_m, 0, BH, d, max_m};
-        CK(run_lloyd(k, c->cfg.iters_k, false, s), "k stage lloyd");
+        // stage 0: U is every key in order and the stage's centres start at 0
+        if (t == 0) make_fast(c, k, K, false, c->cent_k, cstride, c->st_m, 0, c->st_labels, c->dmin_k);
+        CK(run_lloyd(c, k, c->cfg.iters_k, false, s), "k stage lloyd");
         // line 14: d_i = ||k_i - c(k_i)||
         CK(launch_stage_dist(c->dmin_k, c->st_dist, c->u_cnt, c->st_m, L, BH, t == 0 ? c->tau_acc : nullptr, s),
            "stage dist");
@@ -255,9 +318,11 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
     CK(cudaMemcpyAsync(c->stages, c->h_st_m, sizeof(int) * BH, cudaMemcpyHostToDevice, s), "stages");
     CK(cudaStreamSynchronize(s), "stage end sync");  // the staging buffers are reused by the next call
     // line 22: every key to its closest centre among all of C
-    AssignArgs fa{K, nullptr, L, nullptr, nullptr, L, c->cent_k, cstride, nullptr, c->n_k, 0, c->labels_k,
-                  c->dmin_k, BH, d};
-    CK(launch_assign_exact(fa, s), "final assign");
+    Lloyd fin;
+    fin.as = AssignArgs{K, nullptr, L, nullptr, nullptr, L, c->cent_k, cstride, nullptr, c->n_k, 0, c->labels_k,
+                        c->dmin_k, BH, d};
+    make_fast(c, fin, K, false, c->cent_k, cstride, c->n_k, 0, c->labels_k, c->dmin_k);
+    CK(assign_pass(c, fin, true, s), "final assign");
     return AC_OK;
 }
 
@@ -271,6 +336,7 @@ __global__ void k_warm_counts(const int *n_k, const uint8_t *dense, int *ncent, 
 ac_status cluster_k_warm(ac_ctx *c, const bf16 *K, cudaStream_t s) {
     const int BH = c->BH, L = c->L, d = c->d;
     const int64_t cstride = (int64_t)c->Ccap * d;
+    if (c->fast_assign) CK(launch_row_sqnorm(K, (int64_t)BH * L, d, c->rowsq_k, s), "row norms");
     k_warm_counts<<<(BH + 127) / 128, 128, 0, s>>>(c->n_k, c->dense, c->st_m, BH);
     AC_NOTE_LAUNCH();
     CK(cudaGetLastError(), "warm counts");
@@ -281,7 +347,8 @@ ac_status cluster_k_warm(ac_ctx *c, const bf16 *K, cudaStream_t s) {
                     c->Ccap, BH};
     k.up = UpdateArgs{K, nullptr, L, nullptr, c->perm_k, c->offs_k, c->Ccap + 1, c->cent_k, cstride, nullptr,
                       c->st_m, 0, BH, d, c->Ccap};
-    CK(run_lloyd(k, c->cfg.iters_warm, false, s), "warm lloyd");
+    make_fast(c, k, K, false, c->cent_k, cstride, c->st_m, 0, c->labels_k, c->dmin_k);
+    CK(run_lloyd(c, k, c->cfg.iters_warm, false, s), "warm lloyd");
     return AC_OK;
 }
 
@@ -325,7 +392,8 @@ void free_all(ac_ctx *c) {
                    c->perm_k, c->offs_k, c->kmax, c->kmin, c->sse, c->mse, c->comp, c->u_idx, c->u_idx2,
                    c->u_cnt, c->st_m, c->st_labels, c->st_dist, c->st_perm, c->st_offs, c->st_counts, c->radix,
                    c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->Qp, c->Kp, c->Vp,
-                   c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err};
+                   c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err, c->chi_q, c->chi_k, c->cn,
+                   c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats};
     for (void *p : dev)
         if (p) cudaFree(p);
     void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err};
@@ -378,6 +446,15 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     c->device = dev;
     c->scale = cfg->scale > 0.f ? cfg->scale : 1.0f / std::sqrt((float)d);
 
+    c->num_sms = prop.multiProcessorCount;
+    {
+        const char *ev = std::getenv("AC_EXACT_ASSIGN");
+        c->fast_assign = !(ev && ev[0] == '1');
+    }
+    c->Cpad_q = (c->Cq + 31) & ~31;
+    c->CH_q = std::min(128, c->Cpad_q);  // two-term chunks
+    c->Cpad_k = (c->Ccap + 31) & ~31;
+    c->CH_k = std::min(256, c->Cpad_k);
     const size_t BH = c->BH, Lz = L, dz = d, Cq = c->Cq, Cc = c->Ccap, m0 = cfg->m0;
     bool okm = true;
     auto A = [&](cudaError_t e) { okm = okm && e == cudaSuccess; };
@@ -420,6 +497,15 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->ranges, BH * Cq * Cc));
     A(dalloc(&c->nboxes, BH * Cq));
     A(dalloc(&c->tile_prefix, BH * Cq + 1));
+    A(dalloc(&c->chi_q, 2 * BH * c->Cpad_q * dz));
+    A(dalloc(&c->chi_k, BH * c->Cpad_k * dz));
+    A(dalloc(&c->cn, BH * std::max(c->Cpad_q, c->Cpad_k)));
+    A(dalloc(&c->hstat, 2 * BH));
+    A(dalloc(&c->rowsq_k, BH * Lz));
+    A(dalloc(&c->cand, BH * Lz));
+    A(dalloc(&c->amb_list, BH * Lz));
+    A(dalloc(&c->amb_count, 1));
+    A(dalloc(&c->asg_stats, 2));
     A(dalloc(&c->Qp, BH * Lz * dz));
     A(dalloc(&c->Kp, BH * Lz * dz));
     A(dalloc(&c->Vp, BH * Lz * dz));
@@ -438,6 +524,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
         return AC_ERR_WORKSPACE;
     }
     if (cudaMemset(c->err, 0, sizeof(uint32_t)) != cudaSuccess ||
+        cudaMemset(c->asg_stats, 0, 2 * sizeof(unsigned long long)) != cudaSuccess ||
         cudaMemset(c->dense, 0, BH) != cudaSuccess || cudaMemset(c->n_k, 0, BH * sizeof(int)) != cudaSuccess) {
         free_all(c);
         delete c;
@@ -445,7 +532,9 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     }
     const int64_t rows = (int64_t)BH * L;
     if (make_tmap(c, &c->tm_q, c->Qp, rows, d, 128) != AC_OK || make_tmap_kv(c, &c->tm_k, c->Kp, rows, d) != AC_OK ||
-        make_tmap_kv(c, &c->tm_v, c->Vp, rows, d) != AC_OK) {
+        make_tmap_kv(c, &c->tm_v, c->Vp, rows, d) != AC_OK ||
+        make_tmap(c, &c->tm_chi_q, c->chi_q, (int64_t)2 * BH * c->Cpad_q, d, c->CH_q) != AC_OK ||
+        make_tmap(c, &c->tm_chi_k, c->chi_k, (int64_t)BH * c->Cpad_k, d, c->CH_k) != AC_OK) {
         free_all(c);
         delete c;
         return AC_ERR_CUDA;
@@ -493,8 +582,16 @@ ac_status ac_cluster_k_multistage(ac_ctx *c, const uint16_t *K, const float *war
         if (warm_cent != c->cent_k)
             CK(cudaMemcpyAsync(c->cent_k, warm_cent, sizeof(float) * BH * c->Ccap * c->d, cudaMemcpyDeviceToDevice, s),
                "warm centres");
-        if (warm_n_k != c->n_k)
+        if (warm_n_k != c->n_k) {
+            // the counts index the centre arrays: check them before any kernel uses them
+            std::vector<int32_t> nk(BH);
+            CK(cudaMemcpyAsync(nk.data(), warm_n_k, sizeof(int) * BH, cudaMemcpyDeviceToHost, s), "warm counts");
+            CK(cudaStreamSynchronize(s), "warm counts");
+            for (size_t h = 0; h < BH; ++h)
+                if (nk[h] < 0 || nk[h] > c->Ccap)
+                    return fail(c, AC_ERR_INVALID_ARG, "warm cluster count out of range [0, n_max + m0]");
             CK(cudaMemcpyAsync(c->n_k, warm_n_k, sizeof(int) * BH, cudaMemcpyDeviceToDevice, s), "warm counts");
+        }
         if (warm_dense) {
             if (warm_dense != c->dense)
                 CK(cudaMemcpyAsync(c->dense, warm_dense, BH, cudaMemcpyDeviceToDevice, s), "warm dense");
@@ -652,6 +749,23 @@ ac_status ac_synchronize(ac_ctx *c, void *stream) {
     return check_dev_err(c, (cudaStream_t)stream);
 }
 
+ac_status ac_get_assign_counters(ac_ctx *c, ac_assign_counters *out, int32_t reset) {
+    if (!c || !out) return AC_ERR_INVALID_ARG;
+    unsigned long long h[2];
+    CK(cudaDeviceSynchronize(), "sync");
+    CK(cudaMemcpy(h, c->asg_stats, sizeof(h), cudaMemcpyDeviceToHost), "assign counters");
+    out->tensor_passes = c->n_fast;
+    out->exact_passes = c->n_exact;
+    out->rows = c->n_fast_rows;
+    out->uncertain_rows = (int64_t)h[0];
+    out->full_rescore_rows = (int64_t)h[1];
+    if (reset) {
+        CK(cudaMemset(c->asg_stats, 0, sizeof(h)), "assign counters reset");
+        c->n_fast = c->n_exact = c->n_fast_rows = 0;
+    }
+    return AC_OK;
+}
+
 ac_status ac_get_attn_counters(ac_ctx *c, ac_attn_counters *out) {
     if (!c || !out) return AC_ERR_INVALID_ARG;
     unsigned long long h[8];
@@ -720,6 +834,12 @@ ac_status ac_state_import(ac_ctx *c, const void *host_buf, int64_t bytes) {
     const size_t BH = c->BH;
     const size_t sz_q = BH * c->Cq * c->d * 4, sz_k = BH * c->Ccap * c->d * 4, sz_n = BH * 4, sz_f = BH,
                  sz_l = BH * c->L * 4;
+    {
+        const int32_t *nk = reinterpret_cast<const int32_t *>(reinterpret_cast<const uint8_t *>(host_buf) + 64 +
+                                                              sz_q + sz_k);
+        for (size_t h = 0; h < BH; ++h)
+            if (nk[h] < 0 || nk[h] > c->Ccap) return fail(c, AC_ERR_INVALID_ARG, "state: cluster count out of range");
+    }
     CK(cudaDeviceSynchronize(), "sync");
     const uint8_t *p = reinterpret_cast<const uint8_t *>(host_buf) + 64;
     CK(cudaMemcpy(c->cent_q, p, sz_q, cudaMemcpyHostToDevice), "import");

@@ -64,6 +64,22 @@ struct ac_ctx {
     int *nboxes;       // [BH*Cq]         8-row key boxes per query cluster
     int *tile_prefix;  // [BH*Cq+1]       attention items (pairs of 128-query tiles), exclusive prefix
 
+    // ---- tensor-core assignment (centres split into bf16 + remainder)
+    int Cpad_q, CH_q, Cpad_k, CH_k;  // padded centre rows per unit, centres per chunk
+    bf16 *chi_q, *chi_k;  // [2, BH, Cpad_q, d] c_hi, c_lo of the query centres; [BH, Cpad_k, d] c_hi of the key centres
+    float *cn;         // [BH, max Cpad] |c_hi|^2
+    unsigned int *hstat;  // [BH, 2]
+    float *rowsq_k;    // [BH, L] |k|^2
+    int4 *cand;        // [BH * L] candidates of uncertain rows
+    int *amb_list;     // [BH * L]
+    int *amb_count;    // [1]
+    unsigned long long *asg_stats;  // [2] uncertain rows, rows rescored against every centre
+    CUtensorMap tm_chi_q, tm_chi_k;
+    CUtensorMap tm_xq, tm_xk;  // caller's Q / K of the current call
+    int num_sms;
+    bool fast_assign;
+    long long n_fast, n_exact, n_fast_rows;
+
     // ---- attention
     bf16 *Qp, *Kp, *Vp;  // [BH, L, d] cluster-order copies
     unsigned long long *counters;  // [8] kept pairs, computed pairs, items, -, first wait failure
@@ -118,6 +134,31 @@ struct AssignArgs {
     int BH, d;
 };
 cudaError_t launch_assign_exact(const AssignArgs &a, cudaStream_t s);
+
+// The same labels from the tensor cores (see assign_mma.cu): rows 0..n-1 of
+// every unit, centres 0..m-1 of the unit at C + h * cstride.
+struct FastAssignArgs {
+    const CUtensorMap *tm_x;   // rows [BH * L, d], box {64, 128}
+    const CUtensorMap *tm_c;   // Chi rows [BH * Cpad (x2 with two terms), d], box {64, CH}
+    const bf16 *X;
+    const float *inv;          // [BH, L] or null
+    const float *rowsq;        // [BH, L] |x|^2 when inv is null
+    int64_t L;
+    const int *nrows; int nrows_const;
+    const float *C; int64_t cstride;
+    const int *ncent; int ncent_const;
+    int Cpad, CH;              // CH <= 256, <= 128 with two terms
+    bool two_term;             // centres as bf16 c_hi + c_lo (else c_hi alone)
+    bf16 *Chi; float *cn; unsigned int *hstat;
+    int *labels;
+    float *dmin;               // or null
+    int4 *cand; int *amb_list; int *amb_count;
+    unsigned long long *stats;
+    uint32_t *err;
+    int BH, d, num_sms;
+};
+cudaError_t launch_assign_fast(const FastAssignArgs &a, cudaStream_t s);
+cudaError_t launch_row_sqnorm(const bf16 *X, int64_t rows, int d, float *out, cudaStream_t s);
 
 // Stable counting sort of labels per unit: perm[h, pos] = row position (or
 // rows[pos]'s index when rows given, see below), offs[h, 0..m], counts[h, 0..m).

@@ -1,0 +1,634 @@
+// assign_mma.cu -- k-means assignment on tcgen05 tensor cores with exact
+// decisions (AdaCluster, arXiv 2604.18348: Sec. 3.1 angular k-means of the
+// queries; Sec. 3.2.2, Algorithm 1 and the warm-started k-means of the keys).
+//
+// The label of a row x is argmin_c D(x, c), D the fp32 squared distance summed
+// in dimension order, ties to the lowest c.  Evaluating every D that way costs
+// three dependent fp32 operations per (row, centre, dimension) on CUDA cores.
+// Here instead:
+//   1. each centre is represented as c' = c_hi (+ c_lo) with c_hi = bf16(c)
+//      (and c_lo = bf16(c - c_hi) where the pass asks for two terms); the
+//      tensor cores form s = x . c' for every centre (key rows are exact bf16;
+//      query rows are scaled by their fp32 inverse norm afterwards);
+//   2. the epilogue keeps per row the 4 smallest A(c) = |c'|^2 - 2 s, the
+//      squared distance to c' less the row's own |x|^2;
+//   3. a rigorous bound E on |D(x, c) - |x|^2 - A(c)| (bf16 split, tensor-core
+//      accumulation, the fp32 rounding of D itself; see assign_bound) decides:
+//      when every other centre's lower bound A - E lies above the best's upper
+//      bound, the best is the exact argmin; otherwise the row's candidates (or,
+//      rarely, all centres) are rescored with the exact arithmetic.
+// The labels are therefore those of the exact definition.  dmin, where used,
+// is recomputed exactly for the chosen centre.
+#include "ac_device.cuh"
+#include "ac_internal.h"
+
+namespace ac {
+namespace {
+
+constexpr int AM = 128;       // rows per tile (MMA M)
+constexpr int ACH_MAX = 256;  // centres per chunk (MMA N at most; 128 with two terms)
+constexpr int A_EPI = 256;    // epilogue threads: two warpgroups
+constexpr int A_THREADS = A_EPI + 64;
+
+template <int D>
+struct ALayout {
+    static constexpr int HALVES = D / 64;
+    static constexpr uint32_t X_BYTES = HALVES * AM * 128;        // one row tile
+    static constexpr uint32_t C_BYTES = HALVES * ACH_MAX * 128;   // one centre chunk (c_hi [, c_lo])
+    static constexpr uint32_t OFF_X = 0;                           // [2] row tiles
+    static constexpr uint32_t OFF_C = OFF_X + 2 * X_BYTES;         // [2] centre chunks
+    static constexpr uint32_t OFF_MG = OFF_C + 2 * C_BYTES;        // [2][AM][8] top-4 hand-over
+    static constexpr uint32_t OFF_BAR = OFF_MG + 2 * AM * 8 * 4;
+    static constexpr uint32_t BYTES = OFF_BAR + 256;
+    static constexpr uint32_t SMEM = BYTES + 1024;
+};
+
+// barriers
+enum {
+    B_XF = 0,   // [2] row tile landed
+    B_XE = 2,   // [2] row tile consumed by the MMAs
+    B_CF = 4,   // [2] centre chunk landed
+    B_CE = 6,   // [2] centre chunk consumed
+    B_AF = 8,   // [2] accumulator chunk ready
+    B_AE = 10,  // [2] accumulator chunk drained (256 arrivals)
+    B_MG = 12,  // [2] upper warpgroup's top-4 written (128 arrivals)
+    B_MR = 14,  // [2] hand-over slot read (128 arrivals)
+    B_DONE = 16,
+    B_N = 17
+};
+
+struct AsgParams {
+    const float *inv;     // [BH, L] (queries) or null
+    const float *rowsq;   // [BH, L] |x|^2 (keys) or null (normalised rows: 1)
+    const float *cn;      // [BH, Cpad]
+    const unsigned int *hstat;  // [BH, 2] max delta, max |c_hi|^2 (float bits)
+    const int *nrows; int nrows_const;
+    const int *ncent; int ncent_const;
+    int64_t L;
+    int BH, Cpad, CH, tiles_per_unit;
+    int two_term;         // c' = c_hi + c_lo (else c_hi)
+    float e_tc;           // tensor-core error coefficient (see assign_bound)
+    int *labels;
+    int4 *cand;
+    int *amb_list, *amb_count;
+    unsigned long long *stats;  // [0] ambiguous rows, [1] rows rescored against every centre
+    uint32_t *err;
+};
+
+// Upper bound of |D(x, c) - |x|^2 - A(c)| for a centre with A(c) = a.
+//   dup   = max(a + |x|^2, 0) + 2 e  bounds |x - c'|^2 (e covers the error
+//           of a: the tensor core's fp32 accumulation of the n products --
+//           allowed two units in the last place per addition, twice the
+//           round-to-nearest bound, so n 2^-23 (|x|^2 + |c'|^2) --, the query
+//           scaling and the roundings of |c'|^2 and of a);
+//   |x - c|^2 - |x - c'|^2 is at most 2 sqrt(dup) delta + delta^2 (triangle
+//   inequality, delta = max |c - c'|);
+//   D itself, d products and d - 1 sums in fp32, is within (d + 2) 2^-24 of
+//   |x - c|^2 <= (sqrt(dup) + delta)^2; 2^-16 covers d <= 128.
+// The result is widened by 2^-10 of itself plus 2^-20 of the magnitudes for
+// the rounding of this fp32 evaluation and of the comparisons.
+__device__ __forceinline__ float assign_bound(float a, float sq, float delta, float e) {
+    const float dup = fmaxf(a + sq, 0.f) + 2.f * e;
+    const float r = sqrtf(dup);
+    const float split = (2.f * r + delta) * delta;
+    const float rr = r + delta;
+    const float b = split + e + 1.52587890625e-05f * rr * rr + 9.5367431640625e-07f * (fabsf(a) + sq);
+    return b * 1.0009765625f;
+}
+
+__device__ __forceinline__ void top4_insert(float v, int c, float &d1, float &d2, float &d3, float &d4, int &i1,
+                                            int &i2, int &i3, int &i4) {
+    if (v < d4) {
+        if (v < d3) {
+            d4 = d3;
+            i4 = i3;
+            if (v < d2) {
+                d3 = d2;
+                i3 = i2;
+                if (v < d1) {
+                    d2 = d1;
+                    i2 = i1;
+                    d1 = v;
+                    i1 = c;
+                } else {
+                    d2 = v;
+                    i2 = c;
+                }
+            } else {
+                d3 = v;
+                i3 = c;
+            }
+        } else {
+            d4 = v;
+            i4 = c;
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(A_THREADS, 1)
+    k_assign_mma(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_c,
+                 const AsgParams p) {
+    using LY = ALayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t bar0 = sbase + LY::OFF_BAR;
+#define ABAR(i) (bar0 + 8u * (uint32_t)(i))
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + LY::OFF_BAR + 8 * B_N);
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(ABAR(B_XF + i), 1);
+            mbar_init(ABAR(B_XE + i), 1);
+            mbar_init(ABAR(B_CF + i), 1);
+            mbar_init(ABAR(B_CE + i), 1);
+            mbar_init(ABAR(B_AF + i), 1);
+            mbar_init(ABAR(B_AE + i), A_EPI);
+            mbar_init(ABAR(B_MG + i), 128);
+            mbar_init(ABAR(B_MR + i), 128);
+        }
+        mbar_init(ABAR(B_DONE), 1);
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int ntiles = p.BH * p.tiles_per_unit;
+    bool ok = true;
+
+    if (warp == 8) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t g = 0, tc = 0;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                const int h = t / p.tiles_per_unit, rt = t % p.tiles_per_unit;
+                const int n = p.nrows ? p.nrows[h] : p.nrows_const;
+                const int m = p.ncent ? p.ncent[h] : p.ncent_const;
+                if (rt * AM >= n || m <= 0) continue;
+                const uint32_t xs = tc & 1;
+                if (tc >= 2 && !mbar_wait_or_abort(ABAR(B_XE + xs), ((tc >> 1) - 1) & 1, p.err)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(ABAR(B_XF + xs), LY::X_BYTES);
+                for (int hf = 0; hf < LY::HALVES; ++hf)
+                    tma_load_2d(sbase + LY::OFF_X + xs * LY::X_BYTES + hf * AM * 128, &tm_x, hf * 64,
+                                (int)(h * p.L + rt * AM), ABAR(B_XF + xs));
+                ++tc;
+                const int nch = (m + p.CH - 1) / p.CH;
+                for (int ch = 0; ch < nch; ++ch, ++g) {
+                    const uint32_t s = g & 1;
+                    if (g >= 2 && !mbar_wait_or_abort(ABAR(B_CE + s), ((g >> 1) - 1) & 1, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t terms = p.two_term ? 2u : 1u;
+                    mbar_arrive_expect_tx(ABAR(B_CF + s), terms * LY::HALVES * p.CH * 128);
+                    for (int hf = 0; hf < LY::HALVES; ++hf)
+                        tma_load_2d(sbase + LY::OFF_C + s * LY::C_BYTES + hf * p.CH * 128, &tm_c, hf * 64,
+                                    h * p.Cpad + ch * p.CH, ABAR(B_CF + s));
+                    if (p.two_term)  // c_lo rows follow c_hi rows in the tensor map
+                        for (int hf = 0; hf < LY::HALVES; ++hf)
+                            tma_load_2d(sbase + LY::OFF_C + s * LY::C_BYTES + (LY::HALVES + hf) * p.CH * 128, &tm_c,
+                                        hf * 64, (p.BH + h) * p.Cpad + ch * p.CH, ABAR(B_CF + s));
+                }
+            }
+            // nothing may still be landing in shared memory when the block exits
+            for (uint32_t k = (g >= 2 ? g - 2 : 0); k < g; ++k) mbar_wait(ABAR(B_CF + (k & 1)), (k >> 1) & 1);
+            for (uint32_t k = (tc >= 2 ? tc - 2 : 0); k < tc; ++k) mbar_wait(ABAR(B_XF + (k & 1)), (k >> 1) & 1);
+            if (!ok) set_err(p.err, DEV_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t g = 0, tc = 0;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                const int h = t / p.tiles_per_unit, rt = t % p.tiles_per_unit;
+                const int n = p.nrows ? p.nrows[h] : p.nrows_const;
+                const int m = p.ncent ? p.ncent[h] : p.ncent_const;
+                if (rt * AM >= n || m <= 0) continue;
+                const uint32_t xs = tc & 1;
+                if (!mbar_wait_or_abort(ABAR(B_XF + xs), (tc >> 1) & 1, p.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t xa = sbase + LY::OFF_X + xs * LY::X_BYTES;
+                const int nch = (m + p.CH - 1) / p.CH;
+                for (int ch = 0; ch < nch; ++ch, ++g) {
+                    const uint32_t s = g & 1;
+                    if (!mbar_wait_or_abort(ABAR(B_CF + s), (g >> 1) & 1, p.err) ||
+                        (g >= 2 && !mbar_wait_or_abort(ABAR(B_AE + s), ((g >> 1) - 1) & 1, p.err))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int rem = m - ch * p.CH;
+                    const int N = rem >= p.CH ? p.CH : ((rem + 31) & ~31);
+                    const uint32_t idesc = idesc_bf16_f32(AM, N, false);
+                    const uint32_t ca = sbase + LY::OFF_C + s * LY::C_BYTES;
+                    const int nk = (p.two_term ? 2 : 1) * (D / 16);
+                    for (int kk = 0; kk < nk; ++kk) {
+                        const int kx = kk % (D / 16);  // x . c_hi, then x . c_lo
+                        const uint32_t xoff = (kx >> 2) * (AM * 128) + (kx & 3) * 32;
+                        const uint32_t coff = (kk >> 2) * (p.CH * 128) + (kk & 3) * 32;
+                        tc_mma_bf16(tmem + s * ACH_MAX, sdesc_sw128(xa + xoff, 16, 1024),
+                                    sdesc_sw128(ca + coff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(ABAR(B_AF + s));
+                    tc_commit(ABAR(B_CE + s));
+                }
+                if (!ok) break;
+                tc_commit(ABAR(B_XE + xs));
+                ++tc;
+            }
+            tc_commit(ABAR(B_DONE));
+            if (!mbar_wait(ABAR(B_DONE), 0)) ok = false;
+            if (!ok) set_err(p.err, DEV_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue
+        // Warpgroup wg takes the 32-column groups wg, wg + 2, ... of every
+        // chunk; warp w reads tensor-memory lanes 32 (w % 4) .. + 31, i.e. rows.
+        const int wg = warp >> 2;
+        const int rloc = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        float *mg = reinterpret_cast<float *>(sm + LY::OFF_MG);
+        uint32_t g = 0, tc = 0;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const int h = t / p.tiles_per_unit, rt = t % p.tiles_per_unit;
+            const int n = p.nrows ? p.nrows[h] : p.nrows_const;
+            const int m = p.ncent ? p.ncent[h] : p.ncent_const;
+            if (rt * AM >= n || m <= 0) continue;
+            const int row = rt * AM + rloc;
+            const bool valid = row < n;
+            const int64_t f = (int64_t)h * p.L + row;
+            const float inv = p.inv ? (valid ? p.inv[f] : 0.f) : 1.f;
+            const float m2i = -2.f * inv;
+            const float *cnh = p.cn + (int64_t)h * p.Cpad;
+            float d1 = INFINITY, d2 = INFINITY, d3 = INFINITY, d4 = INFINITY;
+            int i1 = 0, i2 = -1, i3 = -1, i4 = -1;
+            const int nch = (m + p.CH - 1) / p.CH;
+            for (int ch = 0; ch < nch; ++ch, ++g) {
+                const uint32_t s = g & 1;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(ABAR(B_AF + s), (g >> 1) & 1, p.err))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int rem = m - ch * p.CH;
+                const int N = rem >= p.CH ? p.CH : ((rem + 31) & ~31);
+                for (int cg = wg * 32; cg < N; cg += 64) {
+                    // |c'|^2 of these 32 centres (same address in every lane: one
+                    // broadcast load each; +inf past the last centre)
+                    float4 cnq[8];
+                    const float4 *cn4 = reinterpret_cast<const float4 *>(cnh + ch * p.CH + cg);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) cnq[q] = __ldg(cn4 + q);
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + s * ACH_MAX + cg, r);
+                    tmem_ld_wait();
+                    float v[32];
+                    float mn = INFINITY;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 cq = cnq[q];
+                        v[4 * q + 0] = fmaf(m2i, __uint_as_float(r[4 * q + 0]), cq.x);
+                        v[4 * q + 1] = fmaf(m2i, __uint_as_float(r[4 * q + 1]), cq.y);
+                        v[4 * q + 2] = fmaf(m2i, __uint_as_float(r[4 * q + 2]), cq.z);
+                        v[4 * q + 3] = fmaf(m2i, __uint_as_float(r[4 * q + 3]), cq.w);
+                        mn = fminf(mn, fminf(fminf(v[4 * q], v[4 * q + 1]), fminf(v[4 * q + 2], v[4 * q + 3])));
+                    }
+                    if (mn < d4) {
+                        const int c0 = ch * p.CH + cg;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) top4_insert(v[i], c0 + i, d1, d2, d3, d4, i1, i2, i3, i4);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(ABAR(B_AE + s));
+            }
+            if (!ok) break;
+            // hand the upper warpgroup's top-4 to the lower one
+            const uint32_t slot = tc & 1;
+            float *mrow = mg + ((int)slot * AM + rloc) * 8;
+            if (wg == 1) {
+                if (tc >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(ABAR(B_MR + slot), ((tc >> 1) - 1) & 1,
+                                                                           p.err))) {
+                    ok = false;
+                    break;
+                }
+                reinterpret_cast<float4 *>(mrow)[0] = make_float4(d1, d2, d3, d4);
+                reinterpret_cast<int4 *>(mrow)[1] = make_int4(i1, i2, i3, i4);
+                mbar_arrive(ABAR(B_MG + slot));
+            } else {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(ABAR(B_MG + slot), (tc >> 1) & 1, p.err))) {
+                    ok = false;
+                    break;
+                }
+                const float4 od = reinterpret_cast<const float4 *>(mrow)[0];
+                const int4 oi = reinterpret_cast<const int4 *>(mrow)[1];
+                mbar_arrive(ABAR(B_MR + slot));
+                top4_insert(od.x, oi.x, d1, d2, d3, d4, i1, i2, i3, i4);
+                top4_insert(od.y, oi.y, d1, d2, d3, d4, i1, i2, i3, i4);
+                top4_insert(od.z, oi.z, d1, d2, d3, d4, i1, i2, i3, i4);
+                top4_insert(od.w, oi.w, d1, d2, d3, d4, i1, i2, i3, i4);
+                if (valid) {
+                    const float sq = p.rowsq ? p.rowsq[f] : 1.f;
+                    const float delta = __uint_as_float(p.hstat[2 * h]);
+                    const float e = p.e_tc * (sq + __uint_as_float(p.hstat[2 * h + 1]));
+                    const float ub = d1 + assign_bound(d1, sq, delta, e);
+                    const bool a2 = i2 >= 0 && d2 - assign_bound(d2, sq, delta, e) <= ub;
+                    const bool a3 = i3 >= 0 && d3 - assign_bound(d3, sq, delta, e) <= ub;
+                    const bool a4 = i4 >= 0 && d4 - assign_bound(d4, sq, delta, e) <= ub;
+                    // A - E(A) grows with A once sqrt(dup) > delta, so the centres
+                    // beyond the kept four are settled when the fourth is.
+                    const bool beyond =
+                        m > 4 && (a4 || sqrtf(fmaxf(d4 + sq, 0.f) + 2.f * e) <= 2.f * delta);
+                    p.labels[f] = i1;
+                    if (a2 || a3 || a4 || beyond) {
+                        const int pos = atomicAdd(p.amb_count, 1);
+                        p.amb_list[pos] = (int)f;
+                        p.cand[pos] = beyond ? make_int4(-2, 0, 0, 0)
+                                             : make_int4(i1, a2 ? i2 : -1, a3 ? i3 : -1, a4 ? i4 : -1);
+                        if (beyond) atomicAdd(p.stats + 1, 1ull);
+                    }
+                }
+            }
+            ++tc;
+        }
+        if (!ok) set_err(p.err, DEV_ERR_TIMEOUT);
+    }
+#undef ABAR
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// Exact fp32 squared distance, dimensions in order (the definition's arithmetic).
+template <bool NORM>
+__device__ __forceinline__ float exact_sqdist(const bf16 *__restrict__ xr, float s, const float *__restrict__ c,
+                                              int d) {
+    float acc = 0.f;
+    const uint4 *x8 = reinterpret_cast<const uint4 *>(xr);
+    const float4 *c4 = reinterpret_cast<const float4 *>(c);
+    for (int k8 = 0; k8 < d / 8; ++k8) {
+        const uint4 xv = x8[k8];
+        const float4 ca = c4[2 * k8], cb = c4[2 * k8 + 1];
+        const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+        const float cc[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float x = __uint_as_float((j & 1) ? (w[j >> 1] & 0xFFFF0000u) : (w[j >> 1] << 16));
+            if (NORM) x = __fmul_rn(x, s);
+            const float t = __fsub_rn(x, cc[j]);
+            acc = __fadd_rn(acc, __fmul_rn(t, t));
+        }
+    }
+    return acc;
+}
+
+// One warp per uncertain row: exact distances of the candidates (lanes 0-3) or
+// of every centre (lane-strided, ascending per lane), argmin with the lowest
+// index among equal distances.
+template <bool NORM>
+__global__ void k_assign_resolve(const bf16 *__restrict__ X, const float *__restrict__ inv, int64_t L, int d,
+                                 const float *__restrict__ C, int64_t cstride, const int *__restrict__ ncent,
+                                 int ncent_const, const int4 *__restrict__ cand, const int *__restrict__ amb_list,
+                                 const int *__restrict__ amb_count, int *__restrict__ labels,
+                                 unsigned long long *__restrict__ stats) {
+    const int n = *amb_count;
+    const int lane = threadIdx.x & 31;
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, nw = (gridDim.x * blockDim.x) >> 5;
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(stats, (unsigned long long)n);
+    for (int i = gw; i < n; i += nw) {
+        const int64_t f = amb_list[i];
+        const int h = (int)(f / L);
+        const int m = ncent ? ncent[h] : ncent_const;
+        const bf16 *xr = X + f * d;
+        const float s = NORM ? inv[f] : 1.f;
+        const float *Ch = C + (int64_t)h * cstride;
+        const int4 cd = cand[i];
+        float best = INFINITY;
+        int arg = 0x7FFFFFFF;
+        if (cd.x == -2) {
+            for (int c = lane; c < m; c += 32) {
+                const float v = exact_sqdist<NORM>(xr, s, Ch + (int64_t)c * d, d);
+                if (v < best) {
+                    best = v;
+                    arg = c;
+                }
+            }
+        } else if (lane < 4) {
+            const int c = lane == 0 ? cd.x : lane == 1 ? cd.y : lane == 2 ? cd.z : cd.w;
+            if (c >= 0) {
+                best = exact_sqdist<NORM>(xr, s, Ch + (int64_t)c * d, d);
+                arg = c;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+            const int oa = __shfl_xor_sync(0xFFFFFFFFu, arg, o);
+            if (ob < best || (ob == best && oa < arg)) {
+                best = ob;
+                arg = oa;
+            }
+        }
+        if (lane == 0) labels[f] = arg == 0x7FFFFFFF ? 0 : arg;
+    }
+}
+
+// dmin[f] = exact distance of row f to its labelled centre.
+template <bool NORM>
+__global__ void k_exact_dmin(const bf16 *__restrict__ X, const float *__restrict__ inv, int64_t L, int d,
+                             const float *__restrict__ C, int64_t cstride, const int *__restrict__ nrows,
+                             int nrows_const, const int *__restrict__ ncent, int ncent_const,
+                             const int *__restrict__ labels, float *__restrict__ dmin) {
+    const int h = blockIdx.y;
+    const int row = blockIdx.x * blockDim.x + threadIdx.x;
+    const int n = nrows ? nrows[h] : nrows_const;
+    const int m = ncent ? ncent[h] : ncent_const;
+    if (row >= n || m <= 0) return;
+    const int64_t f = (int64_t)h * L + row;
+    dmin[f] = exact_sqdist<NORM>(X + f * d, NORM ? inv[f] : 1.f, C + (int64_t)h * cstride + (int64_t)labels[f] * d,
+                                 d);
+}
+
+// |x|^2 of every row (it only enters the error bound; fp32 is enough).
+__global__ void k_row_sqnorm(const bf16 *__restrict__ X, int64_t rows, int d, float *__restrict__ out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= rows) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(X + i * d);
+    float ss = 0.f;
+    for (int k8 = 0; k8 < d / 8; ++k8) {
+        const uint4 v = src[k8];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const float a = __uint_as_float(w[t] << 16), b = __uint_as_float(w[t] & 0xFFFF0000u);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+        }
+    }
+    out[i] = ss;
+}
+
+// c_hi = bf16(c) (nearest), c_lo = bf16(c - c_hi) with two terms, c' their
+// sum; cn = fp32(|c'|^2); per unit the largest delta = |c - c'| and the
+// largest |c'|^2, both in fp64 rounded up.  Chi holds [BH, Cpad, d] c_hi rows
+// then (two terms) [BH, Cpad, d] c_lo rows.  Rows c >= m up to Cpad are zero
+// with cn = +inf.
+__global__ void k_centre_prep(const float *__restrict__ C, int64_t cstride, const int *__restrict__ ncent,
+                              int ncent_const, int d, int Cpad, int two_term, bf16 *__restrict__ Chi,
+                              float *__restrict__ cn, unsigned int *__restrict__ hstat) {
+    const int c = blockIdx.x, h = blockIdx.y;
+    const int m = ncent ? ncent[h] : ncent_const;
+    const int64_t lo_off = (int64_t)gridDim.y * Cpad * d;
+    bf16 *dst = Chi + ((int64_t)h * Cpad + c) * d;
+    if (c >= m) {
+        for (int k = threadIdx.x; k < d; k += blockDim.x) {
+            dst[k] = __float2bfloat16_rn(0.f);
+            if (two_term) dst[lo_off + k] = __float2bfloat16_rn(0.f);
+        }
+        if (threadIdx.x == 0) cn[(int64_t)h * Cpad + c] = INFINITY;
+        return;
+    }
+    const float *src = C + (int64_t)h * cstride + (int64_t)c * d;
+    double e2 = 0.0, n2 = 0.0;
+    for (int k = threadIdx.x; k < d; k += blockDim.x) {
+        const float v = src[k];
+        const bf16 hi = __float2bfloat16_rn(v);
+        dst[k] = hi;
+        double rep = (double)__bfloat162float(hi);
+        if (two_term) {
+            const bf16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));  // v - hi is exact in fp32
+            dst[lo_off + k] = lo;
+            rep += (double)__bfloat162float(lo);
+        }
+        const double r = (double)v - rep;
+        e2 += r * r;
+        n2 += rep * rep;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        e2 += __shfl_down_sync(0xFFFFFFFFu, e2, o);
+        n2 += __shfl_down_sync(0xFFFFFFFFu, n2, o);
+    }
+    __shared__ double se[4], sn[4];
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+        se[w] = e2;
+        sn[w] = n2;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double te = 0.0, tn = 0.0;
+        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+            te += se[i];
+            tn += sn[i];
+        }
+        cn[(int64_t)h * Cpad + c] = (float)tn;
+        const float delta = __double2float_ru(sqrt(te) * (1.0 + 1e-12));
+        atomicMax(&hstat[2 * h], __float_as_uint(delta));
+        atomicMax(&hstat[2 * h + 1], __float_as_uint(__double2float_ru(tn)));
+    }
+}
+
+template <int D>
+cudaError_t launch_mma(const FastAssignArgs &a, const AsgParams &p, int grid, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(k_assign_mma<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)ALayout<D>::SMEM);
+    if (e != cudaSuccess) return e;
+    k_assign_mma<D><<<grid, A_THREADS, ALayout<D>::SMEM, s>>>(*a.tm_x, *a.tm_c, p);
+    AC_NOTE_LAUNCH();
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_row_sqnorm(const bf16 *X, int64_t rows, int d, float *out, cudaStream_t s) {
+    if (rows <= 0) return cudaSuccess;
+    k_row_sqnorm<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(X, rows, d, out);
+    AC_NOTE_LAUNCH();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_assign_fast(const FastAssignArgs &a, cudaStream_t s) {
+    cudaError_t e;
+    const int BH = a.BH;
+    if (BH <= 0 || a.L <= 0) return cudaSuccess;
+    // 1. split the centres
+    if ((e = cudaMemsetAsync(a.hstat, 0, sizeof(unsigned int) * 2 * BH, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.amb_count, 0, sizeof(int), s)) != cudaSuccess) return e;
+    k_centre_prep<<<dim3(a.Cpad, BH), 64, 0, s>>>(a.C, a.cstride, a.ncent, a.ncent_const, a.d, a.Cpad,
+                                                  a.two_term ? 1 : 0, a.Chi, a.cn, a.hstat);
+    AC_NOTE_LAUNCH();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 2. tensor-core pass with the top-4 epilogue
+    AsgParams p;
+    p.inv = a.inv;
+    p.rowsq = a.rowsq;
+    p.cn = a.cn;
+    p.hstat = a.hstat;
+    p.nrows = a.nrows;
+    p.nrows_const = a.nrows_const;
+    p.ncent = a.ncent;
+    p.ncent_const = a.ncent_const;
+    p.L = a.L;
+    p.BH = BH;
+    p.Cpad = a.Cpad;
+    p.CH = a.CH;
+    p.tiles_per_unit = (int)((a.L + AM - 1) / AM);
+    p.two_term = a.two_term ? 1 : 0;
+    p.e_tc = (float)(a.two_term ? 2 * a.d : a.d) * 1.1920928955078125e-07f;  // products * 2^-23
+    p.labels = a.labels;
+    p.cand = a.cand;
+    p.amb_list = a.amb_list;
+    p.amb_count = a.amb_count;
+    p.stats = a.stats;
+    p.err = a.err;
+    const int ntiles = BH * p.tiles_per_unit;
+    const int grid = ntiles < a.num_sms ? ntiles : a.num_sms;
+    e = a.d == 128 ? launch_mma<128>(a, p, grid, s) : launch_mma<64>(a, p, grid, s);
+    if (e != cudaSuccess) return e;
+    // 3. exact rescoring of the uncertain rows
+    if (a.inv)
+        k_assign_resolve<true><<<4 * a.num_sms, 256, 0, s>>>(a.X, a.inv, a.L, a.d, a.C, a.cstride, a.ncent,
+                                                             a.ncent_const, a.cand, a.amb_list, a.amb_count,
+                                                             a.labels, a.stats);
+    else
+        k_assign_resolve<false><<<4 * a.num_sms, 256, 0, s>>>(a.X, a.inv, a.L, a.d, a.C, a.cstride, a.ncent,
+                                                              a.ncent_const, a.cand, a.amb_list, a.amb_count,
+                                                              a.labels, a.stats);
+    AC_NOTE_LAUNCH();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 4. exact distance to the chosen centre
+    if (a.dmin) {
+        const int maxn = a.nrows ? (int)a.L : a.nrows_const;
+        const dim3 grid2((maxn + 127) / 128, BH);
+        if (a.inv)
+            k_exact_dmin<true><<<grid2, 128, 0, s>>>(a.X, a.inv, a.L, a.d, a.C, a.cstride, a.nrows, a.nrows_const,
+                                                     a.ncent, a.ncent_const, a.labels, a.dmin);
+        else
+            k_exact_dmin<false><<<grid2, 128, 0, s>>>(a.X, a.inv, a.L, a.d, a.C, a.cstride, a.nrows,
+                                                      a.nrows_const, a.ncent, a.ncent_const, a.labels, a.dmin);
+        AC_NOTE_LAUNCH();
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace ac

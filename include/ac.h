@@ -239,6 +239,26 @@ typedef struct ac_attn_counters {
 
 AC_API ac_status ac_get_attn_counters(ac_ctx *ctx, ac_attn_counters *out);
 
+/* Diagnostics of the k-means assignments since the context was created (or
+ * last reset).  The assignments of Sec. 3.1 and of Algorithm 1 (stage 0, the
+ * final pass over all of C) and of the warm-started Lloyd passes run on the
+ * tensor cores: centres split into bf16 + remainder, x . c_hi per pair, then
+ * a rigorous error bound decides each row; rows the bound cannot settle are
+ * rescored with the exact fp32 arithmetic, so labels equal the exact
+ * definition's.  Stages t >= 1 of Algorithm 1 (gathered rows) and inputs not
+ * 16-byte aligned take the exact CUDA-core kernel.  The environment variable
+ * AC_EXACT_ASSIGN=1 at ac_create forces the exact kernel everywhere.
+ * Synchronises `ctx`'s device; reset != 0 zeroes the counters afterwards. */
+typedef struct ac_assign_counters {
+    int64_t tensor_passes;      /* assignment passes run on the tensor cores   */
+    int64_t exact_passes;       /* assignment passes run by the exact kernel   */
+    int64_t rows;               /* rows assigned by the tensor-core passes     */
+    int64_t uncertain_rows;     /* of those, rescored exactly (candidates)     */
+    int64_t full_rescore_rows;  /* of those, rescored against every centre     */
+} ac_assign_counters;
+
+AC_API ac_status ac_get_assign_counters(ac_ctx *ctx, ac_assign_counters *out, int32_t reset);
+
 /* The query clustering of ac_cluster_q (normalise, then Lloyd k-means with
  * Cq centres) without a context and without allocating device memory.  The
  * paper has no counterpart of this entry point; it exists for callers that
