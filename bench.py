@@ -309,6 +309,7 @@ def main():
                 "computed_tile_flops_per_launch": 4.0 * cfg.d * cnt["computed_pairs"]}
 
     extra = {"step0": split0, "warm": splitw, "counters_last_call": cnt,
+             "assign_counters_since_create": lay.assign_counters(),
              "kept_pair_frac": cnt["kept_pairs"] / float(cfg.H * cfg.L * cfg.L),
              "tile_efficiency": cnt["kept_pairs"] / max(1, cnt["computed_pairs"])}
     # dense SDPA on the same tensors (one warm step's inputs)

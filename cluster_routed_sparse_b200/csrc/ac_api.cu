@@ -367,7 +367,7 @@ ac_status key_stats_impl(ac_ctx *c, const bf16 *K, cudaStream_t s) {
 ac_status score_select_impl(ac_ctx *c, int topk, cudaStream_t s) {
     SelectArgs a{c->cent_q, c->kmax, c->kmin, c->counts_k, c->n_k, c->dense, c->offs_k, c->counts_q,
                  c->Cq, c->Ccap, c->d, c->BH, c->L, topk != 0 ? topk : c->cfg.topk,
-                 c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix};
+                 c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->rbox};
     CK(launch_score_select(a, s), "score select");
     return AC_OK;
 }
@@ -378,7 +378,7 @@ ac_status sparse_attn_impl(ac_ctx *c, const bf16 *Q, const bf16 *K, const bf16 *
     CK(launch_permute_rows(V, c->perm_k, c->Vp, c->L, c->d, c->BH, s), "permute v");
     CK(cudaMemsetAsync(c->counters, 0, 8 * sizeof(unsigned long long), s), "counters");
     AttnArgs a{&c->tm_q, &c->tm_k, &c->tm_v, O, c->perm_q, c->offs_q, c->counts_q, c->tile_prefix, c->ranges,
-               c->nboxes, c->ksel, c->dense, c->L, c->Cq, c->Ccap, c->BH, c->d,
+               c->nboxes, c->ksel, c->rbox, c->dense, c->L, c->Cq, c->Ccap, c->BH, c->d,
                (float)(c->scale * 1.4426950408889634), c->err, c->counters};
     if (c->timing) CK(cudaEventRecord(c->ev[6], s), "event");
     CK(launch_sparse_attn(a, s), "sparse attention");
@@ -393,7 +393,7 @@ void free_all(ac_ctx *c) {
                    c->u_cnt, c->st_m, c->st_labels, c->st_dist, c->st_perm, c->st_offs, c->st_counts, c->radix,
                    c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->Qp, c->Kp, c->Vp,
                    c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err, c->chi_q, c->chi_k, c->cn,
-                   c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats};
+                   c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats, c->rbox};
     for (void *p : dev)
         if (p) cudaFree(p);
     void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err};
@@ -496,6 +496,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->ksel, BH));
     A(dalloc(&c->ranges, BH * Cq * Cc));
     A(dalloc(&c->nboxes, BH * Cq));
+    A(dalloc(&c->rbox, BH * Cq * (Cc + 1)));
     A(dalloc(&c->tile_prefix, BH * Cq + 1));
     A(dalloc(&c->chi_q, 2 * BH * c->Cpad_q * dz));
     A(dalloc(&c->chi_k, BH * c->Cpad_k * dz));

@@ -62,6 +62,7 @@ struct ac_ctx {
     int *ksel;         // [BH]
     int2 *ranges;      // [BH, Cq, Ccap]  (start row in cluster order, count)
     int *nboxes;       // [BH*Cq]         8-row key boxes per query cluster
+    int *rbox;         // [BH*Cq, Ccap+1] first box of each selected range (exclusive prefix)
     int *tile_prefix;  // [BH*Cq+1]       attention items (pairs of 128-query tiles), exclusive prefix
 
     // ---- tensor-core assignment (centres split into bf16 + remainder)
@@ -230,13 +231,14 @@ struct SelectArgs {
     const int *n_k; const uint8_t *dense; const int *offs_k; const int *counts_q;
     int Cq, Ccap, d, BH, L, topk;
     float *score; int *sel; int *ksel; int2 *ranges; int *nboxes; int *tile_prefix;
+    int *rbox;
 };
 cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s);
 
 struct AttnArgs {
     const CUtensorMap *tm_q, *tm_k, *tm_v;
     bf16 *O; const int *perm_q; const int *offs_q; const int *counts_q;
-    const int *tile_prefix; const int2 *ranges; const int *nboxes; const int *ksel;
+    const int *tile_prefix; const int2 *ranges; const int *nboxes; const int *ksel; const int *rbox;
     const uint8_t *dense; int L, Cq, Ccap, BH, d;
     float scale_log2;
     uint32_t *err; unsigned long long *counters;

@@ -44,6 +44,7 @@ constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= NTHREADS * 168, "register split exceeds the launch");
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int RG_CACHE = 2048;  // key ranges kept in shared memory (more: read from global)
+constexpr int kPolyChunk = 3;   // of the 4 32-column chunks of a key tile, this one takes exp2_poly
 // K/V tile layout in shared memory: 16 boxes, each [column half][8 rows][128 B]
 // (one 3-D TMA copy per box); an 8-row group is BOX_BYTES after the previous.
 
@@ -58,7 +59,8 @@ struct Layout {
     static constexpr uint32_t OFF_V = OFF_K + NS * KV_BYTES;
     static constexpr uint32_t OFF_MASK = OFF_V + NS * KV_BYTES;  // [NS][4] uint32
     static constexpr uint32_t OFF_RG = OFF_MASK + 64;            // [RG_CACHE] int2 key ranges
-    static constexpr uint32_t OFF_BAR = OFF_RG + RG_CACHE * 8;
+    static constexpr uint32_t OFF_RB = OFF_RG + RG_CACHE * 8;    // [RG_CACHE + 1] first box of each range
+    static constexpr uint32_t OFF_BAR = OFF_RB + (RG_CACHE + 1) * 4 + 12;
     static constexpr uint32_t BYTES = OFF_BAR + 256;
     static constexpr uint32_t SMEM = BYTES + 1024;  // 1024-byte alignment slack
 };
@@ -74,37 +76,25 @@ enum {
     NBAR = 12
 };
 
-struct KeyWalker {
-    const int2 *rg;
-    int nr, r, o;
-    __device__ __forceinline__ void init(const int2 *g, int n) {
-        rg = g;
-        nr = n;
-        r = 0;
-        o = 0;
-    }
-    // Next 8-row box: first row (within the unit) and number of valid rows.
-    __device__ __forceinline__ void next(int &start, int &cnt) {
-        if (r < nr) {
-            const int2 g = rg[r];
-            start = g.x + o;
-            const int rem = g.y - o;
-            cnt = rem < 8 ? rem : 8;
-            o += cnt;
-            if (o >= g.y) {
-                ++r;
-                o = 0;
-            }
-        } else {
-            start = 0;
-            cnt = 0;
-        }
-    }
-};
+// 2^x on the FMA pipe, so that part of the exponentials bypass the
+// special-function unit (one ex2 per element would take as long as the two
+// matrix products of a tile).  Range reduction x = n + f with n = round(x),
+// |f| <= 1/2 (Cody and Waite), n read from the low mantissa bits of
+// x + 1.5 * 2^23; 2^f by a cubic fitted here for least maximum relative error
+// on [-1/2, 1/2] (1.02e-4, below the 2^-9 rounding of the bf16 P it feeds);
+// 2^n added to the exponent field.  x is clamped at -126, so -inf (a masked
+// column) gives at most 2^-126 instead of 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -126.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    const float q = fmaf(fmaf(fmaf(0.05500858277f, f, 0.24221037328f), f, 0.69328290224f), f, 1.0f);
+    return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
 
 struct AttnParams {
     bf16 *O;
-    const int *perm_q, *offs_q, *counts_q, *tile_prefix, *nboxes, *ksel;
+    const int *perm_q, *offs_q, *counts_q, *tile_prefix, *nboxes, *ksel, *rbox;
     const int2 *ranges;
     const uint8_t *dense;
     int L, Cq, Ccap, BH;
@@ -153,7 +143,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int64_t unit_row = (int64_t)h * p.L;
     const int n_tiles = (p.nboxes[hq] + BOXES - 1) / BOXES;
     const int2 *rg = p.ranges + (int64_t)hq * p.Ccap;
+    const int *rb = p.rbox + (int64_t)hq * (p.Ccap + 1);
     const int nr = p.dense[h] ? 1 : p.ksel[h];
+    const int nbox = p.nboxes[hq];
 
     const uint32_t bar0 = sbase + LY::OFF_BAR;
 #define BAR(i) (bar0 + 8u * (uint32_t)(i))
@@ -192,50 +184,72 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp >= 8) {
       reg_dealloc<kRegsOther>();
       if (warp == 8) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (whole warp)
+        // Key tile j is boxes 16j .. 16j+15 of the concatenated selected ranges.
+        // Lane l < 16 finds the range of box 16j + l by a binary search over
+        // the first boxes of 32 ranges from r0 (one tile spans at most 16
+        // ranges), then issues that box's K and V copies; lane 16 finds the
+        // range that starts the next tile.
         int2 *rg_s = reinterpret_cast<int2 *>(sm + LY::OFF_RG);
-        const bool rg_cached = nr <= RG_CACHE;
-        if (rg_cached)
+        int *rb_s = reinterpret_cast<int *>(sm + LY::OFF_RB);
+        const bool cached = nr <= RG_CACHE;
+        if (cached) {
             for (int i = lane; i < nr; i += 32) rg_s[i] = rg[i];
+            for (int i = lane; i <= nr; i += 32) rb_s[i] = rb[i];
+        }
         __syncwarp();
+        const int2 *rgp = cached ? rg_s : rg;
+        const int *rbp = cached ? rb_s : rb;
         if (lane == 0) {
             mbar_arrive_expect_tx(BAR(B_QF), 2 * LY::Q_TILE);
             for (int t = 0; t < 2; ++t)
                 for (int hf = 0; hf < LY::HALVES; ++hf)
                     tma_load_2d(sbase + LY::OFF_Q + t * LY::Q_TILE + hf * BM * 128, &tm_q, hf * 64,
                                 (int)(unit_row + row0 + t * BM), BAR(B_QF));
-            KeyWalker w;
-            w.init(rg_cached ? rg_s : rg, nr);
-            int issued = 0;
-            for (int j = 0; j < n_tiles; ++j) {
-                const int s = j % NS;
-                if (j >= NS && !WAIT(1, B_KVE + s, j, ((j / NS) - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                // pass 1: validity masks of the 16 boxes; pass 2: their loads
-                KeyWalker w2 = w;
-                uint32_t vm[4] = {0u, 0u, 0u, 0u};
+        }
+        int r0 = 0, issued = 0;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int s = j % NS;
+            const int b = j * BOXES + lane;
+            const int pv = r0 + lane <= nr ? rbp[r0 + lane] : 0x7FFFFFFF;
+            int k = 0;
 #pragma unroll
-                for (int b = 0; b < BOXES; ++b) {
-                    int st, c;
-                    w.next(st, c);
-                    vm[b >> 2] |= (c >= 8 ? 0xFFu : ((1u << c) - 1u)) << ((b & 3) * 8);
-                }
-                *reinterpret_cast<uint4 *>(masks + 4 * s) = make_uint4(vm[0], vm[1], vm[2], vm[3]);
-                mbar_arrive_expect_tx(BAR(B_KVF + s), 2 * LY::KV_BYTES);  // releases the masks
-                const uint32_t kd = sbase + LY::OFF_K + s * LY::KV_BYTES;
-                const uint32_t vd = sbase + LY::OFF_V + s * LY::KV_BYTES;
-#pragma unroll 1
-                for (int b = 0; b < BOXES; ++b) {
-                    int st, c;
-                    w2.next(st, c);
-                    const int row = (int)(unit_row + st);
-                    tma_load_3d(kd + b * LY::BOX_BYTES, &tm_k, 0, row, 0, BAR(B_KVF + s));
-                    tma_load_3d(vd + b * LY::BOX_BYTES, &tm_v, 0, row, 0, BAR(B_KVF + s));
-                }
-                ++issued;
+            for (int st = 16; st >= 1; st >>= 1) {
+                const int v = __shfl_sync(0xFFFFFFFFu, pv, min(k + st, 31));
+                if (k + st <= 31 && v <= b) k += st;
             }
+            const int r = r0 + k;
+            const int first = __shfl_sync(0xFFFFFFFFu, pv, k);
+            int start = 0, cnt = 0;
+            if (lane < BOXES && b < nbox) {
+                const int2 g = rgp[r];
+                const int o = (b - first) * 8;
+                start = g.x + o;
+                cnt = min(8, g.y - o);
+            }
+            const int rnext = __shfl_sync(0xFFFFFFFFu, r, BOXES);
+            uint32_t bits = lane < BOXES ? (cnt >= 8 ? 0xFFu : ((1u << cnt) - 1u)) << ((lane & 3) * 8) : 0u;
+            bits |= __shfl_xor_sync(0xFFFFFFFFu, bits, 1);
+            bits |= __shfl_xor_sync(0xFFFFFFFFu, bits, 2);
+            if (j >= NS && !__all_sync(0xFFFFFFFFu, WAIT(1, B_KVE + s, j, ((j / NS) - 1) & 1))) {
+                ok = false;
+                break;
+            }
+            if (lane < BOXES && (lane & 3) == 0) masks[4 * s + (lane >> 2)] = bits;
+            __syncwarp();
+            if (lane == 0) mbar_arrive_expect_tx(BAR(B_KVF + s), 2 * LY::KV_BYTES);  // releases the masks
+            __syncwarp();
+            if (lane < BOXES) {
+                const int row = (int)(unit_row + start);
+                tma_load_3d(sbase + LY::OFF_K + s * LY::KV_BYTES + lane * LY::BOX_BYTES, &tm_k, 0, row, 0,
+                            BAR(B_KVF + s));
+                tma_load_3d(sbase + LY::OFF_V + s * LY::KV_BYTES + lane * LY::BOX_BYTES, &tm_v, 0, row, 0,
+                            BAR(B_KVF + s));
+            }
+            r0 = rnext;
+            ++issued;
+        }
+        if (lane == 0) {
             // Loads still in flight must land before the CTA exits.
             for (int j = issued - NS < 0 ? 0 : issued - NS; j < issued; ++j)
                 if (!WAIT(2, B_KVF + (j % NS), j, (j / NS) & 1)) ok = false;
@@ -402,8 +416,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const int c = half * 2 + cc;
 #pragma unroll
                         for (int i = 0; i < 32; i += 2) {
-                            const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), sl2, neg_m));
-                            const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), sl2, neg_m));
+                            const float x0 = fmaf(__uint_as_float(r[c][i]), sl2, neg_m);
+                            const float x1 = fmaf(__uint_as_float(r[c][i + 1]), sl2, neg_m);
+                            const float p0 = c == kPolyChunk ? exp2_poly(x0) : ex2_approx(x0);
+                            const float p1 = c == kPolyChunk ? exp2_poly(x1) : ex2_approx(x1);
                             ps[i & 7] += p0;
                             ps[(i + 1) & 7] += p1;
                             pk[cc * 16 + (i >> 1)] = pack_bf16x2(p0, p1);
@@ -477,6 +493,7 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s) {
     p.nboxes = a.nboxes;
     p.ksel = a.ksel;
     p.ranges = a.ranges;
+    p.rbox = a.rbox;
     p.dense = a.dense;
     p.L = a.L;
     p.Cq = a.Cq;

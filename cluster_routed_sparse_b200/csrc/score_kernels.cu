@@ -88,23 +88,33 @@ __global__ void __launch_bounds__(SEL_THREADS) k_score_select(SelectArgs a) {
     int pos;
     Scan(tmp.scan).ExclusiveSum(mine, pos);
     __syncthreads();
+    // 8-row boxes of the kept clusters: exclusive prefix in selection order
     int boxes = 0;
+    for (int c = c0; c < c1; ++c)
+        if (flag[c]) boxes += (cnt[c] + 7) / 8;
+    int bpos, nb;
+    Scan(tmp.scan).ExclusiveSum(boxes, bpos, nb);
+    __syncthreads();
     const int *offs = a.offs_k + (int64_t)h * (a.Ccap + 1);
+    int *rbox = a.rbox + (int64_t)hq * (a.Ccap + 1);
     for (int c = c0; c < c1; ++c) {
         if (!flag[c]) continue;
         a.sel[(int64_t)hq * a.Ccap + pos] = c;
         a.ranges[(int64_t)hq * a.Ccap + pos] = make_int2(offs[c], cnt[c]);
-        boxes += (cnt[c] + 7) / 8;
+        rbox[pos] = bpos;
+        bpos += (cnt[c] + 7) / 8;
         ++pos;
     }
-    const int nb = Red(tmp.red).Sum(boxes);
     __syncthreads();
     if (tid == 0) {
         if (a.dense[h]) {  // Algorithm 3 line 6: every key of the unit
             a.ranges[(int64_t)hq * a.Ccap] = make_int2(0, a.L);
             a.nboxes[hq] = (a.L + 7) / 8;
+            rbox[0] = 0;
+            rbox[1] = (a.L + 7) / 8;
         } else {
             a.nboxes[hq] = nb;
+            rbox[k] = nb;
         }
     }
 }
