@@ -125,6 +125,30 @@ __device__ __forceinline__ void top4_insert(float v, int c, float &d1, float &d2
     }
 }
 
+// r[i] for a run-time i without local memory: a 5-level select tree.
+__device__ __forceinline__ float pick32(const uint32_t (&r)[32], int i) {
+    uint32_t a[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) a[k] = (i & 1) ? r[2 * k + 1] : r[2 * k];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = (i & 2) ? a[2 * k + 1] : a[2 * k];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) a[k] = (i & 4) ? a[2 * k + 1] : a[2 * k];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) a[k] = (i & 8) ? a[2 * k + 1] : a[2 * k];
+    return __uint_as_float((i & 16) ? a[1] : a[0]);
+}
+
+// Largest A that can still matter once the best so far is d1: every centre
+// with A > T has A - E(A) > d1 + E(d1) >= the final best's upper bound.  With
+// sqrt(dup) > 2 delta the slope of E is below 0.51, so T = d1 + 4.5 E(d1)
+// suffices; otherwise A - E(A) need not grow with A and nothing is skipped.
+__device__ __forceinline__ float assign_threshold(float d1, float sq, float delta, float e) {
+    if (!(d1 < INFINITY)) return INFINITY;
+    if (sqrtf(fmaxf(d1 + sq, 0.f) + 2.f * e) <= 2.f * delta) return INFINITY;
+    return d1 + 4.5f * assign_bound(d1, sq, delta, e);
+}
+
 template <int D>
 __global__ void __launch_bounds__(A_THREADS, 1)
     k_assign_mma(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_c,
@@ -259,60 +283,116 @@ __global__ void __launch_bounds__(A_THREADS, 1)
         // ------------------------------------------------ epilogue
         // Warpgroup wg takes the 32-column groups wg, wg + 2, ... of every
         // chunk; warp w reads tensor-memory lanes 32 (w % 4) .. + 31, i.e. rows.
+        // A group costs one FMA and one min per centre: only groups whose
+        // minimum reaches the threshold T of assign_threshold (rare after the
+        // first) insert into the row's top-4 list.  The per-row and per-unit
+        // scalars of the next tile and the centre norms of the next group are
+        // loaded ahead, so no global load latency sits on the chunk path.
         const int wg = warp >> 2;
         const int rloc = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         float *mg = reinterpret_cast<float *>(sm + LY::OFF_MG);
+        struct TileScalars {
+            float inv, sq;
+            uint32_t delta, cmax;
+            int m;
+        };
+        auto fetch = [&](int tt, TileScalars &v) {
+            if (tt >= ntiles) return;
+            const int hh = tt / p.tiles_per_unit;
+            const int row = (tt % p.tiles_per_unit) * AM + rloc;
+            const int nn = p.nrows ? p.nrows[hh] : p.nrows_const;
+            const int64_t ff = (int64_t)hh * p.L + row;
+            v.m = p.ncent ? p.ncent[hh] : p.ncent_const;
+            v.inv = p.inv && row < nn ? p.inv[ff] : 1.f;
+            v.sq = p.rowsq && row < nn ? p.rowsq[ff] : 1.f;
+            v.delta = p.hstat[2 * hh];
+            v.cmax = p.hstat[2 * hh + 1];
+        };
+        TileScalars cur{1.f, 1.f, 0u, 0u, 0}, nxt{1.f, 1.f, 0u, 0u, 0};
+        fetch(blockIdx.x, cur);
         uint32_t g = 0, tc = 0;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, cur = nxt) {
+            fetch(t + gridDim.x, nxt);
             const int h = t / p.tiles_per_unit, rt = t % p.tiles_per_unit;
             const int n = p.nrows ? p.nrows[h] : p.nrows_const;
-            const int m = p.ncent ? p.ncent[h] : p.ncent_const;
+            const int m = cur.m;
             if (rt * AM >= n || m <= 0) continue;
             const int row = rt * AM + rloc;
             const bool valid = row < n;
             const int64_t f = (int64_t)h * p.L + row;
-            const float inv = p.inv ? (valid ? p.inv[f] : 0.f) : 1.f;
-            const float m2i = -2.f * inv;
+            const float m2i = -2.f * cur.inv;
+            const float sq = cur.sq;
+            const float delta = __uint_as_float(cur.delta);
+            const float e = p.e_tc * (sq + __uint_as_float(cur.cmax));
             const float *cnh = p.cn + (int64_t)h * p.Cpad;
             float d1 = INFINITY, d2 = INFINITY, d3 = INFINITY, d4 = INFINITY;
             int i1 = 0, i2 = -1, i3 = -1, i4 = -1;
+            float T = INFINITY;
             const int nch = (m + p.CH - 1) / p.CH;
+            // the column groups of this warpgroup, over all chunks of the tile
+            float4 cq[8];
+            auto load_cn = [&](int c0, float4 (&dst)[8]) {
+                const float4 *cn4 = reinterpret_cast<const float4 *>(cnh + c0);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) dst[q] = __ldg(cn4 + q);
+            };
+            if (wg * 32 < m) load_cn(wg * 32, cq);
             for (int ch = 0; ch < nch; ++ch, ++g) {
                 const uint32_t s = g & 1;
+                const int rem = m - ch * p.CH;
+                const int N = rem >= p.CH ? p.CH : ((rem + 31) & ~31);
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(ABAR(B_AF + s), (g >> 1) & 1, p.err))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const int rem = m - ch * p.CH;
-                const int N = rem >= p.CH ? p.CH : ((rem + 31) & ~31);
                 for (int cg = wg * 32; cg < N; cg += 64) {
-                    // |c'|^2 of these 32 centres (same address in every lane: one
-                    // broadcast load each; +inf past the last centre)
-                    float4 cnq[8];
-                    const float4 *cn4 = reinterpret_cast<const float4 *>(cnh + ch * p.CH + cg);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) cnq[q] = __ldg(cn4 + q);
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_off + s * ACH_MAX + cg, r);
+                    // next group of this warpgroup: same chunk, else the next chunk
+                    float4 cqn[8];
+                    const int ncg = cg + 64 < N ? ch * p.CH + cg + 64 : (ch + 1) * p.CH + wg * 32;
+                    if (ncg < m) load_cn(ncg, cqn);
                     tmem_ld_wait();
-                    float v[32];
                     float mn = INFINITY;
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 cq = cnq[q];
-                        v[4 * q + 0] = fmaf(m2i, __uint_as_float(r[4 * q + 0]), cq.x);
-                        v[4 * q + 1] = fmaf(m2i, __uint_as_float(r[4 * q + 1]), cq.y);
-                        v[4 * q + 2] = fmaf(m2i, __uint_as_float(r[4 * q + 2]), cq.z);
-                        v[4 * q + 3] = fmaf(m2i, __uint_as_float(r[4 * q + 3]), cq.w);
-                        mn = fminf(mn, fminf(fminf(v[4 * q], v[4 * q + 1]), fminf(v[4 * q + 2], v[4 * q + 3])));
+                        const float v0 = fmaf(m2i, __uint_as_float(r[4 * q + 0]), cq[q].x);
+                        const float v1 = fmaf(m2i, __uint_as_float(r[4 * q + 1]), cq[q].y);
+                        const float v2 = fmaf(m2i, __uint_as_float(r[4 * q + 2]), cq[q].z);
+                        const float v3 = fmaf(m2i, __uint_as_float(r[4 * q + 3]), cq[q].w);
+                        r[4 * q + 0] = __float_as_uint(v0);
+                        r[4 * q + 1] = __float_as_uint(v1);
+                        r[4 * q + 2] = __float_as_uint(v2);
+                        r[4 * q + 3] = __float_as_uint(v3);
+                        mn = fminf(mn, fminf(fminf(v0, v1), fminf(v2, v3)));
                     }
-                    if (mn < d4) {
-                        const int c0 = ch * p.CH + cg;
+                    // This group holds the best so far or a near tie for some
+                    // row of the warp: mark the columns within the new threshold
+                    // (one compare and one select per column, the same
+                    // instructions in every lane).  Usually only the minimum
+                    // is marked and goes into the list directly; a row with
+                    // several marked columns inserts them one by one.
+                    const bool need = mn <= T;
+                    if (__any_sync(0xFFFFFFFFu, need)) {
+                        const float Tn = need ? assign_threshold(fminf(d1, mn), sq, delta, e) : T;
+                        uint32_t msk = 0u;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) top4_insert(v[i], c0 + i, d1, d2, d3, d4, i1, i2, i3, i4);
+                        for (int i = 0; i < 32; ++i) msk |= __uint_as_float(r[i]) <= Tn ? (1u << i) : 0u;
+                        if (need) {
+                            T = Tn;
+                            const int c0 = ch * p.CH + cg;
+                            // marked columns in turn; the value of column i is
+                            // picked from the 32 registers by a select tree on i
+                            for (uint32_t mm = msk; mm != 0u; mm &= mm - 1u) {
+                                const int i = __ffs(mm) - 1;
+                                top4_insert(pick32(r, i), c0 + i, d1, d2, d3, d4, i1, i2, i3, i4);
+                            }
+                        }
                     }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) cq[q] = cqn[q];
                 }
                 tc_fence_before();
                 mbar_arrive(ABAR(B_AE + s));
@@ -343,9 +423,6 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                 top4_insert(od.z, oi.z, d1, d2, d3, d4, i1, i2, i3, i4);
                 top4_insert(od.w, oi.w, d1, d2, d3, d4, i1, i2, i3, i4);
                 if (valid) {
-                    const float sq = p.rowsq ? p.rowsq[f] : 1.f;
-                    const float delta = __uint_as_float(p.hstat[2 * h]);
-                    const float e = p.e_tc * (sq + __uint_as_float(p.hstat[2 * h + 1]));
                     const float ub = d1 + assign_bound(d1, sq, delta, e);
                     const bool a2 = i2 >= 0 && d2 - assign_bound(d2, sq, delta, e) <= ub;
                     const bool a3 = i3 >= 0 && d3 - assign_bound(d3, sq, delta, e) <= ub;
