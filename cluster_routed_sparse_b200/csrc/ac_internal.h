@@ -148,7 +148,7 @@ struct FastAssignArgs {
     const int *nrows; int nrows_const;
     const float *C; int64_t cstride;
     const int *ncent; int ncent_const;
-    int Cpad, CH;              // CH <= 256, <= 128 with two terms
+    int Cpad, CH;              // CH <= 128, <= 96 with two terms
     bool two_term;             // centres as bf16 c_hi + c_lo (else c_hi alone)
     bf16 *Chi; float *cn; unsigned int *hstat;
     int *labels;

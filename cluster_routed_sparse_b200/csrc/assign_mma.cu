@@ -25,36 +25,40 @@
 namespace ac {
 namespace {
 
-constexpr int AM = 128;       // rows per tile (MMA M)
-constexpr int ACH_MAX = 256;  // centres per chunk (MMA N at most; 128 with two terms)
-constexpr int A_EPI = 256;    // epilogue threads: two warpgroups
+constexpr int AM = 128;       // rows per MMA (M)
+constexpr int AU = 2 * AM;    // rows per work unit: two MMAs share every centre chunk
+constexpr int ACH = 128;      // centres per chunk at most (MMA N)
+constexpr int A_EPI = 256;    // epilogue threads: one per row of the unit
 constexpr int A_THREADS = A_EPI + 64;
+constexpr int A_NCMAX = 3;    // centre chunk stages (2 with two-term centres)
 
+// Shared memory: [2] row units (two 128-row tiles each) | [NC] centre chunks.
+// A chunk holds the c_hi rows (and the c_lo rows) of up to ACH centres, each
+// operand as [column half][rows][128 B] with the 128-byte swizzle.
 template <int D>
 struct ALayout {
     static constexpr int HALVES = D / 64;
-    static constexpr uint32_t X_BYTES = HALVES * AM * 128;        // one row tile
-    static constexpr uint32_t C_BYTES = HALVES * ACH_MAX * 128;   // one centre chunk (c_hi [, c_lo])
-    static constexpr uint32_t OFF_X = 0;                           // [2] row tiles
-    static constexpr uint32_t OFF_C = OFF_X + 2 * X_BYTES;         // [2] centre chunks
-    static constexpr uint32_t OFF_MG = OFF_C + 2 * C_BYTES;        // [2][AM][8] top-4 hand-over
-    static constexpr uint32_t OFF_BAR = OFF_MG + 2 * AM * 8 * 4;
+    static constexpr uint32_t XT_BYTES = HALVES * AM * 128;  // one 128-row tile
+    static constexpr uint32_t X_BYTES = 2 * XT_BYTES;        // one unit
+    static constexpr uint32_t OFF_X = 0;
+    static constexpr uint32_t OFF_C = OFF_X + 2 * X_BYTES;
+    // three c_hi stages of ACH centres, or two c_hi + c_lo stages of up to 96
+    static constexpr uint32_t C_REGION = 3 * HALVES * ACH * 128;
+    static constexpr uint32_t OFF_BAR = OFF_C + C_REGION;
     static constexpr uint32_t BYTES = OFF_BAR + 256;
     static constexpr uint32_t SMEM = BYTES + 1024;
 };
 
 // barriers
 enum {
-    B_XF = 0,   // [2] row tile landed
-    B_XE = 2,   // [2] row tile consumed by the MMAs
-    B_CF = 4,   // [2] centre chunk landed
-    B_CE = 6,   // [2] centre chunk consumed
-    B_AF = 8,   // [2] accumulator chunk ready
-    B_AE = 10,  // [2] accumulator chunk drained (256 arrivals)
-    B_MG = 12,  // [2] upper warpgroup's top-4 written (128 arrivals)
-    B_MR = 14,  // [2] hand-over slot read (128 arrivals)
-    B_DONE = 16,
-    B_N = 17
+    B_XF = 0,    // [2] row unit landed
+    B_XE = 2,    // [2] row unit consumed by the MMAs
+    B_CF = 4,    // [3] centre chunk landed
+    B_CE = 7,    // [3] centre chunk consumed
+    B_AF = 10,   // [2] accumulators of a chunk ready
+    B_AE = 12,   // [2] accumulators drained (256 arrivals)
+    B_DONE = 14,
+    B_N = 15
 };
 
 struct AsgParams {
@@ -65,8 +69,10 @@ struct AsgParams {
     const int *nrows; int nrows_const;
     const int *ncent; int ncent_const;
     int64_t L;
-    int BH, Cpad, CH, tiles_per_unit;
+    int BH, Cpad, CH, units_per_head;
     int two_term;         // c' = c_hi + c_lo (else c_hi)
+    int nc;               // centre chunk stages
+    uint32_t c_stage;     // bytes of one centre chunk stage
     float e_tc;           // tensor-core error coefficient (see assign_bound)
     int *labels;
     int4 *cand;
@@ -162,16 +168,17 @@ __global__ void __launch_bounds__(A_THREADS, 1)
     const uint32_t bar0 = sbase + LY::OFF_BAR;
 #define ABAR(i) (bar0 + 8u * (uint32_t)(i))
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + LY::OFF_BAR + 8 * B_N);
+    const int nc = p.nc;
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(ABAR(B_XF + i), 1);
             mbar_init(ABAR(B_XE + i), 1);
-            mbar_init(ABAR(B_CF + i), 1);
-            mbar_init(ABAR(B_CE + i), 1);
             mbar_init(ABAR(B_AF + i), 1);
             mbar_init(ABAR(B_AE + i), A_EPI);
-            mbar_init(ABAR(B_MG + i), 128);
-            mbar_init(ABAR(B_MR + i), 128);
+        }
+        for (int i = 0; i < A_NCMAX; ++i) {
+            mbar_init(ABAR(B_CF + i), 1);
+            mbar_init(ABAR(B_CE + i), 1);
         }
         mbar_init(ABAR(B_DONE), 1);
         fence_mbar_init();
@@ -184,63 +191,65 @@ __global__ void __launch_bounds__(A_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int ntiles = p.BH * p.tiles_per_unit;
+    const int nunits = p.BH * p.units_per_head;
+    const uint32_t terms = p.two_term ? 2u : 1u;
     bool ok = true;
 
     if (warp == 8) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t g = 0, tc = 0;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const int h = t / p.tiles_per_unit, rt = t % p.tiles_per_unit;
+            uint32_t g = 0, uc = 0;
+            for (int t = blockIdx.x; t < nunits && ok; t += gridDim.x) {
+                const int h = t / p.units_per_head, ru = t % p.units_per_head;
                 const int n = p.nrows ? p.nrows[h] : p.nrows_const;
                 const int m = p.ncent ? p.ncent[h] : p.ncent_const;
-                if (rt * AM >= n || m <= 0) continue;
-                const uint32_t xs = tc & 1;
-                if (tc >= 2 && !mbar_wait_or_abort(ABAR(B_XE + xs), ((tc >> 1) - 1) & 1, p.err)) {
+                if (ru * AU >= n || m <= 0) continue;
+                const uint32_t xs = uc & 1;
+                if (uc >= 2 && !mbar_wait_or_abort(ABAR(B_XE + xs), ((uc >> 1) - 1) & 1, p.err)) {
                     ok = false;
                     break;
                 }
                 mbar_arrive_expect_tx(ABAR(B_XF + xs), LY::X_BYTES);
-                for (int hf = 0; hf < LY::HALVES; ++hf)
-                    tma_load_2d(sbase + LY::OFF_X + xs * LY::X_BYTES + hf * AM * 128, &tm_x, hf * 64,
-                                (int)(h * p.L + rt * AM), ABAR(B_XF + xs));
-                ++tc;
+                for (int i = 0; i < 2; ++i)
+                    for (int hf = 0; hf < LY::HALVES; ++hf)
+                        tma_load_2d(sbase + LY::OFF_X + xs * LY::X_BYTES + i * LY::XT_BYTES + hf * AM * 128, &tm_x,
+                                    hf * 64, (int)(h * p.L + ru * AU + i * AM), ABAR(B_XF + xs));
+                ++uc;
                 const int nch = (m + p.CH - 1) / p.CH;
                 for (int ch = 0; ch < nch; ++ch, ++g) {
-                    const uint32_t s = g & 1;
-                    if (g >= 2 && !mbar_wait_or_abort(ABAR(B_CE + s), ((g >> 1) - 1) & 1, p.err)) {
+                    const uint32_t c = g % nc, k = g / nc;
+                    if (g >= (uint32_t)nc && !mbar_wait_or_abort(ABAR(B_CE + c), (k - 1) & 1, p.err)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t terms = p.two_term ? 2u : 1u;
-                    mbar_arrive_expect_tx(ABAR(B_CF + s), terms * LY::HALVES * p.CH * 128);
+                    const uint32_t cs = sbase + LY::OFF_C + c * p.c_stage;
+                    mbar_arrive_expect_tx(ABAR(B_CF + c), terms * LY::HALVES * p.CH * 128);
                     for (int hf = 0; hf < LY::HALVES; ++hf)
-                        tma_load_2d(sbase + LY::OFF_C + s * LY::C_BYTES + hf * p.CH * 128, &tm_c, hf * 64,
-                                    h * p.Cpad + ch * p.CH, ABAR(B_CF + s));
-                    if (p.two_term)  // c_lo rows follow c_hi rows in the tensor map
+                        tma_load_2d(cs + hf * p.CH * 128, &tm_c, hf * 64, h * p.Cpad + ch * p.CH, ABAR(B_CF + c));
+                    if (p.two_term)  // c_lo rows follow the c_hi rows of all units in the tensor map
                         for (int hf = 0; hf < LY::HALVES; ++hf)
-                            tma_load_2d(sbase + LY::OFF_C + s * LY::C_BYTES + (LY::HALVES + hf) * p.CH * 128, &tm_c,
-                                        hf * 64, (p.BH + h) * p.Cpad + ch * p.CH, ABAR(B_CF + s));
+                            tma_load_2d(cs + (LY::HALVES + hf) * p.CH * 128, &tm_c, hf * 64,
+                                        (p.BH + h) * p.Cpad + ch * p.CH, ABAR(B_CF + c));
                 }
             }
             // nothing may still be landing in shared memory when the block exits
-            for (uint32_t k = (g >= 2 ? g - 2 : 0); k < g; ++k) mbar_wait(ABAR(B_CF + (k & 1)), (k >> 1) & 1);
-            for (uint32_t k = (tc >= 2 ? tc - 2 : 0); k < tc; ++k) mbar_wait(ABAR(B_XF + (k & 1)), (k >> 1) & 1);
+            for (uint32_t k = (g >= (uint32_t)nc ? g - nc : 0); k < g; ++k)
+                mbar_wait(ABAR(B_CF + (k % nc)), (k / nc) & 1);
+            for (uint32_t k = (uc >= 2 ? uc - 2 : 0); k < uc; ++k) mbar_wait(ABAR(B_XF + (k & 1)), (k >> 1) & 1);
             if (!ok) set_err(p.err, DEV_ERR_TIMEOUT);
         }
         __syncwarp();
     } else if (warp == 9) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            uint32_t g = 0, tc = 0;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const int h = t / p.tiles_per_unit, rt = t % p.tiles_per_unit;
+            uint32_t g = 0, uc = 0;
+            for (int t = blockIdx.x; t < nunits && ok; t += gridDim.x) {
+                const int h = t / p.units_per_head, ru = t % p.units_per_head;
                 const int n = p.nrows ? p.nrows[h] : p.nrows_const;
                 const int m = p.ncent ? p.ncent[h] : p.ncent_const;
-                if (rt * AM >= n || m <= 0) continue;
-                const uint32_t xs = tc & 1;
-                if (!mbar_wait_or_abort(ABAR(B_XF + xs), (tc >> 1) & 1, p.err)) {
+                if (ru * AU >= n || m <= 0) continue;
+                const uint32_t xs = uc & 1;
+                if (!mbar_wait_or_abort(ABAR(B_XF + xs), (uc >> 1) & 1, p.err)) {
                     ok = false;
                     break;
                 }
@@ -248,9 +257,9 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                 const uint32_t xa = sbase + LY::OFF_X + xs * LY::X_BYTES;
                 const int nch = (m + p.CH - 1) / p.CH;
                 for (int ch = 0; ch < nch; ++ch, ++g) {
-                    const uint32_t s = g & 1;
-                    if (!mbar_wait_or_abort(ABAR(B_CF + s), (g >> 1) & 1, p.err) ||
-                        (g >= 2 && !mbar_wait_or_abort(ABAR(B_AE + s), ((g >> 1) - 1) & 1, p.err))) {
+                    const uint32_t c = g % nc, a = g & 1;
+                    if (!mbar_wait_or_abort(ABAR(B_CF + c), (g / nc) & 1, p.err) ||
+                        (g >= 2 && !mbar_wait_or_abort(ABAR(B_AE + a), ((g >> 1) - 1) & 1, p.err))) {
                         ok = false;
                         break;
                     }
@@ -258,21 +267,23 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                     const int rem = m - ch * p.CH;
                     const int N = rem >= p.CH ? p.CH : ((rem + 31) & ~31);
                     const uint32_t idesc = idesc_bf16_f32(AM, N, false);
-                    const uint32_t ca = sbase + LY::OFF_C + s * LY::C_BYTES;
-                    const int nk = (p.two_term ? 2 : 1) * (D / 16);
-                    for (int kk = 0; kk < nk; ++kk) {
-                        const int kx = kk % (D / 16);  // x . c_hi, then x . c_lo
-                        const uint32_t xoff = (kx >> 2) * (AM * 128) + (kx & 3) * 32;
-                        const uint32_t coff = (kk >> 2) * (p.CH * 128) + (kk & 3) * 32;
-                        tc_mma_bf16(tmem + s * ACH_MAX, sdesc_sw128(xa + xoff, 16, 1024),
-                                    sdesc_sw128(ca + coff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                    const uint32_t ca = sbase + LY::OFF_C + c * p.c_stage;
+                    const int nk = (int)terms * (D / 16);
+                    for (int i = 0; i < 2; ++i) {
+                        for (int kk = 0; kk < nk; ++kk) {
+                            const int kx = kk % (D / 16);  // x . c_hi, then x . c_lo
+                            const uint32_t xoff = i * LY::XT_BYTES + (kx >> 2) * (AM * 128) + (kx & 3) * 32;
+                            const uint32_t coff = (kk >> 2) * (p.CH * 128) + (kk & 3) * 32;
+                            tc_mma_bf16(tmem + (a * 2 + i) * ACH, sdesc_sw128(xa + xoff, 16, 1024),
+                                        sdesc_sw128(ca + coff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                        }
                     }
-                    tc_commit(ABAR(B_AF + s));
-                    tc_commit(ABAR(B_CE + s));
+                    tc_commit(ABAR(B_AF + a));
+                    tc_commit(ABAR(B_CE + c));
                 }
                 if (!ok) break;
                 tc_commit(ABAR(B_XE + xs));
-                ++tc;
+                ++uc;
             }
             tc_commit(ABAR(B_DONE));
             if (!mbar_wait(ABAR(B_DONE), 0)) ok = false;
@@ -281,26 +292,25 @@ __global__ void __launch_bounds__(A_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue
-        // Warpgroup wg takes the 32-column groups wg, wg + 2, ... of every
-        // chunk; warp w reads tensor-memory lanes 32 (w % 4) .. + 31, i.e. rows.
-        // A group costs one FMA and one min per centre: only groups whose
-        // minimum reaches the threshold T of assign_threshold (rare after the
-        // first) insert into the row's top-4 list.  The per-row and per-unit
-        // scalars of the next tile and the centre norms of the next group are
-        // loaded ahead, so no global load latency sits on the chunk path.
-        const int wg = warp >> 2;
-        const int rloc = (warp & 3) * 32 + lane;
+        // Warp w owns rows 32 (w % 4) .. + 31 of tile w / 4 of the unit (tensor
+        // memory lanes 32 (w % 4) ..), one row per thread, all centres.  A
+        // 32-column group costs one FMA and one min per centre; only groups
+        // whose minimum reaches the threshold T of assign_threshold (rare after
+        // the first ones) mark their columns under it and insert those into the
+        // row's top-4 list.  The per-row and per-unit scalars of the next unit
+        // and the centre norms of the next group are loaded ahead.
+        const int ti = warp >> 2;
+        const int rloc = ti * AM + (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        float *mg = reinterpret_cast<float *>(sm + LY::OFF_MG);
-        struct TileScalars {
+        struct UnitScalars {
             float inv, sq;
             uint32_t delta, cmax;
             int m;
         };
-        auto fetch = [&](int tt, TileScalars &v) {
-            if (tt >= ntiles) return;
-            const int hh = tt / p.tiles_per_unit;
-            const int row = (tt % p.tiles_per_unit) * AM + rloc;
+        auto fetch = [&](int tt, UnitScalars &v) {
+            if (tt >= nunits) return;
+            const int hh = tt / p.units_per_head;
+            const int row = (tt % p.units_per_head) * AU + rloc;
             const int nn = p.nrows ? p.nrows[hh] : p.nrows_const;
             const int64_t ff = (int64_t)hh * p.L + row;
             v.m = p.ncent ? p.ncent[hh] : p.ncent_const;
@@ -309,16 +319,21 @@ __global__ void __launch_bounds__(A_THREADS, 1)
             v.delta = p.hstat[2 * hh];
             v.cmax = p.hstat[2 * hh + 1];
         };
-        TileScalars cur{1.f, 1.f, 0u, 0u, 0}, nxt{1.f, 1.f, 0u, 0u, 0};
+        auto load_cn = [&](const float *src, float4 (&dst)[8]) {
+            const float4 *cn4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[q] = __ldg(cn4 + q);
+        };
+        UnitScalars cur{1.f, 1.f, 0u, 0u, 0}, nxt{1.f, 1.f, 0u, 0u, 0};
         fetch(blockIdx.x, cur);
-        uint32_t g = 0, tc = 0;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, cur = nxt) {
+        uint32_t g = 0;
+        for (int t = blockIdx.x; t < nunits && ok; t += gridDim.x, cur = nxt) {
             fetch(t + gridDim.x, nxt);
-            const int h = t / p.tiles_per_unit, rt = t % p.tiles_per_unit;
+            const int h = t / p.units_per_head, ru = t % p.units_per_head;
             const int n = p.nrows ? p.nrows[h] : p.nrows_const;
             const int m = cur.m;
-            if (rt * AM >= n || m <= 0) continue;
-            const int row = rt * AM + rloc;
+            if (ru * AU >= n || m <= 0) continue;
+            const int row = ru * AU + rloc;
             const bool valid = row < n;
             const int64_t f = (int64_t)h * p.L + row;
             const float m2i = -2.f * cur.inv;
@@ -330,30 +345,24 @@ __global__ void __launch_bounds__(A_THREADS, 1)
             int i1 = 0, i2 = -1, i3 = -1, i4 = -1;
             float T = INFINITY;
             const int nch = (m + p.CH - 1) / p.CH;
-            // the column groups of this warpgroup, over all chunks of the tile
             float4 cq[8];
-            auto load_cn = [&](int c0, float4 (&dst)[8]) {
-                const float4 *cn4 = reinterpret_cast<const float4 *>(cnh + c0);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) dst[q] = __ldg(cn4 + q);
-            };
-            if (wg * 32 < m) load_cn(wg * 32, cq);
+            load_cn(cnh, cq);
             for (int ch = 0; ch < nch; ++ch, ++g) {
-                const uint32_t s = g & 1;
+                const uint32_t a = g & 1;
                 const int rem = m - ch * p.CH;
                 const int N = rem >= p.CH ? p.CH : ((rem + 31) & ~31);
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(ABAR(B_AF + s), (g >> 1) & 1, p.err))) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(ABAR(B_AF + a), (g >> 1) & 1, p.err))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                for (int cg = wg * 32; cg < N; cg += 64) {
+                for (int cg = 0; cg < N; cg += 32) {
                     uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + s * ACH_MAX + cg, r);
-                    // next group of this warpgroup: same chunk, else the next chunk
+                    tmem_ld32(tmem + lane_off + (a * 2 + ti) * ACH + cg, r);
+                    // norms of the next group: same chunk, else the next chunk
                     float4 cqn[8];
-                    const int ncg = cg + 64 < N ? ch * p.CH + cg + 64 : (ch + 1) * p.CH + wg * 32;
-                    if (ncg < m) load_cn(ncg, cqn);
+                    const int ncg = cg + 32 < N ? ch * p.CH + cg + 32 : (ch + 1) * p.CH;
+                    if (ncg < m) load_cn(cnh + ncg, cqn);
                     tmem_ld_wait();
                     float mn = INFINITY;
 #pragma unroll
@@ -371,9 +380,7 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                     // This group holds the best so far or a near tie for some
                     // row of the warp: mark the columns within the new threshold
                     // (one compare and one select per column, the same
-                    // instructions in every lane).  Usually only the minimum
-                    // is marked and goes into the list directly; a row with
-                    // several marked columns inserts them one by one.
+                    // instructions in every lane), then insert the marked ones.
                     const bool need = mn <= T;
                     if (__any_sync(0xFFFFFFFFu, need)) {
                         const float Tn = need ? assign_threshold(fminf(d1, mn), sq, delta, e) : T;
@@ -383,8 +390,8 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                         if (need) {
                             T = Tn;
                             const int c0 = ch * p.CH + cg;
-                            // marked columns in turn; the value of column i is
-                            // picked from the 32 registers by a select tree on i
+                            // the value of column i is picked from the 32
+                            // registers by a select tree on i
                             for (uint32_t mm = msk; mm != 0u; mm &= mm - 1u) {
                                 const int i = __ffs(mm) - 1;
                                 top4_insert(pick32(r, i), c0 + i, d1, d2, d3, d4, i1, i2, i3, i4);
@@ -395,53 +402,26 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                     for (int q = 0; q < 8; ++q) cq[q] = cqn[q];
                 }
                 tc_fence_before();
-                mbar_arrive(ABAR(B_AE + s));
+                mbar_arrive(ABAR(B_AE + a));
             }
             if (!ok) break;
-            // hand the upper warpgroup's top-4 to the lower one
-            const uint32_t slot = tc & 1;
-            float *mrow = mg + ((int)slot * AM + rloc) * 8;
-            if (wg == 1) {
-                if (tc >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(ABAR(B_MR + slot), ((tc >> 1) - 1) & 1,
-                                                                           p.err))) {
-                    ok = false;
-                    break;
-                }
-                reinterpret_cast<float4 *>(mrow)[0] = make_float4(d1, d2, d3, d4);
-                reinterpret_cast<int4 *>(mrow)[1] = make_int4(i1, i2, i3, i4);
-                mbar_arrive(ABAR(B_MG + slot));
-            } else {
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(ABAR(B_MG + slot), (tc >> 1) & 1, p.err))) {
-                    ok = false;
-                    break;
-                }
-                const float4 od = reinterpret_cast<const float4 *>(mrow)[0];
-                const int4 oi = reinterpret_cast<const int4 *>(mrow)[1];
-                mbar_arrive(ABAR(B_MR + slot));
-                top4_insert(od.x, oi.x, d1, d2, d3, d4, i1, i2, i3, i4);
-                top4_insert(od.y, oi.y, d1, d2, d3, d4, i1, i2, i3, i4);
-                top4_insert(od.z, oi.z, d1, d2, d3, d4, i1, i2, i3, i4);
-                top4_insert(od.w, oi.w, d1, d2, d3, d4, i1, i2, i3, i4);
-                if (valid) {
-                    const float ub = d1 + assign_bound(d1, sq, delta, e);
-                    const bool a2 = i2 >= 0 && d2 - assign_bound(d2, sq, delta, e) <= ub;
-                    const bool a3 = i3 >= 0 && d3 - assign_bound(d3, sq, delta, e) <= ub;
-                    const bool a4 = i4 >= 0 && d4 - assign_bound(d4, sq, delta, e) <= ub;
-                    // A - E(A) grows with A once sqrt(dup) > delta, so the centres
-                    // beyond the kept four are settled when the fourth is.
-                    const bool beyond =
-                        m > 4 && (a4 || sqrtf(fmaxf(d4 + sq, 0.f) + 2.f * e) <= 2.f * delta);
-                    p.labels[f] = i1;
-                    if (a2 || a3 || a4 || beyond) {
-                        const int pos = atomicAdd(p.amb_count, 1);
-                        p.amb_list[pos] = (int)f;
-                        p.cand[pos] = beyond ? make_int4(-2, 0, 0, 0)
-                                             : make_int4(i1, a2 ? i2 : -1, a3 ? i3 : -1, a4 ? i4 : -1);
-                        if (beyond) atomicAdd(p.stats + 1, 1ull);
-                    }
+            if (valid) {
+                const float ub = d1 + assign_bound(d1, sq, delta, e);
+                const bool a2 = i2 >= 0 && d2 - assign_bound(d2, sq, delta, e) <= ub;
+                const bool a3 = i3 >= 0 && d3 - assign_bound(d3, sq, delta, e) <= ub;
+                const bool a4 = i4 >= 0 && d4 - assign_bound(d4, sq, delta, e) <= ub;
+                // A - E(A) grows with A once sqrt(dup) > delta, so the centres
+                // beyond the kept four are settled when the fourth is.
+                const bool beyond = m > 4 && (a4 || sqrtf(fmaxf(d4 + sq, 0.f) + 2.f * e) <= 2.f * delta);
+                p.labels[f] = i1;
+                if (a2 || a3 || a4 || beyond) {
+                    const int pos = atomicAdd(p.amb_count, 1);
+                    p.amb_list[pos] = (int)f;
+                    p.cand[pos] = beyond ? make_int4(-2, 0, 0, 0)
+                                         : make_int4(i1, a2 ? i2 : -1, a3 ? i3 : -1, a4 ? i4 : -1);
+                    if (beyond) atomicAdd(p.stats + 1, 1ull);
                 }
             }
-            ++tc;
         }
         if (!ok) set_err(p.err, DEV_ERR_TIMEOUT);
     }
@@ -624,6 +604,8 @@ __global__ void k_centre_prep(const float *__restrict__ C, int64_t cstride, cons
     }
 }
 
+static_assert(ALayout<128>::SMEM <= 232448, "assignment kernel exceeds the shared memory of a block");
+
 template <int D>
 cudaError_t launch_mma(const FastAssignArgs &a, const AsgParams &p, int grid, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(k_assign_mma<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -668,7 +650,7 @@ cudaError_t launch_assign_fast(const FastAssignArgs &a, cudaStream_t s) {
     p.BH = BH;
     p.Cpad = a.Cpad;
     p.CH = a.CH;
-    p.tiles_per_unit = (int)((a.L + AM - 1) / AM);
+    p.units_per_head = (int)((a.L + AU - 1) / AU);
     p.two_term = a.two_term ? 1 : 0;
     p.e_tc = (float)(a.two_term ? 2 * a.d : a.d) * 1.1920928955078125e-07f;  // products * 2^-23
     p.labels = a.labels;
@@ -677,8 +659,14 @@ cudaError_t launch_assign_fast(const FastAssignArgs &a, cudaStream_t s) {
     p.amb_count = a.amb_count;
     p.stats = a.stats;
     p.err = a.err;
-    const int ntiles = BH * p.tiles_per_unit;
-    const int grid = ntiles < a.num_sms ? ntiles : a.num_sms;
+    p.c_stage = (uint32_t)((a.two_term ? 2 : 1) * (a.d / 64) * a.CH * 128);
+    p.nc = a.two_term ? 2 : 3;
+    // the centre stages must fit their region of shared memory
+    if (a.CH < 32 || a.CH > ACH || (a.CH & 31) || (a.two_term && a.CH > 96) || (a.Cpad & 31) ||
+        (uint64_t)p.nc * p.c_stage > 3ull * (a.d / 64) * ACH * 128)
+        return cudaErrorInvalidValue;
+    const int nunits = BH * p.units_per_head;
+    const int grid = nunits < a.num_sms ? nunits : a.num_sms;
     e = a.d == 128 ? launch_mma<128>(a, p, grid, s) : launch_mma<64>(a, p, grid, s);
     if (e != cudaSuccess) return e;
     // 3. exact rescoring of the uncertain rows
