@@ -426,6 +426,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     if (cfg->tau_mode == AC_TAU_PERCENTILE && (cfg->tau_value < 1.f || cfg->tau_value > 1000.f))
         return AC_ERR_INVALID_ARG;
     if ((int64_t)cfg->n_max + cfg->m0 > 16384) return AC_ERR_INVALID_ARG;
+    if (((int64_t)cfg->Cq + 64) * d * 4 > 200 * 1024) return AC_ERR_INVALID_ARG;  // query centroids staged whole
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return AC_ERR_UNSUPPORTED;

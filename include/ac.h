@@ -103,8 +103,11 @@ typedef struct ac_stage_times {
 } ac_stage_times;
 
 /* Create a context for [B, H, L, d] layers and allocate its workspace.
- * cfg is copied.  Requires B, H, L >= 1; d in {64, 128}; 1 <= Cq <= L;
- * 1 <= m0 <= L; n_max >= 1; iteration counts >= 0; an sm_100 device current.
+ * cfg is copied.  Requires B, H, L >= 1; d in {64, 128}; 1 <= Cq <= L and
+ * (Cq + 64) * d * 4 <= 200 KiB (Cq <= 336 at d = 128: the query centroids of
+ * a head are staged whole in shared memory for Eq. (1)); 1 <= m0 <= L;
+ * n_max >= 1; n_max + m0 <= 16384; iteration counts >= 0; an sm_100 device
+ * current.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 AC_API ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32_t d,
                     ac_ctx **out);
