@@ -78,10 +78,11 @@ ac_status make_tmap(ac_ctx *c, CUtensorMap *tm, void *base, int64_t rows, int d,
     return AC_OK;
 }
 
-// K and V boxes: 8 rows x all d columns in one copy, laid out in shared memory
-// as [column half][8 rows][64 columns] (dims: column, row, half; the half
-// stride is 128 bytes, the row stride d*2 bytes), 128-byte swizzle.
-ac_status make_tmap_kv(ac_ctx *c, CUtensorMap *tm, void *base, int64_t rows, int d) {
+// K and V boxes of G 8-row groups x all d columns in one copy, laid out in
+// shared memory as [group][column half][8 rows][64 columns] (dims: column,
+// row in group, half, group; strides d*2, 128 and 8*d*2 bytes), 128-byte
+// swizzle.  The rows must be group-aligned, as the padded Kp / Vp are.
+ac_status make_tmap_kv(ac_ctx *c, CUtensorMap *tm, void *base, int64_t groups, int d, int G) {
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
         cudaDriverEntryPointQueryResult q;
@@ -92,14 +93,14 @@ ac_status make_tmap_kv(ac_ctx *c, CUtensorMap *tm, void *base, int64_t rows, int
         fn = reinterpret_cast<EncodeTiledFn>(p);
     }
     const int halves = d / 64;
-    cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)halves};
-    cuuint64_t strides[2] = {(cuuint64_t)d * 2, 128};
-    cuuint32_t box[3] = {64, 8, (cuuint32_t)halves};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+    cuuint64_t dims[4] = {64, 8, (cuuint64_t)halves, (cuuint64_t)groups};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, 128, (cuuint64_t)d * 16};
+    cuuint32_t box[4] = {64, 8, (cuuint32_t)halves, (cuuint32_t)G};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(c, AC_ERR_CUDA, "cuTensorMapEncodeTiled (K/V boxes) failed");
+    if (r != CUDA_SUCCESS) return fail(c, AC_ERR_CUDA, "cuTensorMapEncodeTiled (K/V group boxes) failed");
     return AC_OK;
 }
 
@@ -367,18 +368,19 @@ ac_status key_stats_impl(ac_ctx *c, const bf16 *K, cudaStream_t s) {
 ac_status score_select_impl(ac_ctx *c, int topk, cudaStream_t s) {
     SelectArgs a{c->cent_q, c->kmax, c->kmin, c->counts_k, c->n_k, c->dense, c->offs_k, c->counts_q,
                  c->Cq, c->Ccap, c->d, c->BH, c->L, topk != 0 ? topk : c->cfg.topk,
-                 c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->rbox};
+                 c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->rbox, c->pgoff, c->nrange};
     CK(launch_score_select(a, s), "score select");
     return AC_OK;
 }
 
 ac_status sparse_attn_impl(ac_ctx *c, const bf16 *Q, const bf16 *K, const bf16 *V, bf16 *O, cudaStream_t s) {
     CK(launch_permute_rows(Q, c->perm_q, c->Qp, c->L, c->d, c->BH, s), "permute q");
-    CK(launch_permute_rows(K, c->perm_k, c->Kp, c->L, c->d, c->BH, s), "permute k");
-    CK(launch_permute_rows(V, c->perm_k, c->Vp, c->L, c->d, c->BH, s), "permute v");
+    CK(launch_permute_kv_padded(K, V, c->perm_k, c->labels_k, c->offs_k, c->Ccap + 1, c->pgoff, c->Ccap, c->Kp, c->Vp,
+                                c->L, c->Lpad, c->d, c->BH, s),
+       "permute k, v");
     CK(cudaMemsetAsync(c->counters, 0, 8 * sizeof(unsigned long long), s), "counters");
-    AttnArgs a{&c->tm_q, &c->tm_k, &c->tm_v, O, c->perm_q, c->offs_q, c->counts_q, c->tile_prefix, c->ranges,
-               c->nboxes, c->ksel, c->rbox, c->dense, c->L, c->Cq, c->Ccap, c->BH, c->d,
+    AttnArgs a{&c->tm_q, c->tm_kg, c->tm_vg, O, c->perm_q, c->offs_q, c->counts_q, c->tile_prefix, c->ranges,
+               c->nboxes, c->nrange, c->rbox, c->L, c->Lpad, c->Cq, c->Ccap, c->BH, c->d,
                (float)(c->scale * 1.4426950408889634), c->err, c->counters};
     if (c->timing) CK(cudaEventRecord(c->ev[6], s), "event");
     CK(launch_sparse_attn(a, s), "sparse attention");
@@ -393,7 +395,7 @@ void free_all(ac_ctx *c) {
                    c->u_cnt, c->st_m, c->st_labels, c->st_dist, c->st_perm, c->st_offs, c->st_counts, c->radix,
                    c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->Qp, c->Kp, c->Vp,
                    c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err, c->chi_q, c->chi_k, c->cn,
-                   c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats, c->rbox};
+                   c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats, c->rbox, c->pgoff, c->nrange};
     for (void *p : dev)
         if (p) cudaFree(p);
     void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err};
@@ -444,6 +446,11 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     c->BH = B * H;
     c->Cq = cfg->Cq;
     c->Ccap = cfg->n_max + cfg->m0;
+    c->Lpad = ((L + 7) & ~7) + 8 * c->Ccap + 8;  // keys padded per cluster; the last group stays zero
+    if ((int64_t)c->B * c->H * c->Lpad >= (int64_t)1 << 31) {
+        delete c;
+        return AC_ERR_INVALID_ARG;
+    }
     c->device = dev;
     c->scale = cfg->scale > 0.f ? cfg->scale : 1.0f / std::sqrt((float)d);
 
@@ -509,8 +516,10 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->amb_count, 1));
     A(dalloc(&c->asg_stats, 2));
     A(dalloc(&c->Qp, BH * Lz * dz));
-    A(dalloc(&c->Kp, BH * Lz * dz));
-    A(dalloc(&c->Vp, BH * Lz * dz));
+    A(dalloc(&c->Kp, BH * (size_t)c->Lpad * dz));
+    A(dalloc(&c->Vp, BH * (size_t)c->Lpad * dz));
+    A(dalloc(&c->pgoff, BH * Cc));
+    A(dalloc(&c->nrange, BH * Cq));
     A(dalloc(&c->counters, 8));
     A(dalloc(&c->err, 1));
     A(cudaMallocHost(&c->h_u_cnt, BH * sizeof(int)));
@@ -527,14 +536,20 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     }
     if (cudaMemset(c->err, 0, sizeof(uint32_t)) != cudaSuccess ||
         cudaMemset(c->asg_stats, 0, 2 * sizeof(unsigned long long)) != cudaSuccess ||
-        cudaMemset(c->dense, 0, BH) != cudaSuccess || cudaMemset(c->n_k, 0, BH * sizeof(int)) != cudaSuccess) {
+        cudaMemset(c->dense, 0, BH) != cudaSuccess || cudaMemset(c->n_k, 0, BH * sizeof(int)) != cudaSuccess ||
+        // padding rows of Kp / Vp are read (and masked) by the attention: keep them finite
+        cudaMemset(c->Kp, 0, BH * (size_t)c->Lpad * dz * sizeof(bf16)) != cudaSuccess ||
+        cudaMemset(c->Vp, 0, BH * (size_t)c->Lpad * dz * sizeof(bf16)) != cudaSuccess) {
         free_all(c);
         delete c;
         return AC_ERR_CUDA;
     }
     const int64_t rows = (int64_t)BH * L;
-    if (make_tmap(c, &c->tm_q, c->Qp, rows, d, 128) != AC_OK || make_tmap_kv(c, &c->tm_k, c->Kp, rows, d) != AC_OK ||
-        make_tmap_kv(c, &c->tm_v, c->Vp, rows, d) != AC_OK ||
+    bool maps_ok = make_tmap(c, &c->tm_q, c->Qp, rows, d, 128) == AC_OK;
+    for (int i = 0; i < 4 && maps_ok; ++i)
+        maps_ok = make_tmap_kv(c, &c->tm_kg[i], c->Kp, (int64_t)BH * c->Lpad / 8, d, 1 << i) == AC_OK &&
+                  make_tmap_kv(c, &c->tm_vg[i], c->Vp, (int64_t)BH * c->Lpad / 8, d, 1 << i) == AC_OK;
+    if (!maps_ok ||
         make_tmap(c, &c->tm_chi_q, c->chi_q, (int64_t)2 * BH * c->Cpad_q, d, c->CH_q) != AC_OK ||
         make_tmap(c, &c->tm_chi_k, c->chi_k, (int64_t)BH * c->Cpad_k, d, c->CH_k) != AC_OK) {
         free_all(c);

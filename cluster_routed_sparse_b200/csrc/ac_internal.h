@@ -82,9 +82,15 @@ struct ac_ctx {
     long long n_fast, n_exact, n_fast_rows;
 
     // ---- attention
-    bf16 *Qp, *Kp, *Vp;  // [BH, L, d] cluster-order copies
+    bf16 *Qp;          // [BH, L, d] queries in cluster order
+    bf16 *Kp, *Vp;     // [BH, Lpad, d] keys / values in cluster order, every key
+                       // cluster starting on an 8-row group (padding rows zero)
+    int Lpad;          // rows per unit of Kp / Vp: L rounded up to 8, plus 8 per cluster
+    int *pgoff;        // [BH, Ccap] first 8-row group of each key cluster in Kp / Vp
+    int *nrange;       // [BH*Cq] key ranges the attention walks (k, or all clusters when dense)
     unsigned long long *counters;  // [8] kept pairs, computed pairs, items, -, first wait failure
-    CUtensorMap tm_q, tm_k, tm_v;
+    CUtensorMap tm_q;
+    CUtensorMap tm_kg[4], tm_vg[4];  // K / V boxes of 1, 2, 4, 8 row groups
 
     // ---- host-buffer forward
     uint16_t *hbufQ, *hbufK, *hbufV, *hbufO;  // device staging of the host entry point
@@ -225,21 +231,25 @@ cudaError_t launch_key_stats(const StatsArgs &a, cudaStream_t s);
 
 cudaError_t launch_permute_rows(const bf16 *X, const int *perm, bf16 *Xp, int64_t L, int d, int BH,
                                 cudaStream_t s);
+// Kp / Vp row 8 pgoff[h, c] + i = K / V row of the i-th key of cluster c.
+cudaError_t launch_permute_kv_padded(const bf16 *K, const bf16 *V, const int *perm, const int *labels,
+                                     const int *offs, int offs_stride, const int *pgoff, int Ccap, bf16 *Kp,
+                                     bf16 *Vp, int64_t L, int64_t Lpad, int d, int BH, cudaStream_t s);
 
 struct SelectArgs {
     const float *cent_q; const bf16 *kmax; const bf16 *kmin; const int *counts_k;
     const int *n_k; const uint8_t *dense; const int *offs_k; const int *counts_q;
     int Cq, Ccap, d, BH, L, topk;
     float *score; int *sel; int *ksel; int2 *ranges; int *nboxes; int *tile_prefix;
-    int *rbox;
+    int *rbox; int *pgoff; int *nrange;
 };
 cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s);
 
 struct AttnArgs {
-    const CUtensorMap *tm_q, *tm_k, *tm_v;
+    const CUtensorMap *tm_q, *tm_kg, *tm_vg;  // tm_kg / tm_vg: [4] box sizes
     bf16 *O; const int *perm_q; const int *offs_q; const int *counts_q;
-    const int *tile_prefix; const int2 *ranges; const int *nboxes; const int *ksel; const int *rbox;
-    const uint8_t *dense; int L, Cq, Ccap, BH, d;
+    const int *tile_prefix; const int2 *ranges; const int *nboxes; const int *nrange; const int *rbox;
+    int L, Lpad, Cq, Ccap, BH, d;
     float scale_log2;
     uint32_t *err; unsigned long long *counters;
 };

@@ -92,12 +92,16 @@ __device__ __forceinline__ float exp2_poly(float x) {
     return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
+struct AttnMaps {
+    CUtensorMap q;
+    CUtensorMap k[4], v[4];  // boxes of 1, 2, 4, 8 row groups
+};
+
 struct AttnParams {
     bf16 *O;
-    const int *perm_q, *offs_q, *counts_q, *tile_prefix, *nboxes, *ksel, *rbox;
-    const int2 *ranges;
-    const uint8_t *dense;
-    int L, Cq, Ccap, BH;
+    const int *perm_q, *offs_q, *counts_q, *tile_prefix, *nboxes, *nrange, *rbox;
+    const int2 *ranges;  // (first 8-row group in Kp / Vp, keys)
+    int L, Lpad, Cq, Ccap, BH;
     float scale_log2;
     uint32_t *err;
     unsigned long long *counters;
@@ -115,8 +119,7 @@ __device__ __forceinline__ void record_wait_failure(const AttnParams &p, int rol
 
 template <int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    k_sparse_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+    k_sparse_attn(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     using LY = Layout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int n_tiles = (p.nboxes[hq] + BOXES - 1) / BOXES;
     const int2 *rg = p.ranges + (int64_t)hq * p.Ccap;
     const int *rb = p.rbox + (int64_t)hq * (p.Ccap + 1);
-    const int nr = p.dense[h] ? 1 : p.ksel[h];
+    const int nr = p.nrange[hq];
     const int nbox = p.nboxes[hq];
 
     const uint32_t bar0 = sbase + LY::OFF_BAR;
@@ -185,11 +188,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       reg_dealloc<kRegsOther>();
       if (warp == 8) {
         // ------------------------------------------------ TMA producer (whole warp)
-        // Key tile j is boxes 16j .. 16j+15 of the concatenated selected ranges.
-        // Lane l < 16 finds the range of box 16j + l by a binary search over
-        // the first boxes of 32 ranges from r0 (one tile spans at most 16
-        // ranges), then issues that box's K and V copies; lane 16 finds the
-        // range that starts the next tile.
+        // Key tile j is 8-row groups 16j .. 16j+15 of the concatenated walked
+        // ranges (every range starts on a group of the padded Kp / Vp).  At
+        // most 16 ranges meet a tile: lane l takes the part of range r0 + l
+        // inside it, sets its groups' column masks and copies them with as
+        // few boxes as possible (8, 4, 2, 1 groups); lanes 16-31 fill the
+        // slots past the last group from an all-zero group.
         int2 *rg_s = reinterpret_cast<int2 *>(sm + LY::OFF_RG);
         int *rb_s = reinterpret_cast<int *>(sm + LY::OFF_RB);
         const bool cached = nr <= RG_CACHE;
@@ -200,51 +204,62 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         const int2 *rgp = cached ? rg_s : rg;
         const int *rbp = cached ? rb_s : rb;
+        const int unit_group = h * (p.Lpad / 8);
+        const int zero_group = unit_group + p.Lpad / 8 - 1;  // never written: zero
         if (lane == 0) {
             mbar_arrive_expect_tx(BAR(B_QF), 2 * LY::Q_TILE);
             for (int t = 0; t < 2; ++t)
                 for (int hf = 0; hf < LY::HALVES; ++hf)
-                    tma_load_2d(sbase + LY::OFF_Q + t * LY::Q_TILE + hf * BM * 128, &tm_q, hf * 64,
+                    tma_load_2d(sbase + LY::OFF_Q + t * LY::Q_TILE + hf * BM * 128, &maps.q, hf * 64,
                                 (int)(unit_row + row0 + t * BM), BAR(B_QF));
         }
         int r0 = 0, issued = 0;
         for (int j = 0; j < n_tiles; ++j) {
             const int s = j % NS;
-            const int b = j * BOXES + lane;
-            const int pv = r0 + lane <= nr ? rbp[r0 + lane] : 0x7FFFFFFF;
-            int k = 0;
+            const int t0 = j * BOXES, t1 = t0 + BOXES;
+            const int r = r0 + lane;
+            const int rb0 = r <= nr ? rbp[r] : 0x7FFFFFFF;
+            const int rb1 = __shfl_down_sync(0xFFFFFFFFu, rb0, 1);
+            const bool mine = lane < BOXES && r < nr && rb0 < t1;
+            const int a0 = mine ? max(rb0, t0) : 0, a1 = mine ? min(rb1, t1) : 0;
+            int2 g = make_int2(0, 0);
+            if (mine) g = rgp[r];
+            uint32_t w[4] = {0u, 0u, 0u, 0u};
+            for (int sl = a0; sl < a1; ++sl) {
+                const int v = min(8, g.y - 8 * (sl - rb0));
+                const uint32_t byte = v >= 8 ? 0xFFu : ((1u << v) - 1u);
+                const int ls = sl - t0;
+                w[ls >> 2] |= byte << ((ls & 3) * 8);
+            }
 #pragma unroll
-            for (int st = 16; st >= 1; st >>= 1) {
-                const int v = __shfl_sync(0xFFFFFFFFu, pv, min(k + st, 31));
-                if (k + st <= 31 && v <= b) k += st;
-            }
-            const int r = r0 + k;
-            const int first = __shfl_sync(0xFFFFFFFFu, pv, k);
-            int start = 0, cnt = 0;
-            if (lane < BOXES && b < nbox) {
-                const int2 g = rgp[r];
-                const int o = (b - first) * 8;
-                start = g.x + o;
-                cnt = min(8, g.y - o);
-            }
-            const int rnext = __shfl_sync(0xFFFFFFFFu, r, BOXES);
-            uint32_t bits = lane < BOXES ? (cnt >= 8 ? 0xFFu : ((1u << cnt) - 1u)) << ((lane & 3) * 8) : 0u;
-            bits |= __shfl_xor_sync(0xFFFFFFFFu, bits, 1);
-            bits |= __shfl_xor_sync(0xFFFFFFFFu, bits, 2);
+            for (int q = 0; q < 4; ++q) w[q] = __reduce_or_sync(0xFFFFFFFFu, w[q]);
+            const int rnext = r0 + __popc(__ballot_sync(0xFFFFFFFFu, mine && rb1 <= t1));
             if (j >= NS && !__all_sync(0xFFFFFFFFu, WAIT(1, B_KVE + s, j, ((j / NS) - 1) & 1))) {
                 ok = false;
                 break;
             }
-            if (lane < BOXES && (lane & 3) == 0) masks[4 * s + (lane >> 2)] = bits;
+            if (lane < 4) masks[4 * s + lane] = lane == 0 ? w[0] : lane == 1 ? w[1] : lane == 2 ? w[2] : w[3];
             __syncwarp();
             if (lane == 0) mbar_arrive_expect_tx(BAR(B_KVF + s), 2 * LY::KV_BYTES);  // releases the masks
             __syncwarp();
-            if (lane < BOXES) {
-                const int row = (int)(unit_row + start);
-                tma_load_3d(sbase + LY::OFF_K + s * LY::KV_BYTES + lane * LY::BOX_BYTES, &tm_k, 0, row, 0,
-                            BAR(B_KVF + s));
-                tma_load_3d(sbase + LY::OFF_V + s * LY::KV_BYTES + lane * LY::BOX_BYTES, &tm_v, 0, row, 0,
-                            BAR(B_KVF + s));
+            const uint32_t kd = sbase + LY::OFF_K + s * LY::KV_BYTES;
+            const uint32_t vd = sbase + LY::OFF_V + s * LY::KV_BYTES;
+            if (mine) {
+                int ls = a0 - t0, gi = unit_group + g.x + (a0 - rb0), left = a1 - a0;
+                while (left > 0) {
+                    const int lg = left >= 8 ? 3 : left >= 4 ? 2 : left >= 2 ? 1 : 0;
+                    tma_load_4d(kd + ls * LY::BOX_BYTES, &maps.k[lg], 0, 0, 0, gi, BAR(B_KVF + s));
+                    tma_load_4d(vd + ls * LY::BOX_BYTES, &maps.v[lg], 0, 0, 0, gi, BAR(B_KVF + s));
+                    ls += 1 << lg;
+                    gi += 1 << lg;
+                    left -= 1 << lg;
+                }
+            }
+            const int filled = min(max(nbox - t0, 0), BOXES);
+            if (lane >= BOXES && lane - BOXES < BOXES - filled) {
+                const int ls = filled + lane - BOXES;
+                tma_load_4d(kd + ls * LY::BOX_BYTES, &maps.k[0], 0, 0, 0, zero_group, BAR(B_KVF + s));
+                tma_load_4d(vd + ls * LY::BOX_BYTES, &maps.v[0], 0, 0, 0, zero_group, BAR(B_KVF + s));
             }
             r0 = rnext;
             ++issued;
@@ -491,11 +506,17 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s) {
     p.counts_q = a.counts_q;
     p.tile_prefix = a.tile_prefix;
     p.nboxes = a.nboxes;
-    p.ksel = a.ksel;
     p.ranges = a.ranges;
     p.rbox = a.rbox;
-    p.dense = a.dense;
+    p.nrange = a.nrange;
+    p.Lpad = a.Lpad;
     p.L = a.L;
+    AttnMaps maps;
+    maps.q = *a.tm_q;
+    for (int i = 0; i < 4; ++i) {
+        maps.k[i] = a.tm_kg[i];
+        maps.v[i] = a.tm_vg[i];
+    }
     p.Cq = a.Cq;
     p.Ccap = a.Ccap;
     p.BH = a.BH;
@@ -508,13 +529,13 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s) {
         e = cudaFuncSetAttribute(k_sparse_attn<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)Layout<128>::SMEM);
         if (e != cudaSuccess) return e;
-        k_sparse_attn<128><<<grid, NTHREADS, Layout<128>::SMEM, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, p);
+        k_sparse_attn<128><<<grid, NTHREADS, Layout<128>::SMEM, s>>>(maps, p);
         AC_NOTE_LAUNCH();
     } else {
         e = cudaFuncSetAttribute(k_sparse_attn<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)Layout<64>::SMEM);
         if (e != cudaSuccess) return e;
-        k_sparse_attn<64><<<grid, NTHREADS, Layout<64>::SMEM, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, p);
+        k_sparse_attn<64><<<grid, NTHREADS, Layout<64>::SMEM, s>>>(maps, p);
         AC_NOTE_LAUNCH();
     }
     return cudaGetLastError();

@@ -537,4 +537,36 @@ cudaError_t launch_permute_rows(const bf16 *X, const int *perm, bf16 *Xp, int64_
     return cudaGetLastError();
 }
 
+// Kp[h, 8 pgoff[h, c] + i] = K[h, perm[h, offs[h, c] + i]] (and V alike): the
+// keys of cluster c in order, the cluster starting on an 8-row group.
+__global__ void k_permute_kv_padded(const bf16 *__restrict__ K, const bf16 *__restrict__ V,
+                                    const int *__restrict__ perm, const int *__restrict__ labels,
+                                    const int *__restrict__ offs, int offs_stride, const int *__restrict__ pgoff,
+                                    int Ccap, bf16 *__restrict__ Kp, bf16 *__restrict__ Vp, int64_t L, int64_t Lpad,
+                                    int d, int64_t total_rows) {
+    const int lanes_per_row = d / 8;
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = g / lanes_per_row;
+    const int part = (int)(g % lanes_per_row);
+    if (row >= total_rows) return;
+    const int64_t h = row / L, pos = row % L;
+    const int tok = perm[row];
+    const int c = labels[h * L + tok];
+    const int64_t dst = h * Lpad + 8ll * pgoff[h * Ccap + c] + (pos - offs[h * offs_stride + c]);
+    const int64_t src = h * L + tok;
+    reinterpret_cast<uint4 *>(Kp + dst * d)[part] = reinterpret_cast<const uint4 *>(K + src * d)[part];
+    reinterpret_cast<uint4 *>(Vp + dst * d)[part] = reinterpret_cast<const uint4 *>(V + src * d)[part];
+}
+
+cudaError_t launch_permute_kv_padded(const bf16 *K, const bf16 *V, const int *perm, const int *labels,
+                                     const int *offs, int offs_stride, const int *pgoff, int Ccap, bf16 *Kp,
+                                     bf16 *Vp, int64_t L, int64_t Lpad, int d, int BH, cudaStream_t s) {
+    const int64_t rows = (int64_t)BH * L;
+    const int64_t threads = rows * (d / 8);
+    k_permute_kv_padded<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(K, V, perm, labels, offs, offs_stride,
+                                                                          pgoff, Ccap, Kp, Vp, L, Lpad, d, rows);
+    AC_NOTE_LAUNCH();
+    return cudaGetLastError();
+}
+
 }  // namespace ac

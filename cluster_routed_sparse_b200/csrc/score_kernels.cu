@@ -179,34 +179,61 @@ __global__ void __launch_bounds__(SEL_THREADS) k_score_select(SelectArgs a) {
     int pos;
     Scan(tmp.scan).ExclusiveSum(mine, pos);
     __syncthreads();
-    // 8-row boxes of the kept clusters: exclusive prefix in selection order
-    int boxes = 0;
     for (int c = c0; c < c1; ++c)
-        if (flag[c]) boxes += (cnt[c] + 7) / 8;
-    int bpos, nb;
-    Scan(tmp.scan).ExclusiveSum(boxes, bpos, nb);
-    __syncthreads();
-    const int *offs = a.offs_k + (int64_t)h * (a.Ccap + 1);
-    int *rbox = a.rbox + (int64_t)hq * (a.Ccap + 1);
+        if (flag[c]) a.sel[(int64_t)hq * a.Ccap + pos++] = c;
+    // The key ranges the attention walks: the kept clusters, or every
+    // non-empty cluster of a dense unit (Algorithm 3 line 6), in cluster
+    // order, each as (first 8-row group in Kp / Vp, keys); rbox is the
+    // exclusive prefix of their 8-row groups.
+    const bool dense = a.dense[h] != 0;
+    int walk = 0, groups = 0;
     for (int c = c0; c < c1; ++c) {
-        if (!flag[c]) continue;
-        a.sel[(int64_t)hq * a.Ccap + pos] = c;
-        a.ranges[(int64_t)hq * a.Ccap + pos] = make_int2(offs[c], cnt[c]);
-        rbox[pos] = bpos;
-        bpos += (cnt[c] + 7) / 8;
-        ++pos;
+        const int w = dense ? cnt[c] != 0 : flag[c];
+        walk += w;
+        groups += w ? (cnt[c] + 7) / 8 : 0;
     }
     __syncthreads();
+    int rpos, nr;
+    Scan(tmp.scan).ExclusiveSum(walk, rpos, nr);
+    __syncthreads();
+    int gpos, ng;
+    Scan(tmp.scan).ExclusiveSum(groups, gpos, ng);
+    __syncthreads();
+    const int *pg = a.pgoff + (int64_t)h * a.Ccap;
+    int *rbox = a.rbox + (int64_t)hq * (a.Ccap + 1);
+    for (int c = c0; c < c1; ++c) {
+        const int w = dense ? cnt[c] != 0 : flag[c];
+        if (!w) continue;
+        a.ranges[(int64_t)hq * a.Ccap + rpos] = make_int2(pg[c], cnt[c]);
+        rbox[rpos] = gpos;
+        gpos += (cnt[c] + 7) / 8;
+        ++rpos;
+    }
     if (tid == 0) {
-        if (a.dense[h]) {  // Algorithm 3 line 6: every key of the unit
-            a.ranges[(int64_t)hq * a.Ccap] = make_int2(0, a.L);
-            a.nboxes[hq] = (a.L + 7) / 8;
-            rbox[0] = 0;
-            rbox[1] = (a.L + 7) / 8;
-        } else {
-            a.nboxes[hq] = nb;
-            rbox[k] = nb;
-        }
+        a.nrange[hq] = nr;
+        a.nboxes[hq] = ng;
+        rbox[nr] = ng;
+    }
+}
+
+// First 8-row group of every key cluster of a unit in Kp / Vp: exclusive
+// prefix of ceil(count / 8) in cluster order.  One block per unit.
+__global__ void __launch_bounds__(SEL_THREADS) k_group_offsets(const int *counts_k, const int *n_k, int Ccap,
+                                                             int *pgoff) {
+    typedef cub::BlockScan<int, SEL_THREADS> Scan;
+    __shared__ typename Scan::TempStorage tmp;
+    const int h = blockIdx.x, tid = threadIdx.x;
+    const int nk = n_k[h];
+    const int *cnt = counts_k + (int64_t)h * Ccap;
+    const int seg = (nk + SEL_THREADS - 1) / SEL_THREADS;
+    const int c0 = min(nk, tid * seg), c1 = min(nk, c0 + seg);
+    int g = 0;
+    for (int c = c0; c < c1; ++c) g += (cnt[c] + 7) / 8;
+    int pos;
+    Scan(tmp).ExclusiveSum(g, pos);
+    for (int c = c0; c < c1; ++c) {
+        pgoff[(int64_t)h * Ccap + c] = pos;
+        pos += (cnt[c] + 7) / 8;
     }
 }
 
@@ -245,6 +272,9 @@ cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s) {
     e = cudaFuncSetAttribute(k_score_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(smem < 48 * 1024 ? 48 * 1024 : smem));
     if (e != cudaSuccess) return e;
+    k_group_offsets<<<a.BH, SEL_THREADS, 0, s>>>(a.counts_k, a.n_k, a.Ccap, a.pgoff);
+    AC_NOTE_LAUNCH();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_score_select<<<a.BH * a.Cq, SEL_THREADS, smem, s>>>(a);
     AC_NOTE_LAUNCH();
     e = cudaGetLastError();
