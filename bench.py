@@ -195,6 +195,22 @@ def workload_config():
 
 
 # ---------------------------------------------------------------- main
+# DRAM bytes (read + write) of one k_sparse_attn launch per head, from the ncu capture summarised
+# in profiles/k_sparse_attn_wan14b_h8.md (8 heads, scaled by heads), valid only for the kernel
+# source it was taken on: any change to attn_kernel.cu turns the figure into null.
+ATTN_TRAFFIC = {"sha256_prefix": "e2bc600c81be3bda", "bytes_per_head": (313.696512e6 + 133.403648e6) / 8}
+
+
+def attn_traffic_bytes(heads):
+    import hashlib
+    src = os.path.join(ROOT, "cluster_routed_sparse_b200", "csrc", "attn_kernel.cu")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    if not digest.startswith(ATTN_TRAFFIC["sha256_prefix"]):
+        return None
+    return round(ATTN_TRAFFIC["bytes_per_head"] * heads)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -301,9 +317,10 @@ def main():
     peak_src = "of measured (bf16_tflops_sustained)" if peak_tf else "of fallback"
     peak_tf = peak_tf or 1400.0
     attn_flops = 4.0 * cfg.d * cnt["kept_pairs"]  # last call (a warm step)
+    traffic = attn_traffic_bytes(cfg.H)
     achieved = attn_flops / (splitw["attn_kernel_ms"] * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": round(achieved / peak_tf, 4), "traffic": None, "peak_source": peak_src,
+                "frac": round(achieved / peak_tf, 4), "traffic": traffic, "peak_source": peak_src,
                 "kernel": "k_sparse_attn (warm-step launch)",
                 "algorithmic_flops_per_launch": attn_flops,
                 "computed_tile_flops_per_launch": 4.0 * cfg.d * cnt["computed_pairs"]}
