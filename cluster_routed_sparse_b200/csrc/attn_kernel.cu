@@ -57,7 +57,7 @@ struct Layout {
     static constexpr uint32_t OFF_Q = 0;                        // two query tiles
     static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_TILE;
     static constexpr uint32_t OFF_V = OFF_K + NS * KV_BYTES;
-    static constexpr uint32_t OFF_MASK = OFF_V + NS * KV_BYTES;  // [NS][4] uint32
+    static constexpr uint32_t OFF_MASK = OFF_V + NS * KV_BYTES;  // [4][4] uint32 (tile j in slot j % 4)
     static constexpr uint32_t OFF_RG = OFF_MASK + 64;            // [RG_CACHE] int2 key ranges
     static constexpr uint32_t OFF_RB = OFF_RG + RG_CACHE * 8;    // [RG_CACHE + 1] first box of each range
     static constexpr uint32_t OFF_BAR = OFF_RB + (RG_CACHE + 1) * 4 + 12;
@@ -66,14 +66,16 @@ struct Layout {
 };
 
 enum {
-    B_KVF = 0,   // [NS] K/V stage filled (TMA tx) -- also publishes the masks
-    B_KVE = 2,   // [NS] K/V stage free (MMA commit after both PV products)
-    B_QF = 4,    // query tiles filled
-    B_SF = 5,    // [2] S_i written (MMA commit)
-    B_PF = 7,    // [2] P_i written (+ O_i rescaled) by the 128 softmax threads
-    B_OF = 9,    // [2] last PV_i complete (MMA commit)
-    B_DONE = 11, // every MMA complete
-    NBAR = 12
+    B_KF = 0,    // [NS] K stage filled (TMA tx) -- also publishes the tile's masks
+    B_KE = 2,    // [NS] K stage free (MMA commit after both S products)
+    B_VF = 4,    // [NS] V stage filled
+    B_VE = 6,    // [NS] V stage free (MMA commit after both PV products)
+    B_QF = 8,    // query tiles filled
+    B_SF = 9,    // [2] S_i written (MMA commit)
+    B_PF = 11,   // [2] P_i written (+ O_i rescaled) by the 128 softmax threads
+    B_OF = 13,   // [2] last PV_i complete (MMA commit)
+    B_DONE = 15, // every MMA complete
+    NBAR = 16
 };
 
 // 2^x on the FMA pipe, so that part of the exponentials bypass the
@@ -83,13 +85,22 @@ enum {
 // x + 1.5 * 2^23; 2^f by a cubic fitted here for least maximum relative error
 // on [-1/2, 1/2] (1.02e-4, below the 2^-9 rounding of the bf16 P it feeds);
 // 2^n added to the exponent field.  x is clamped at -126, so -inf (a masked
-// column) gives at most 2^-126 instead of 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -126.f);
-    const float t = x + 12582912.f;
-    const float f = x - (t - 12582912.f);
-    const float q = fmaf(fmaf(fmaf(0.05500858277f, f, 0.24221037328f), f, 0.69328290224f), f, 1.0f);
-    return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+// column) gives at most 2^-126 instead of 0.  Two elements per call, in
+// packed fp32 pairs.
+constexpr float kExp2C3 = 0.05500858277f, kExp2C2 = 0.24221037328f, kExp2C1 = 0.69328290224f;
+constexpr float kRoundMagic = 12582912.f;  // 1.5 * 2^23
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &p0, float &p1) {
+    const uint64_t x = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t t = f2_add(x, f2_pack(kRoundMagic, kRoundMagic));
+    const uint64_t f = f2_sub(x, f2_sub(t, f2_pack(kRoundMagic, kRoundMagic)));
+    uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+    q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
+    q = f2_fma(q, f, f2_pack(1.f, 1.f));
+    float q0, q1, t0, t1;
+    f2_unpack(q, q0, q1);
+    f2_unpack(t, t0, t1);
+    p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+    p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 struct AttnMaps {
@@ -162,8 +173,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) {
-            mbar_init(BAR(B_KVF + i), 1);
-            mbar_init(BAR(B_KVE + i), 1);
+            mbar_init(BAR(B_KF + i), 1);
+            mbar_init(BAR(B_KE + i), 1);
+            mbar_init(BAR(B_VF + i), 1);
+            mbar_init(BAR(B_VE + i), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(BAR(B_SF + i), 1);
@@ -224,50 +237,77 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int a0 = mine ? max(rb0, t0) : 0, a1 = mine ? min(rb1, t1) : 0;
             int2 g = make_int2(0, 0);
             if (mine) g = rgp[r];
-            uint32_t w[4] = {0u, 0u, 0u, 0u};
-            for (int sl = a0; sl < a1; ++sl) {
-                const int v = min(8, g.y - 8 * (sl - rb0));
-                const uint32_t byte = v >= 8 ? 0xFFu : ((1u << v) - 1u);
-                const int ls = sl - t0;
-                w[ls >> 2] |= byte << ((ls & 3) * 8);
-            }
+            // column masks of the 16 groups (8 bits each, 4 per word) from the
+            // groups of this lane's part; the last group of a range may be partial
+            uint32_t w[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) w[q] = __reduce_or_sync(0xFFFFFFFFu, w[q]);
+            for (int q = 0; q < 4; ++q) {
+                uint32_t word = 0u;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int sl = t0 + 4 * q + b;
+                    const int v = min(8, g.y - 8 * (sl - rb0));
+                    const uint32_t byte = v >= 8 ? 0xFFu : ((1u << max(v, 0)) - 1u);
+                    word |= (sl >= a0 && sl < a1) ? byte << (8 * b) : 0u;
+                }
+                w[q] = __reduce_or_sync(0xFFFFFFFFu, word);
+            }
             const int rnext = r0 + __popc(__ballot_sync(0xFFFFFFFFu, mine && rb1 <= t1));
-            if (j >= NS && !__all_sync(0xFFFFFFFFu, WAIT(1, B_KVE + s, j, ((j / NS) - 1) & 1))) {
+            const int filled = min(max(nbox - t0, 0), BOXES);
+            const int gfirst = unit_group + g.x + (a0 - rb0);
+            // K: its stage frees once both S products of tile j - NS are done;
+            // the masks go to slot j % 4 (the softmax of tile j - 4 is over by then)
+            if (j >= NS && !__all_sync(0xFFFFFFFFu, WAIT(1, B_KE + s, j, ((j / NS) - 1) & 1))) {
                 ok = false;
                 break;
             }
-            if (lane < 4) masks[4 * s + lane] = lane == 0 ? w[0] : lane == 1 ? w[1] : lane == 2 ? w[2] : w[3];
+            if (lane < 4) masks[4 * (j & 3) + lane] = lane == 0 ? w[0] : lane == 1 ? w[1] : lane == 2 ? w[2] : w[3];
             __syncwarp();
-            if (lane == 0) mbar_arrive_expect_tx(BAR(B_KVF + s), 2 * LY::KV_BYTES);  // releases the masks
+            if (lane == 0) mbar_arrive_expect_tx(BAR(B_KF + s), LY::KV_BYTES);  // releases the masks
             __syncwarp();
             const uint32_t kd = sbase + LY::OFF_K + s * LY::KV_BYTES;
-            const uint32_t vd = sbase + LY::OFF_V + s * LY::KV_BYTES;
             if (mine) {
-                int ls = a0 - t0, gi = unit_group + g.x + (a0 - rb0), left = a1 - a0;
+                int ls = a0 - t0, gi = gfirst, left = a1 - a0;
                 while (left > 0) {
                     const int lg = left >= 8 ? 3 : left >= 4 ? 2 : left >= 2 ? 1 : 0;
-                    tma_load_4d(kd + ls * LY::BOX_BYTES, &maps.k[lg], 0, 0, 0, gi, BAR(B_KVF + s));
-                    tma_load_4d(vd + ls * LY::BOX_BYTES, &maps.v[lg], 0, 0, 0, gi, BAR(B_KVF + s));
+                    tma_load_4d(kd + ls * LY::BOX_BYTES, &maps.k[lg], 0, 0, 0, gi, BAR(B_KF + s));
                     ls += 1 << lg;
                     gi += 1 << lg;
                     left -= 1 << lg;
                 }
             }
-            const int filled = min(max(nbox - t0, 0), BOXES);
-            if (lane >= BOXES && lane - BOXES < BOXES - filled) {
-                const int ls = filled + lane - BOXES;
-                tma_load_4d(kd + ls * LY::BOX_BYTES, &maps.k[0], 0, 0, 0, zero_group, BAR(B_KVF + s));
-                tma_load_4d(vd + ls * LY::BOX_BYTES, &maps.v[0], 0, 0, 0, zero_group, BAR(B_KVF + s));
+            if (lane >= BOXES && lane - BOXES < BOXES - filled)
+                tma_load_4d(kd + (filled + lane - BOXES) * LY::BOX_BYTES, &maps.k[0], 0, 0, 0, zero_group,
+                            BAR(B_KF + s));
+            // V: its stage frees once both PV products of tile j - NS are done
+            if (j >= NS && !__all_sync(0xFFFFFFFFu, WAIT(1, B_VE + s, j, ((j / NS) - 1) & 1))) {
+                ok = false;
+                break;
             }
+            if (lane == 0) mbar_arrive_expect_tx(BAR(B_VF + s), LY::KV_BYTES);
+            __syncwarp();
+            const uint32_t vd = sbase + LY::OFF_V + s * LY::KV_BYTES;
+            if (mine) {
+                int ls = a0 - t0, gi = gfirst, left = a1 - a0;
+                while (left > 0) {
+                    const int lg = left >= 8 ? 3 : left >= 4 ? 2 : left >= 2 ? 1 : 0;
+                    tma_load_4d(vd + ls * LY::BOX_BYTES, &maps.v[lg], 0, 0, 0, gi, BAR(B_VF + s));
+                    ls += 1 << lg;
+                    gi += 1 << lg;
+                    left -= 1 << lg;
+                }
+            }
+            if (lane >= BOXES && lane - BOXES < BOXES - filled)
+                tma_load_4d(vd + (filled + lane - BOXES) * LY::BOX_BYTES, &maps.v[0], 0, 0, 0, zero_group,
+                            BAR(B_VF + s));
             r0 = rnext;
             ++issued;
         }
         if (lane == 0) {
             // Loads still in flight must land before the CTA exits.
             for (int j = issued - NS < 0 ? 0 : issued - NS; j < issued; ++j)
-                if (!WAIT(2, B_KVF + (j % NS), j, (j / NS) & 1)) ok = false;
+                if (!WAIT(2, B_KF + (j % NS), j, (j / NS) & 1) || !WAIT(2, B_VF + (j % NS), j, (j / NS) & 1))
+                    ok = false;
             if (!WAIT(2, B_QF, 0, 0)) ok = false;
             if (!ok) set_err(p.err, DEV_ERR_TIMEOUT);
         }
@@ -299,16 +339,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             };
             if (!WAIT(3, B_QF, 0, 0)) ok = false;
             if (ok && n_tiles > 0) {
-                if (!WAIT(3, B_KVF, 0, 0)) ok = false;
+                if (!WAIT(3, B_KF, 0, 0)) ok = false;
                 tc_fence_after();
                 if (ok) {
                     issue_s(0, 0);
                     if (has1) issue_s(1, 0);
+                    tc_commit(BAR(B_KE + 0));
                 }
             }
             for (int j = 0; j < n_tiles && ok; ++j) {
                 const bool more = j + 1 < n_tiles;
-                if (!WAIT(3, B_PF + 0, j, j & 1)) {
+                if (!WAIT(3, B_PF + 0, j, j & 1) || !WAIT(3, B_VF + (j % NS), j, (j / NS) & 1)) {
                     ok = false;
                     break;
                 }
@@ -316,7 +357,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 issue_pv(0, j);
                 if (!more) tc_commit(BAR(B_OF + 0));
                 if (more) {
-                    if (!WAIT(3, B_KVF + ((j + 1) % NS), j + 1, ((j + 1) / NS) & 1)) {
+                    if (!WAIT(3, B_KF + ((j + 1) % NS), j + 1, ((j + 1) / NS) & 1)) {
                         ok = false;
                         break;
                     }
@@ -333,7 +374,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!more) tc_commit(BAR(B_OF + 1));
                     if (more) issue_s(1, j + 1);
                 }
-                tc_commit(BAR(B_KVE + (j % NS)));
+                if (more) tc_commit(BAR(B_KE + ((j + 1) % NS)));  // K(j+1): both S products issued
+                tc_commit(BAR(B_VE + (j % NS)));                  // V(j): both PV products issued
             }
             tc_commit(BAR(B_DONE));
             if (!WAIT(4, B_DONE, 0, 0)) ok = false;
@@ -358,11 +400,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int s = j % NS;
                 // Wait outcomes are combined across the warp: the TMEM loads and
                 // stores below are warp-collective, so a warp leaves together.
-                if (!__all_sync(0xFFFFFFFFu, WAIT(5 + wg, B_KVF + s, j, (j / NS) & 1))) {
+                if (!__all_sync(0xFFFFFFFFu, WAIT(5 + wg, B_KF + s, j, (j / NS) & 1))) {
                     ok = false;
                     break;
                 }
-                const uint4 mk = *reinterpret_cast<const uint4 *>(masks + 4 * s);
+                const uint4 mk = *reinterpret_cast<const uint4 *>(masks + 4 * (j & 3));
                 const uint32_t vm[4] = {mk.x, mk.y, mk.z, mk.w};
                 kept_cols += __popc(vm[0]) + __popc(vm[1]) + __popc(vm[2]) + __popc(vm[3]);
                 if (!__all_sync(0xFFFFFFFFu, WAIT(5 + wg, B_SF + wg, j, j & 1))) {
@@ -383,16 +425,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         for (int i = 0; i < 32; ++i) r[c][i] = ((vm[c] >> i) & 1u) ? r[c][i] : 0xFF800000u;
                     }
                 }
-                // Row maximum with 8 independent partial maxima.
+                // Row maximum: 8 independent partial maxima, three-input max.
                 float pm[8];
 #pragma unroll
                 for (int a = 0; a < 8; ++a) pm[a] = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) pm[i & 7] = fmaxf(pm[i & 7], __uint_as_float(r[c][i]));
-                const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                         fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+                    for (int i = 0; i < 32; i += 2)
+                        pm[(i >> 1) & 7] = fmax3(pm[(i >> 1) & 7], __uint_as_float(r[c][i]),
+                                                 __uint_as_float(r[c][i + 1]));
+                const float tmax = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
                 const float m_new = fmaxf(m_run, tmax * sl2);
                 // The rescale touches TMEM with warp-collective (.sync.aligned)
                 // loads and stores, so the decision must be uniform across the
@@ -417,12 +460,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     m_run = m_new;
                 }
-                // p = 2^(s * scale * log2(e) - m): one FMA and one ex2 per element;
-                // -inf columns give 0.  Row sum with 8 independent partial sums.
-                const float neg_m = -m_run;
-                float ps[8];
+                // p = 2^(s * scale * log2(e) - m): one FMA and one ex2 per element,
+                // in packed pairs; -inf columns give 0.  Row sum with 8
+                // independent partial sums (4 packed pairs).
+                const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_run, -m_run);
+                uint64_t ps2[4];
 #pragma unroll
-                for (int a = 0; a < 8; ++a) ps[a] = 0.f;
+                for (int a = 0; a < 4; ++a) ps2[a] = f2_pack(0.f, 0.f);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[32];
@@ -431,17 +475,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const int c = half * 2 + cc;
 #pragma unroll
                         for (int i = 0; i < 32; i += 2) {
-                            const float x0 = fmaf(__uint_as_float(r[c][i]), sl2, neg_m);
-                            const float x1 = fmaf(__uint_as_float(r[c][i + 1]), sl2, neg_m);
-                            const float p0 = c == kPolyChunk ? exp2_poly(x0) : ex2_approx(x0);
-                            const float p1 = c == kPolyChunk ? exp2_poly(x1) : ex2_approx(x1);
-                            ps[i & 7] += p0;
-                            ps[(i + 1) & 7] += p1;
+                            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])),
+                                                       sl2x2, negm2);
+                            float x0, x1, p0, p1;
+                            f2_unpack(x2, x0, x1);
+                            if (c == kPolyChunk) {
+                                exp2_poly2(x0, x1, p0, p1);
+                            } else {
+                                p0 = ex2_approx(x0);
+                                p1 = ex2_approx(x1);
+                            }
+                            ps2[(i >> 1) & 3] = f2_add(ps2[(i >> 1) & 3], f2_pack(p0, p1));
                             pk[cc * 16 + (i >> 1)] = pack_bf16x2(p0, p1);
                         }
                     }
                     tmem_st32(tS + half * 32, pk);  // P columns [32*half, 32*half+32)
                 }
+                float ps[8];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) f2_unpack(ps2[a], ps[2 * a], ps[2 * a + 1]);
                 const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 tmem_st_wait();
                 l_run += rs;
