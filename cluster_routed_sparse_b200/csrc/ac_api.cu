@@ -218,7 +218,7 @@ ac_status cluster_q_impl(ac_ctx *c, const bf16 *Q, const float *init, int iters,
     k.as = AssignArgs{Q, c->inv_q, L, nullptr, nullptr, c->L, c->cent_q, (int64_t)c->Cq * c->d, nullptr,
                       nullptr, c->Cq, c->labels_q, nullptr, c->BH, c->d};
     k.so = SortArgs{c->labels_q, L, nullptr, c->L, nullptr, c->Cq, c->Cq, c->perm_q, c->offs_q, c->Cq + 1,
-                    c->counts_q, c->Cq, c->BH};
+                    c->counts_q, c->Cq, c->BH, c->sort_scratch};
     k.up = UpdateArgs{Q, c->inv_q, L, nullptr, c->perm_q, c->offs_q, c->Cq + 1, c->cent_q,
                       (int64_t)c->Cq * c->d, nullptr, nullptr, c->Cq, c->BH, c->d, c->Cq};
     make_fast(c, k, Q, true, c->cent_q, (int64_t)c->Cq * c->d, nullptr, c->Cq, c->labels_q, nullptr);
@@ -283,7 +283,7 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
         k.as = AssignArgs{K, nullptr, L, c->u_idx, c->u_cnt, 0, c->cent_k, cstride, c->n_k, c->st_m, 0,
                           c->st_labels, c->dmin_k, BH, d};
         k.so = SortArgs{c->st_labels, L, c->u_cnt, 0, c->st_m, 0, max_m, c->st_perm, c->st_offs, m0 + 1, nullptr,
-                        0, BH};
+                        0, BH, c->sort_scratch};
         k.up = UpdateArgs{K, nullptr, L, c->u_idx, c->st_perm, c->st_offs, m0 + 1, c->cent_k, cstride, c->n_k,
                           c->st_m, 0, BH, d, max_m};
         // stage 0: U is every key in order and the stage's centres start at 0
@@ -345,7 +345,7 @@ ac_status cluster_k_warm(ac_ctx *c, const bf16 *K, cudaStream_t s) {
     k.as = AssignArgs{K, nullptr, L, nullptr, nullptr, L, c->cent_k, cstride, nullptr, c->st_m, 0, c->labels_k,
                       c->dmin_k, BH, d};
     k.so = SortArgs{c->labels_k, L, nullptr, L, c->n_k, 0, c->Ccap, c->perm_k, c->offs_k, c->Ccap + 1, c->counts_k,
-                    c->Ccap, BH};
+                    c->Ccap, BH, c->sort_scratch};
     k.up = UpdateArgs{K, nullptr, L, nullptr, c->perm_k, c->offs_k, c->Ccap + 1, c->cent_k, cstride, nullptr,
                       c->st_m, 0, BH, d, c->Ccap};
     make_fast(c, k, K, false, c->cent_k, cstride, c->st_m, 0, c->labels_k, c->dmin_k);
@@ -356,7 +356,7 @@ ac_status cluster_k_warm(ac_ctx *c, const bf16 *K, cudaStream_t s) {
 // Cluster-order permutation of the keys and the per-cluster statistics.
 ac_status key_stats_impl(ac_ctx *c, const bf16 *K, cudaStream_t s) {
     SortArgs so{c->labels_k, c->L, nullptr, c->L, c->n_k, 0, c->Ccap, c->perm_k, c->offs_k, c->Ccap + 1,
-                c->counts_k, c->Ccap, c->BH};
+                c->counts_k, c->Ccap, c->BH, c->sort_scratch};
     CK(launch_counting_sort(so, s), "k sort");
     StatsArgs st{K, c->L, c->perm_k, c->offs_k, c->Ccap + 1, c->dmin_k, c->n_k, c->Ccap, c->d, c->BH,
                  c->counts_k, c->kmax, c->kmin, c->sse, c->mse, c->comp};
@@ -395,7 +395,8 @@ void free_all(ac_ctx *c) {
                    c->u_cnt, c->st_m, c->st_labels, c->st_dist, c->st_perm, c->st_offs, c->st_counts, c->radix,
                    c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->Qp, c->Kp, c->Vp,
                    c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err, c->chi_q, c->chi_k, c->cn,
-                   c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats, c->rbox, c->pgoff, c->nrange};
+                   c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats, c->rbox, c->pgoff, c->nrange,
+                   c->sort_scratch};
     for (void *p : dev)
         if (p) cudaFree(p);
     void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err};
@@ -499,6 +500,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->st_offs, BH * (m0 + 1)));
     A(dalloc(&c->st_counts, BH * m0));
     A(dalloc(&c->radix, 260));
+    A(dalloc(&c->sort_scratch, BH * 128 * std::max(Cc, Cq)));
     A(dalloc(&c->score, BH * Cq * Cc));
     A(dalloc(&c->sel, BH * Cq * Cc));
     A(dalloc(&c->ksel, BH));

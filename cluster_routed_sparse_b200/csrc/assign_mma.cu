@@ -435,23 +435,33 @@ __global__ void __launch_bounds__(A_THREADS, 1)
 }
 
 // Exact fp32 squared distance, dimensions in order (the definition's arithmetic).
+// The row and the centre are read 32 dimensions at a time, all loads of a block
+// issued before its arithmetic, so the load latency is paid d / 32 times.
 template <bool NORM>
 __device__ __forceinline__ float exact_sqdist(const bf16 *__restrict__ xr, float s, const float *__restrict__ c,
                                               int d) {
     float acc = 0.f;
     const uint4 *x8 = reinterpret_cast<const uint4 *>(xr);
     const float4 *c4 = reinterpret_cast<const float4 *>(c);
-    for (int k8 = 0; k8 < d / 8; ++k8) {
-        const uint4 xv = x8[k8];
-        const float4 ca = c4[2 * k8], cb = c4[2 * k8 + 1];
-        const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
-        const float cc[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+    for (int b = 0; b < d / 32; ++b) {
+        uint4 xv[4];
+        float4 cv[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float x = __uint_as_float((j & 1) ? (w[j >> 1] & 0xFFFF0000u) : (w[j >> 1] << 16));
-            if (NORM) x = __fmul_rn(x, s);
-            const float t = __fsub_rn(x, cc[j]);
-            acc = __fadd_rn(acc, __fmul_rn(t, t));
+        for (int q = 0; q < 4; ++q) xv[q] = x8[4 * b + q];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) cv[q] = c4[8 * b + q];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t w[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
+            const float cc[8] = {cv[2 * q].x, cv[2 * q].y, cv[2 * q].z, cv[2 * q].w,
+                                 cv[2 * q + 1].x, cv[2 * q + 1].y, cv[2 * q + 1].z, cv[2 * q + 1].w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float x = __uint_as_float((j & 1) ? (w[j >> 1] & 0xFFFF0000u) : (w[j >> 1] << 16));
+                if (NORM) x = __fmul_rn(x, s);
+                const float t = __fsub_rn(x, cc[j]);
+                acc = __fadd_rn(acc, __fmul_rn(t, t));
+            }
         }
     }
     return acc;

@@ -138,7 +138,119 @@ cudaError_t launch_assign_exact(const AssignArgs &a, cudaStream_t s) {
 // per-warp histograms give each warp its first slot per label, then every
 // warp scatters its chunk in order (warp-level match gives in-order ranks).
 constexpr int SORT_WARPS = 8;
+constexpr int SORT_SEGS = 16;                        // blocks per unit
+constexpr int SORT_CHUNKS = SORT_SEGS * SORT_WARPS;  // contiguous row chunks per unit, one per warp
 
+// Stable counting sort of the labels of every unit in three passes over
+// SORT_CHUNKS contiguous row chunks (one warp each, SORT_SEGS blocks per unit):
+// (1) per-chunk label histograms; (2) per unit, exclusive offsets of the labels
+// and the first slot of every (label, chunk) in chunk order; (3) each chunk
+// scatters its rows in order (warp-match ranks within 32 rows).  The result is
+// the same as one sequential stable pass over the rows.
+__global__ void __launch_bounds__(SORT_WARPS * 32) k_sort_hist(SortArgs a) {
+    extern __shared__ int hist[];  // [SORT_WARPS][max_lab]
+    const int seg = blockIdx.x, h = blockIdx.y;
+    const int n = a.nrows ? a.nrows[h] : a.nrows_const;
+    const int m = a.nlab ? a.nlab[h] : a.nlab_const;
+    if (m <= 0) return;  // idle unit
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int *lab = a.labels + (int64_t)h * a.L;
+    for (int i = tid; i < SORT_WARPS * m; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int ci = seg * SORT_WARPS + w;
+    const int chunk = (n + SORT_CHUNKS - 1) / SORT_CHUNKS;
+    const int beg = min(n, ci * chunk), end = min(n, beg + chunk);
+    for (int i = beg + lane; i < end; i += 32) {
+        const int l = lab[i];
+        if ((unsigned)l < (unsigned)m) atomicAdd(&hist[w * m + l], 1);
+    }
+    __syncwarp();
+    int *H = a.scratch + ((int64_t)h * SORT_CHUNKS + ci) * a.max_lab;
+    for (int l = lane; l < m; l += 32) H[l] = hist[w * m + l];
+}
+
+__global__ void __launch_bounds__(256) k_sort_offsets(SortArgs a) {
+    extern __shared__ int tot[];  // [max_lab]
+    typedef cub::BlockScan<int, 256> Scan;
+    __shared__ typename Scan::TempStorage scan_tmp;
+    const int h = blockIdx.x, tid = threadIdx.x;
+    const int n = a.nrows ? a.nrows[h] : a.nrows_const;
+    const int m = a.nlab ? a.nlab[h] : a.nlab_const;
+    if (m <= 0) return;
+    int *H = a.scratch + (int64_t)h * SORT_CHUNKS * a.max_lab;
+    for (int l = tid; l < m; l += 256) {
+        int t = 0;
+        for (int ci = 0; ci < SORT_CHUNKS; ++ci) t += H[(int64_t)ci * a.max_lab + l];
+        tot[l] = t;
+    }
+    __syncthreads();
+    const int sg = (m + 255) / 256;
+    const int l0 = min(m, tid * sg), l1 = min(m, l0 + sg);
+    int local = 0;
+    for (int l = l0; l < l1; ++l) local += tot[l];
+    int run;
+    Scan(scan_tmp).ExclusiveSum(local, run);
+    __syncthreads();
+    for (int l = l0; l < l1; ++l) {
+        const int t = tot[l];
+        tot[l] = run;  // now the label's first slot
+        run += t;
+    }
+    __syncthreads();
+    int *offs = a.offs + (int64_t)h * a.offs_stride;
+    for (int l = tid; l < m; l += 256) {
+        int slot = tot[l];
+        offs[l] = slot;
+        const int first = slot;
+        for (int ci = 0; ci < SORT_CHUNKS; ++ci) {
+            const int c = H[(int64_t)ci * a.max_lab + l];
+            H[(int64_t)ci * a.max_lab + l] = slot;  // first slot of chunk ci for label l
+            slot += c;
+        }
+        if (a.counts) a.counts[(int64_t)h * a.counts_stride + l] = slot - first;
+    }
+    if (tid == 0) offs[m] = n;
+}
+
+__global__ void __launch_bounds__(SORT_WARPS * 32) k_sort_scatter(SortArgs a) {
+    extern __shared__ int hist[];  // [SORT_WARPS][max_lab]
+    const int seg = blockIdx.x, h = blockIdx.y;
+    const int n = a.nrows ? a.nrows[h] : a.nrows_const;
+    const int m = a.nlab ? a.nlab[h] : a.nlab_const;
+    if (m <= 0) return;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int ci = seg * SORT_WARPS + w;
+    const int chunk = (n + SORT_CHUNKS - 1) / SORT_CHUNKS;
+    const int beg = min(n, ci * chunk), end = min(n, beg + chunk);
+    if (beg >= end) return;  // no barrier below: warps leave independently
+    const int *H = a.scratch + ((int64_t)h * SORT_CHUNKS + ci) * a.max_lab;
+    int *hs = hist + w * m;
+    for (int l = lane; l < m; l += 32) hs[l] = H[l];
+    __syncwarp();
+    const int *lab = a.labels + (int64_t)h * a.L;
+    int *perm = a.perm + (int64_t)h * a.L;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = beg; base < end; base += 32) {
+        const int i = base + lane;
+        const bool v = i < end;
+        int l = v ? lab[i] : -1 - lane;
+        if (v && (unsigned)l >= (unsigned)m) l = -1 - lane;  // out of range: never placed
+        const unsigned grp = __match_any_sync(0xFFFFFFFFu, l);
+        const int rank = __popc(grp & lt);
+        int slot = 0;
+        if (l >= 0) slot = hs[l];
+        __syncwarp();
+        if (l >= 0) {
+            perm[slot + rank] = i;
+            if (rank == 0) hs[l] = slot + __popc(grp);
+        }
+        __syncwarp();
+    }
+}
+
+// One block per unit (no scratch memory): per-warp histograms over contiguous
+// chunks, offsets, then an in-order scatter.  Used when the caller provides
+// no histogram scratch (the allocation-free entry point).
 __global__ void __launch_bounds__(SORT_WARPS * 32) k_counting_sort(SortArgs a) {
     extern __shared__ int hist[];  // [SORT_WARPS][max_lab]
     typedef cub::BlockScan<int, SORT_WARPS * 32> Scan;
@@ -158,7 +270,6 @@ __global__ void __launch_bounds__(SORT_WARPS * 32) k_counting_sort(SortArgs a) {
         if ((unsigned)l < (unsigned)m) atomicAdd(&hist[w * m + l], 1);
     }
     __syncthreads();
-    // totals per label -> exclusive offsets (labels split into contiguous segments)
     const int seg = (m + blockDim.x - 1) / blockDim.x;
     const int l0 = min(m, tid * seg), l1 = min(m, l0 + seg);
     int local = 0;
@@ -202,11 +313,30 @@ __global__ void __launch_bounds__(SORT_WARPS * 32) k_counting_sort(SortArgs a) {
 }
 
 cudaError_t launch_counting_sort(const SortArgs &a, cudaStream_t s) {
-    size_t smem = (size_t)SORT_WARPS * a.max_lab * sizeof(int);
-    cudaError_t e = cudaFuncSetAttribute(k_counting_sort, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(smem < 48 * 1024 ? 48 * 1024 : smem));
-    if (e != cudaSuccess) return e;
-    k_counting_sort<<<a.BH, SORT_WARPS * 32, smem, s>>>(a);
+    const size_t smem = (size_t)SORT_WARPS * a.max_lab * sizeof(int);
+    cudaError_t e;
+    if (!a.scratch) {
+        if ((e = cudaFuncSetAttribute(k_counting_sort, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)(smem < 48 * 1024 ? 48 * 1024 : smem))) != cudaSuccess)
+            return e;
+        k_counting_sort<<<a.BH, SORT_WARPS * 32, smem, s>>>(a);
+        AC_NOTE_LAUNCH();
+        return cudaGetLastError();
+    }
+    if ((e = cudaFuncSetAttribute(k_sort_hist, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)(smem < 48 * 1024 ? 48 * 1024 : smem))) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_sort_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)(smem < 48 * 1024 ? 48 * 1024 : smem))) != cudaSuccess)
+        return e;
+    const dim3 grid(SORT_SEGS, a.BH);
+    k_sort_hist<<<grid, SORT_WARPS * 32, smem, s>>>(a);
+    AC_NOTE_LAUNCH();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_sort_offsets<<<a.BH, 256, (size_t)a.max_lab * sizeof(int), s>>>(a);
+    AC_NOTE_LAUNCH();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_sort_scatter<<<grid, SORT_WARPS * 32, smem, s>>>(a);
     AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
@@ -227,15 +357,18 @@ __global__ void k_update(UpdateArgs a) {
     const bf16 *X = a.X + (int64_t)h * a.L * a.d;
     const float *inv = NORM ? a.inv + (int64_t)h * a.L : nullptr;
     float s = 0.f;
-    constexpr int U = 8;
+    // 32 members in flight per step (their rows are scattered over the unit:
+    // the sum is latency bound); the additions stay in ascending order
+    constexpr int U = 32;
     int j = beg;
     for (; j + U <= end; j += U) {
         int tok[U];
         float v[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            int p = perm[j + u];
-            tok[u] = rows ? rows[p] : p;
+        for (int u = 0; u < U; ++u) tok[u] = perm[j + u];
+        if (rows) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) tok[u] = rows[tok[u]];
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -471,23 +604,41 @@ __global__ void k_key_stats(StatsArgs a) {
     const int beg = offs[c], end = offs[c + 1];
     const int *perm = a.perm + (int64_t)h * a.L;
     const bf16 *K = a.K + (int64_t)h * a.L * a.d;
-    float mx = 0.f, mn = 0.f;
-    for (int j = beg; j < end; ++j) {
-        float v = bf2f(K[(int64_t)perm[j] * a.d + k]);
-        if (j == beg) {
-            mx = v;
-            mn = v;
-        } else {
-            mx = v > mx ? v : mx;
-            mn = v < mn ? v : mn;
+    // 16 members in flight per step (scattered rows); max and min are exact
+    // in any order, the SSE is summed in member order
+    constexpr int U = 16;
+    float mx = 0.f, mn = 0.f;  // an empty cluster keeps 0 (and count 0)
+    if (end > beg) mx = mn = bf2f(K[(int64_t)perm[beg] * a.d + k]);
+    int j = beg + 1;
+    for (; j + U <= end; j += U) {
+        float v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) v[u] = bf2f(K[(int64_t)perm[j + u] * a.d + k]);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            mx = v[u] > mx ? v[u] : mx;
+            mn = v[u] < mn ? v[u] : mn;
         }
+    }
+    for (; j < end; ++j) {
+        const float v = bf2f(K[(int64_t)perm[j] * a.d + k]);
+        mx = v > mx ? v : mx;
+        mn = v < mn ? v : mn;
     }
     a.kmax[ci * a.d + k] = __float2bfloat16(mx);
     a.kmin[ci * a.d + k] = __float2bfloat16(mn);
     if (k == 0) {
         float se = 0.f;
         const float *dm = a.dmin + (int64_t)h * a.L;
-        for (int j = beg; j < end; ++j) se = __fadd_rn(se, dm[perm[j]]);
+        int i = beg;
+        for (; i + U <= end; i += U) {
+            float v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) v[u] = dm[perm[i + u]];
+#pragma unroll
+            for (int u = 0; u < U; ++u) se = __fadd_rn(se, v[u]);
+        }
+        for (; i < end; ++i) se = __fadd_rn(se, dm[perm[i]]);
         a.sse[ci] = se;
         a.counts[ci] = end - beg;
     }

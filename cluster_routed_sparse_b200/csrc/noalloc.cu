@@ -100,7 +100,7 @@ extern "C" ac_status ac_cluster_q_noalloc(const uint16_t *Q, int32_t BH, int32_t
     {
         AssignArgs as{Qb, inv, L, nullptr, nullptr, L, centroids_out, cstride, nullptr, nullptr, Cq, labels_out,
                       nullptr, BH, d};
-        SortArgs so{labels_out, L, nullptr, L, nullptr, Cq, Cq, perm, offs, Cq + 1, counts, Cq, BH};
+        SortArgs so{labels_out, L, nullptr, L, nullptr, Cq, Cq, perm, offs, Cq + 1, counts, Cq, BH, nullptr};
         UpdateArgs up{Qb, inv, L, nullptr, perm, offs, Cq + 1, centroids_out, cstride, nullptr, nullptr, Cq, BH, d, Cq};
         for (int t = 0; t < iters; ++t) {
             if ((e = launch_assign_exact(as, s)) != cudaSuccess) goto cuda_error;
