@@ -39,6 +39,20 @@ NOISE_STD = 0.02
 
 
 # ---------------------------------------------------------------- inputs
+def max_over_ranks(ms_local, world, device, dist=None):
+    """The job's time: the slowest rank's (every rank takes part, every rank gets it)."""
+    import torch
+    t = torch.tensor([ms_local], device=device, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(ms, world, cfg):
+    """Whole-job dense-equivalent rate: every rank runs one layer of cfg (weak scaling)."""
+    return world * N_DENOISE * 4.0 * cfg.B * cfg.H * cfg.L * cfg.L * cfg.d / (ms * 1e-3) / 1e12
+
+
 def _gen_head(args):
     cfg, head = args
     from cluster_routed_sparse_b200 import synth
@@ -288,13 +302,10 @@ def main():
     launches = lay.launch_count() - launches1
     lay.synchronize()
     ms_local = e0.elapsed_time(e1) / args.steps
-    t = torch.tensor([ms_local], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks(ms_local, world, dev, dist if world > 1 else None)
 
     dense_flops_layer = 4.0 * cfg.B * cfg.H * cfg.L * cfg.L * cfg.d
-    value = world * N_DENOISE * dense_flops_layer / (ms * 1e-3) / 1e12
+    value = job_tflops(ms, world, cfg)
 
     # stage split (from the same timed calls)
     step0 = [c for i, c in enumerate(per_call) if i % N_DENOISE == 0]
@@ -323,9 +334,26 @@ def main():
                 "frac": round(achieved / peak_tf, 4), "traffic": traffic, "peak_source": peak_src,
                 "kernel": "k_sparse_attn (warm-step launch)",
                 "algorithmic_flops_per_launch": attn_flops,
-                "computed_tile_flops_per_launch": 4.0 * cfg.d * cnt["computed_pairs"]}
+                "computed_tile_flops_per_launch": 4.0 * cfg.d * cnt["computed_pairs"],
+                "computed_frac": round(4.0 * cfg.d * cnt["computed_pairs"] / (splitw["attn_kernel_ms"] * 1e-3) / 1e12
+                                       / peak_tf, 4)}
+    # achieved HBM fraction of the reduction stages of a warm call: the bytes they must read
+    # (a tensor of B*H*L*d bf16 per pass) over their measured time
+    hbm = peaks.get("hbm_gbs") or 6650.0
+    tensor_bytes = 2.0 * cfg.B * cfg.H * cfg.L * cfg.d
+    passes = {"q_cluster_ms": 1 + 3 + 2,   # norms, 3 assignment passes, 2 centre updates
+              "k_cluster_ms": 1 + 3 + 2 + 1,  # norms, 3 passes, 2 updates, exact distances
+              "stats_sort_ms": 1}          # per-cluster max / min / SSE
+    red = {}
+    for k, n in passes.items():
+        gbs = n * tensor_bytes / (splitw[k] * 1e-3) / 1e9
+        red[k.replace("_ms", "")] = {"algorithmic_bytes": n * tensor_bytes, "ms": round(splitw[k], 3),
+                                     "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / hbm, 4)}
 
     extra = {"step0": split0, "warm": splitw, "counters_last_call": cnt,
+             "reduction_stages_hbm": red,
+             "clustering_share_warm": round((splitw["q_cluster_ms"] + splitw["k_cluster_ms"] + splitw["stats_sort_ms"]
+                                             + splitw["score_select_ms"]) / splitw["total_ms"], 4),
              "assign_counters_since_create": lay.assign_counters(),
              "kept_pair_frac": cnt["kept_pairs"] / float(cfg.H * cfg.L * cfg.L),
              "tile_efficiency": cnt["kept_pairs"] / max(1, cnt["computed_pairs"])}

@@ -343,9 +343,89 @@ cudaError_t launch_counting_sort(const SortArgs &a, cudaStream_t s) {
 
 // ------------------------------------------------------------------ update
 // One block per (cluster, unit), one thread per dimension; members summed in
-// ascending order in fp32, then divided by the count.
+// ascending order in fp32, then divided by the count.  The members' rows are
+// scattered over the unit, so they are staged in shared memory by cp.async,
+// UPD_BATCH rows per batch and UPD_STAGES batches in flight, while the
+// threads add the rows of the oldest batch in order.
+constexpr int UPD_BATCH = 32;
+constexpr int UPD_STAGES = 4;
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <bool NORM>
 __global__ void k_update(UpdateArgs a) {
+    extern __shared__ __align__(16) uint8_t upd_sm[];
+    bf16 *rows_s = reinterpret_cast<bf16 *>(upd_sm);                                    // [STAGES][BATCH][d]
+    float *inv_s = reinterpret_cast<float *>(upd_sm + UPD_STAGES * UPD_BATCH * a.d * 2);  // [STAGES][BATCH]
+    const int c = blockIdx.x, h = blockIdx.y, k = threadIdx.x;
+    const int m = a.ncent ? a.ncent[h] : a.ncent_const;
+    if (c >= m) return;
+    const int *offs = a.offs + (int64_t)h * a.offs_stride;
+    const int beg = offs[c], end = offs[c + 1];
+    if (end <= beg) return;  // empty: keep the previous centre
+    const int *perm = a.perm + (int64_t)h * a.L;
+    const int *rows = a.rows ? a.rows + (int64_t)h * a.L : nullptr;
+    const bf16 *X = a.X + (int64_t)h * a.L * a.d;
+    const float *inv = NORM ? a.inv + (int64_t)h * a.L : nullptr;
+    const int nthr = blockDim.x, pieces = a.d / 8;  // 16-byte pieces per row
+    const int nb = (end - beg + UPD_BATCH - 1) / UPD_BATCH;
+    // batch b: members beg + b*BATCH .. into stage b % STAGES
+    auto issue = [&](int b) {
+        if (b < nb) {
+            const int st = b % UPD_STAGES;
+            const int j0 = beg + b * UPD_BATCH;
+            const int cnt = min(UPD_BATCH, end - j0);
+            for (int q = k; q < cnt * pieces; q += nthr) {
+                const int r = q / pieces, part = q % pieces;
+                const int p = perm[j0 + r];
+                const int t = rows ? rows[p] : p;
+                cp_async16(rows_s + ((size_t)st * UPD_BATCH + r) * a.d + part * 8, X + (int64_t)t * a.d + part * 8);
+            }
+            if (NORM && k < cnt) {
+                const int p = perm[j0 + k];
+                inv_s[st * UPD_BATCH + k] = inv[rows ? rows[p] : p];
+            }
+        }
+        cp_async_commit();  // an empty group past the last batch keeps the count uniform
+    };
+#pragma unroll 1
+    for (int b = 0; b < UPD_STAGES - 1; ++b) issue(b);
+    float s = 0.f;
+#pragma unroll 1
+    for (int b = 0; b < nb; ++b) {
+        issue(b + UPD_STAGES - 1);
+        cp_async_wait<UPD_STAGES - 1>();  // batch b has landed (this thread's copies)
+        __syncthreads();                  // ... and every thread's
+        const int st = b % UPD_STAGES;
+        const int cnt = min(UPD_BATCH, end - beg - b * UPD_BATCH);
+        if (k < a.d) {
+            const bf16 *rs = rows_s + (size_t)st * UPD_BATCH * a.d + k;
+            for (int r = 0; r < cnt; ++r) {
+                float v = bf2f(rs[(size_t)r * a.d]);
+                if (NORM) v = __fmul_rn(v, inv_s[st * UPD_BATCH + r]);
+                s = __fadd_rn(s, v);
+            }
+        }
+        __syncthreads();  // stage st is refilled by the next issue
+    }
+    cp_async_wait<0>();
+    if (k < a.d) {
+        const int off = a.coff ? a.coff[h] : 0;
+        a.C[(int64_t)h * a.cstride + (int64_t)(off + c) * a.d + k] = __fdiv_rn(s, (float)(end - beg));
+    }
+}
+
+// The same sums for small clusters (a few dozen members): each thread loads
+// 32 members ahead from global memory, no staging.
+template <bool NORM>
+__global__ void k_update_direct(UpdateArgs a) {
     const int c = blockIdx.x, h = blockIdx.y, k = threadIdx.x;
     const int m = a.ncent ? a.ncent[h] : a.ncent_const;
     if (c >= m || k >= a.d) return;
@@ -357,8 +437,6 @@ __global__ void k_update(UpdateArgs a) {
     const bf16 *X = a.X + (int64_t)h * a.L * a.d;
     const float *inv = NORM ? a.inv + (int64_t)h * a.L : nullptr;
     float s = 0.f;
-    // 32 members in flight per step (their rows are scattered over the unit:
-    // the sum is latency bound); the additions stay in ascending order
     constexpr int U = 32;
     int j = beg;
     for (; j + U <= end; j += U) {
@@ -379,8 +457,8 @@ __global__ void k_update(UpdateArgs a) {
         for (int u = 0; u < U; ++u) s = __fadd_rn(s, v[u]);
     }
     for (; j < end; ++j) {
-        int p = perm[j];
-        int t = rows ? rows[p] : p;
+        const int p = perm[j];
+        const int t = rows ? rows[p] : p;
         float v = bf2f(X[(int64_t)t * a.d + k]);
         if (NORM) v = __fmul_rn(v, inv[t]);
         s = __fadd_rn(s, v);
@@ -391,8 +469,15 @@ __global__ void k_update(UpdateArgs a) {
 
 cudaError_t launch_update(const UpdateArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)a.max_cent, (unsigned)a.BH);
-    if (a.inv) k_update<true><<<grid, a.d, 0, s>>>(a);
-    else k_update<false><<<grid, a.d, 0, s>>>(a);
+    // few, large clusters (queries): staged batches; many small ones: direct
+    if ((int64_t)a.max_cent * 256 <= a.L) {
+        const size_t smem = (size_t)UPD_STAGES * UPD_BATCH * (a.d * 2 + 4);
+        if (a.inv) k_update<true><<<grid, a.d, smem, s>>>(a);
+        else k_update<false><<<grid, a.d, smem, s>>>(a);
+    } else {
+        if (a.inv) k_update_direct<true><<<grid, a.d, 0, s>>>(a);
+        else k_update_direct<false><<<grid, a.d, 0, s>>>(a);
+    }
     AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
