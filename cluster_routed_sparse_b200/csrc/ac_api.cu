@@ -78,6 +78,30 @@ ac_status make_tmap(ac_ctx *c, CUtensorMap *tm, void *base, int64_t rows, int d,
     return AC_OK;
 }
 
+// Rows of 16 bf16, boxes of 8 columns x box_rows rows, no swizzle: in shared
+// memory a box is box_rows x 16 bytes, i.e. 8-row x 16-byte core matrices
+// one after the other.
+ac_status make_tmap_plain16(ac_ctx *c, CUtensorMap *tm, void *base, int64_t rows, int box_rows) {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+            return fail(c, AC_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    cuuint64_t dims[2] = {16, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {32};
+    cuuint32_t box[2] = {8, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(c, AC_ERR_CUDA, "cuTensorMapEncodeTiled (norm parts) failed");
+    return AC_OK;
+}
+
 // K and V boxes of G 8-row groups x all d columns in one copy, laid out in
 // shared memory as [group][column half][8 rows][64 columns] (dims: column,
 // row in group, half, group; strides d*2, 128 and 8*d*2 bytes), 128-byte
@@ -169,6 +193,8 @@ bool make_fast(ac_ctx *c, Lloyd &k, const bf16 *X, bool queries, const float *C,
     FastAssignArgs &a = k.fa;
     a.tm_x = tmx;
     a.tm_c = queries ? &c->tm_chi_q : &c->tm_chi_k;
+    a.tm_cn = queries ? nullptr : &c->tm_cnp_k;
+    a.cnp = queries ? nullptr : c->cnp_k;
     a.X = X;
     a.inv = queries ? c->inv_q : nullptr;
     a.rowsq = queries ? nullptr : c->rowsq_k;
@@ -396,7 +422,7 @@ void free_all(ac_ctx *c) {
                    c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->Qp, c->Kp, c->Vp,
                    c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err, c->chi_q, c->chi_k, c->cn,
                    c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats, c->rbox, c->pgoff, c->nrange,
-                   c->sort_scratch};
+                   c->sort_scratch, c->cnp_k};
     for (void *p : dev)
         if (p) cudaFree(p);
     void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err};
@@ -461,7 +487,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
         c->fast_assign = !(ev && ev[0] == '1');
     }
     c->Cpad_q = (c->Cq + 31) & ~31;
-    c->CH_q = std::min(96, c->Cpad_q);  // two-term chunks (c_hi + c_lo) of at most 96 centres
+    c->CH_q = std::min(64, c->Cpad_q);  // two-term chunks (c_hi + c_lo) of at most 64 centres
     c->Cpad_k = (c->Ccap + 31) & ~31;
     c->CH_k = std::min(128, c->Cpad_k);
     const size_t BH = c->BH, Lz = L, dz = d, Cq = c->Cq, Cc = c->Ccap, m0 = cfg->m0;
@@ -510,6 +536,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->tile_prefix, BH * Cq + 1));
     A(dalloc(&c->chi_q, 2 * BH * c->Cpad_q * dz));
     A(dalloc(&c->chi_k, BH * c->Cpad_k * dz));
+    A(dalloc(&c->cnp_k, BH * c->Cpad_k * 16));
     A(dalloc(&c->cn, BH * std::max(c->Cpad_q, c->Cpad_k)));
     A(dalloc(&c->hstat, 2 * BH));
     A(dalloc(&c->rowsq_k, BH * Lz));
@@ -553,7 +580,8 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
                   make_tmap_kv(c, &c->tm_vg[i], c->Vp, (int64_t)BH * c->Lpad / 8, d, 1 << i) == AC_OK;
     if (!maps_ok ||
         make_tmap(c, &c->tm_chi_q, c->chi_q, (int64_t)2 * BH * c->Cpad_q, d, c->CH_q) != AC_OK ||
-        make_tmap(c, &c->tm_chi_k, c->chi_k, (int64_t)BH * c->Cpad_k, d, c->CH_k) != AC_OK) {
+        make_tmap(c, &c->tm_chi_k, c->chi_k, (int64_t)BH * c->Cpad_k, d, c->CH_k) != AC_OK ||
+        make_tmap_plain16(c, &c->tm_cnp_k, c->cnp_k, (int64_t)BH * c->Cpad_k, c->CH_k) != AC_OK) {
         free_all(c);
         delete c;
         return AC_ERR_CUDA;

@@ -77,6 +77,8 @@ struct ac_ctx {
     int *amb_count;    // [1]
     unsigned long long *asg_stats;  // [2] uncertain rows, rows rescored against every centre
     CUtensorMap tm_chi_q, tm_chi_k;
+    bf16 *cnp_k;       // [BH, Cpad_k, 16] |c'|^2 of the key centres as three bf16 parts
+    CUtensorMap tm_cnp_k;
     CUtensorMap tm_xq, tm_xk;  // caller's Q / K of the current call
     int num_sms;
     bool fast_assign;
@@ -148,6 +150,7 @@ cudaError_t launch_assign_exact(const AssignArgs &a, cudaStream_t s);
 struct FastAssignArgs {
     const CUtensorMap *tm_x;   // rows [BH * L, d], box {64, 128}
     const CUtensorMap *tm_c;   // Chi rows [BH * Cpad (x2 with two terms), d], box {64, CH}
+    const CUtensorMap *tm_cn;  // cnp [BH * Cpad, 16] bf16, box {8, CH}, no swizzle (keys only)
     const bf16 *X;
     const float *inv;          // [BH, L] or null
     const float *rowsq;        // [BH, L] |x|^2 when inv is null
@@ -157,7 +160,7 @@ struct FastAssignArgs {
     const int *ncent; int ncent_const;
     int Cpad, CH;              // CH <= 128, <= 96 with two terms
     bool two_term;             // centres as bf16 c_hi + c_lo (else c_hi alone)
-    bf16 *Chi; float *cn; unsigned int *hstat;
+    bf16 *Chi; bf16 *cnp; float *cn; unsigned int *hstat;
     int *labels;
     float *dmin;               // or null
     int4 *cand; int *amb_list; int *amb_count;

@@ -11,7 +11,10 @@
 //      tensor cores form s = x . c' for every centre (key rows are exact bf16;
 //      query rows are scaled by their fp32 inverse norm afterwards);
 //   2. the epilogue keeps per row the 4 smallest A(c) = |c'|^2 - 2 s, the
-//      squared distance to c' less the row's own |x|^2;
+//      squared distance to c' less the row's own |x|^2 (for keys the tensor
+//      cores add |c'|^2 too: the centre rows hold -2 c_hi, and one more K=16
+//      slice multiplies a constant [1 1 1 0 ...] row by |c'|^2 split into three
+//      bf16 parts, so the accumulator holds A itself);
 //   3. a rigorous bound E on |D(x, c) - |x|^2 - A(c)| (bf16 split, tensor-core
 //      accumulation, the fp32 rounding of D itself; see assign_bound) decides:
 //      when every other centre's lower bound A - E lies above the best's upper
@@ -30,7 +33,8 @@ constexpr int AU = 2 * AM;    // rows per work unit: two MMAs share every centre
 constexpr int ACH = 128;      // centres per chunk at most (MMA N)
 constexpr int A_EPI = 256;    // epilogue threads: one per row of the unit
 constexpr int A_THREADS = A_EPI + 64;
-constexpr int A_NCMAX = 3;    // centre chunk stages (2 with two-term centres)
+constexpr int A_NC = 2;       // centre chunk stages
+constexpr int A_NCMAX = 3;    // barriers reserved
 
 // Shared memory: [2] row units (two 128-row tiles each) | [NC] centre chunks.
 // A chunk holds the c_hi rows (and the c_lo rows) of up to ACH centres, each
@@ -42,9 +46,12 @@ struct ALayout {
     static constexpr uint32_t X_BYTES = 2 * XT_BYTES;        // one unit
     static constexpr uint32_t OFF_X = 0;
     static constexpr uint32_t OFF_C = OFF_X + 2 * X_BYTES;
-    // three c_hi stages of ACH centres, or two c_hi + c_lo stages of up to 96
-    static constexpr uint32_t C_REGION = 3 * HALVES * ACH * 128;
-    static constexpr uint32_t OFF_BAR = OFF_C + C_REGION;
+    // two stages of ACH key centres (-2 c_hi, then the |c'|^2 slice: two
+    // no-swizzle 16-byte columns of ACH rows), or of up to 64 query centres
+    // (c_hi, c_lo)
+    static constexpr uint32_t C_REGION = A_NC * (HALVES * ACH * 128 + ACH * 32);
+    static constexpr uint32_t OFF_XE = OFF_C + C_REGION;  // the constant [1 1 1 0 ...] K slice, 128 rows
+    static constexpr uint32_t OFF_BAR = OFF_XE + AM * 32;
     static constexpr uint32_t BYTES = OFF_BAR + 256;
     static constexpr uint32_t SMEM = BYTES + 1024;
 };
@@ -155,10 +162,10 @@ __device__ __forceinline__ float assign_threshold(float d1, float sq, float delt
     return d1 + 4.5f * assign_bound(d1, sq, delta, e);
 }
 
-template <int D>
+template <int D, bool FOLD>
 __global__ void __launch_bounds__(A_THREADS, 1)
     k_assign_mma(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_c,
-                 const AsgParams p) {
+                 const __grid_constant__ CUtensorMap tm_cn, const AsgParams p) {
     using LY = ALayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -186,6 +193,15 @@ __global__ void __launch_bounds__(A_THREADS, 1)
     if (warp == 9) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
+    }
+    if (FOLD && tid < AM) {
+        // K slice of ones against the |c'|^2 parts: row r = [1 1 1 0 0 0 0 0 | 0 ...] as
+        // core matrices [8-row group][16-byte column][8 rows][16 B] (SBO 256, LBO 128)
+        uint4 *xe = reinterpret_cast<uint4 *>(sm + LY::OFF_XE);
+        const int grp = tid >> 3, rr = tid & 7;
+        xe[grp * 16 + rr] = make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);
+        xe[grp * 16 + 8 + rr] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -223,7 +239,11 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                         break;
                     }
                     const uint32_t cs = sbase + LY::OFF_C + c * p.c_stage;
-                    mbar_arrive_expect_tx(ABAR(B_CF + c), terms * LY::HALVES * p.CH * 128);
+                    mbar_arrive_expect_tx(ABAR(B_CF + c), terms * LY::HALVES * p.CH * 128 + (FOLD ? p.CH * 32 : 0));
+                    if (FOLD)  // the |c'|^2 parts: two 8-column boxes of CH rows, no swizzle
+                        for (int q = 0; q < 2; ++q)
+                            tma_load_2d(cs + LY::HALVES * p.CH * 128 + q * p.CH * 16, &tm_cn, q * 8,
+                                        h * p.Cpad + ch * p.CH, ABAR(B_CF + c));
                     for (int hf = 0; hf < LY::HALVES; ++hf)
                         tma_load_2d(cs + hf * p.CH * 128, &tm_c, hf * 64, h * p.Cpad + ch * p.CH, ABAR(B_CF + c));
                     if (p.two_term)  // c_lo rows follow the c_hi rows of all units in the tensor map
@@ -277,6 +297,9 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                             tc_mma_bf16(tmem + (a * 2 + i) * ACH, sdesc_sw128(xa + xoff, 16, 1024),
                                         sdesc_sw128(ca + coff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
                         }
+                        if (FOLD)  // + |c'|^2 (ones x parts)
+                            tc_mma_bf16(tmem + (a * 2 + i) * ACH, sdesc_noswz(sbase + LY::OFF_XE, 128, 256),
+                                        sdesc_noswz(ca + LY::HALVES * p.CH * 128, p.CH * 16, 128), idesc, 1u);
                     }
                     tc_commit(ABAR(B_AF + a));
                     tc_commit(ABAR(B_CE + c));
@@ -346,7 +369,7 @@ __global__ void __launch_bounds__(A_THREADS, 1)
             float T = INFINITY;
             const int nch = (m + p.CH - 1) / p.CH;
             float4 cq[8];
-            load_cn(cnh, cq);
+            if (!FOLD) load_cn(cnh, cq);
             for (int ch = 0; ch < nch; ++ch, ++g) {
                 const uint32_t a = g & 1;
                 const int rem = m - ch * p.CH;
@@ -359,23 +382,33 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                 for (int cg = 0; cg < N; cg += 32) {
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_off + (a * 2 + ti) * ACH + cg, r);
-                    // norms of the next group: same chunk, else the next chunk
                     float4 cqn[8];
-                    const int ncg = cg + 32 < N ? ch * p.CH + cg + 32 : (ch + 1) * p.CH;
-                    if (ncg < m) load_cn(cnh + ncg, cqn);
+                    if (!FOLD) {
+                        // norms of the next group: same chunk, else the next chunk
+                        const int ncg = cg + 32 < N ? ch * p.CH + cg + 32 : (ch + 1) * p.CH;
+                        if (ncg < m) load_cn(cnh + ncg, cqn);
+                    }
                     tmem_ld_wait();
                     float mn = INFINITY;
+                    if (FOLD) {  // the accumulator holds A already: 4 partial minima, 3-input min
+                        float pmn[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float v0 = fmaf(m2i, __uint_as_float(r[4 * q + 0]), cq[q].x);
-                        const float v1 = fmaf(m2i, __uint_as_float(r[4 * q + 1]), cq[q].y);
-                        const float v2 = fmaf(m2i, __uint_as_float(r[4 * q + 2]), cq[q].z);
-                        const float v3 = fmaf(m2i, __uint_as_float(r[4 * q + 3]), cq[q].w);
-                        r[4 * q + 0] = __float_as_uint(v0);
-                        r[4 * q + 1] = __float_as_uint(v1);
-                        r[4 * q + 2] = __float_as_uint(v2);
-                        r[4 * q + 3] = __float_as_uint(v3);
-                        mn = fminf(mn, fminf(fminf(v0, v1), fminf(v2, v3)));
+                        for (int q = 0; q < 16; ++q)
+                            pmn[q & 3] = fmin3(pmn[q & 3], __uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+                        mn = fminf(fmin3(pmn[0], pmn[1], pmn[2]), pmn[3]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float v0 = fmaf(m2i, __uint_as_float(r[4 * q + 0]), cq[q].x);
+                            const float v1 = fmaf(m2i, __uint_as_float(r[4 * q + 1]), cq[q].y);
+                            const float v2 = fmaf(m2i, __uint_as_float(r[4 * q + 2]), cq[q].z);
+                            const float v3 = fmaf(m2i, __uint_as_float(r[4 * q + 3]), cq[q].w);
+                            r[4 * q + 0] = __float_as_uint(v0);
+                            r[4 * q + 1] = __float_as_uint(v1);
+                            r[4 * q + 2] = __float_as_uint(v2);
+                            r[4 * q + 3] = __float_as_uint(v3);
+                            mn = fminf(mn, fminf(fminf(v0, v1), fminf(v2, v3)));
+                        }
                     }
                     // This group holds the best so far or a near tie for some
                     // row of the warp: mark the columns within the new threshold
@@ -398,8 +431,10 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                             }
                         }
                     }
+                    if (!FOLD) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) cq[q] = cqn[q];
+                        for (int q = 0; q < 8; ++q) cq[q] = cqn[q];
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(ABAR(B_AE + a));
@@ -558,18 +593,24 @@ __global__ void k_row_sqnorm(const bf16 *__restrict__ X, int64_t rows, int d, fl
 // largest |c'|^2, both in fp64 rounded up.  Chi holds [BH, Cpad, d] c_hi rows
 // then (two terms) [BH, Cpad, d] c_lo rows.  Rows c >= m up to Cpad are zero
 // with cn = +inf.
+// With fold (keys), Chi holds -2 c_hi instead (exact: a power-of-two scale) and
+// cnp [BH, Cpad, 16] the parts hi, mid, lo of fp32 |c'|^2 as bf16 (their sum is
+// |c'|^2 to 2^-26 relative), then zeros; a padding row's first part is the
+// largest finite bf16, so its A never wins.
 __global__ void k_centre_prep(const float *__restrict__ C, int64_t cstride, const int *__restrict__ ncent,
-                              int ncent_const, int d, int Cpad, int two_term, bf16 *__restrict__ Chi,
-                              float *__restrict__ cn, unsigned int *__restrict__ hstat) {
+                              int ncent_const, int d, int Cpad, int two_term, int fold, bf16 *__restrict__ Chi,
+                              bf16 *__restrict__ cnp, float *__restrict__ cn, unsigned int *__restrict__ hstat) {
     const int c = blockIdx.x, h = blockIdx.y;
     const int m = ncent ? ncent[h] : ncent_const;
     const int64_t lo_off = (int64_t)gridDim.y * Cpad * d;
     bf16 *dst = Chi + ((int64_t)h * Cpad + c) * d;
+    bf16 *pn = fold ? cnp + ((int64_t)h * Cpad + c) * 16 : nullptr;
     if (c >= m) {
         for (int k = threadIdx.x; k < d; k += blockDim.x) {
             dst[k] = __float2bfloat16_rn(0.f);
             if (two_term) dst[lo_off + k] = __float2bfloat16_rn(0.f);
         }
+        if (fold && threadIdx.x < 16) pn[threadIdx.x] = __ushort_as_bfloat16(threadIdx.x == 0 ? 0x7F7Fu : 0u);
         if (threadIdx.x == 0) cn[(int64_t)h * Cpad + c] = INFINITY;
         return;
     }
@@ -578,7 +619,7 @@ __global__ void k_centre_prep(const float *__restrict__ C, int64_t cstride, cons
     for (int k = threadIdx.x; k < d; k += blockDim.x) {
         const float v = src[k];
         const bf16 hi = __float2bfloat16_rn(v);
-        dst[k] = hi;
+        dst[k] = fold ? __float2bfloat16_rn(-2.f * __bfloat162float(hi)) : hi;
         double rep = (double)__bfloat162float(hi);
         if (two_term) {
             const bf16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));  // v - hi is exact in fp32
@@ -607,7 +648,18 @@ __global__ void k_centre_prep(const float *__restrict__ C, int64_t cstride, cons
             te += se[i];
             tn += sn[i];
         }
-        cn[(int64_t)h * Cpad + c] = (float)tn;
+        const float cnf = (float)tn;
+        cn[(int64_t)h * Cpad + c] = cnf;
+        if (fold) {
+            const bf16 p0 = __float2bfloat16_rn(cnf);
+            const float r1 = cnf - __bfloat162float(p0);
+            const bf16 p1 = __float2bfloat16_rn(r1);
+            const bf16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+            pn[0] = p0;
+            pn[1] = p1;
+            pn[2] = p2;
+            for (int q = 3; q < 16; ++q) pn[q] = __float2bfloat16_rn(0.f);
+        }
         const float delta = __double2float_ru(sqrt(te) * (1.0 + 1e-12));
         atomicMax(&hstat[2 * h], __float_as_uint(delta));
         atomicMax(&hstat[2 * h + 1], __float_as_uint(__double2float_ru(tn)));
@@ -616,12 +668,12 @@ __global__ void k_centre_prep(const float *__restrict__ C, int64_t cstride, cons
 
 static_assert(ALayout<128>::SMEM <= 232448, "assignment kernel exceeds the shared memory of a block");
 
-template <int D>
+template <int D, bool FOLD>
 cudaError_t launch_mma(const FastAssignArgs &a, const AsgParams &p, int grid, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(k_assign_mma<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_assign_mma<D, FOLD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)ALayout<D>::SMEM);
     if (e != cudaSuccess) return e;
-    k_assign_mma<D><<<grid, A_THREADS, ALayout<D>::SMEM, s>>>(*a.tm_x, *a.tm_c, p);
+    k_assign_mma<D, FOLD><<<grid, A_THREADS, ALayout<D>::SMEM, s>>>(*a.tm_x, *a.tm_c, FOLD ? *a.tm_cn : *a.tm_c, p);
     AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
@@ -642,8 +694,9 @@ cudaError_t launch_assign_fast(const FastAssignArgs &a, cudaStream_t s) {
     // 1. split the centres
     if ((e = cudaMemsetAsync(a.hstat, 0, sizeof(unsigned int) * 2 * BH, s)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(a.amb_count, 0, sizeof(int), s)) != cudaSuccess) return e;
+    const bool fold = !a.two_term;
     k_centre_prep<<<dim3(a.Cpad, BH), 64, 0, s>>>(a.C, a.cstride, a.ncent, a.ncent_const, a.d, a.Cpad,
-                                                  a.two_term ? 1 : 0, a.Chi, a.cn, a.hstat);
+                                                  a.two_term ? 1 : 0, fold ? 1 : 0, a.Chi, a.cnp, a.cn, a.hstat);
     AC_NOTE_LAUNCH();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 2. tensor-core pass with the top-4 epilogue
@@ -662,22 +715,25 @@ cudaError_t launch_assign_fast(const FastAssignArgs &a, cudaStream_t s) {
     p.CH = a.CH;
     p.units_per_head = (int)((a.L + AU - 1) / AU);
     p.two_term = a.two_term ? 1 : 0;
-    p.e_tc = (float)(a.two_term ? 2 * a.d : a.d) * 1.1920928955078125e-07f;  // products * 2^-23
+    // products * 2^-23; with the folded |c'|^2 the accumulated terms also sum |c'|^2,
+    // so (d + 16) products at twice the rate
+    p.e_tc = a.two_term ? (float)(2 * a.d) * 1.1920928955078125e-07f : (float)(a.d + 16) * 2.384185791015625e-07f;
     p.labels = a.labels;
     p.cand = a.cand;
     p.amb_list = a.amb_list;
     p.amb_count = a.amb_count;
     p.stats = a.stats;
     p.err = a.err;
-    p.c_stage = (uint32_t)((a.two_term ? 2 : 1) * (a.d / 64) * a.CH * 128);
-    p.nc = a.two_term ? 2 : 3;
+    p.c_stage = (uint32_t)(a.two_term ? 2 * (a.d / 64) * a.CH * 128 : (a.d / 64) * a.CH * 128 + a.CH * 32);
+    p.nc = A_NC;
     // the centre stages must fit their region of shared memory
-    if (a.CH < 32 || a.CH > ACH || (a.CH & 31) || (a.two_term && a.CH > 96) || (a.Cpad & 31) ||
-        (uint64_t)p.nc * p.c_stage > 3ull * (a.d / 64) * ACH * 128)
+    if (a.CH < 32 || a.CH > ACH || (a.CH & 31) || (a.two_term && a.CH > 64) || (a.Cpad & 31) ||
+        (uint64_t)p.nc * p.c_stage > (uint64_t)A_NC * ((a.d / 64) * ACH * 128 + ACH * 32))
         return cudaErrorInvalidValue;
     const int nunits = BH * p.units_per_head;
     const int grid = nunits < a.num_sms ? nunits : a.num_sms;
-    e = a.d == 128 ? launch_mma<128>(a, p, grid, s) : launch_mma<64>(a, p, grid, s);
+    if (fold) e = a.d == 128 ? launch_mma<128, true>(a, p, grid, s) : launch_mma<64, true>(a, p, grid, s);
+    else e = a.d == 128 ? launch_mma<128, false>(a, p, grid, s) : launch_mma<64, false>(a, p, grid, s);
     if (e != cudaSuccess) return e;
     // 3. exact rescoring of the uncertain rows
     if (a.inv)
