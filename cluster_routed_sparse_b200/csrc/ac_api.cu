@@ -170,14 +170,15 @@ cudaError_t assign_pass(ac_ctx *c, const Lloyd &k, bool want_dmin, cudaStream_t 
     return launch_assign_exact(k.as, s);
 }
 
-cudaError_t run_lloyd(ac_ctx *c, Lloyd &k, int T, bool final_sort, cudaStream_t s) {
+cudaError_t run_lloyd(ac_ctx *c, Lloyd &k, int T, bool final_sort, cudaStream_t s, bool final_dmin = true) {
     cudaError_t e;
+    k.up.err = c->err;
     for (int t = 0; t < T; ++t) {
         if ((e = assign_pass(c, k, false, s)) != cudaSuccess) return e;
         if ((e = launch_counting_sort(k.so, s)) != cudaSuccess) return e;
         if ((e = launch_update(k.up, s)) != cudaSuccess) return e;
     }
-    if ((e = assign_pass(c, k, true, s)) != cudaSuccess) return e;
+    if ((e = assign_pass(c, k, final_dmin, s)) != cudaSuccess) return e;
     if (final_sort && (e = launch_counting_sort(k.so, s)) != cudaSuccess) return e;
     return cudaSuccess;
 }
@@ -349,7 +350,7 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
     fin.as = AssignArgs{K, nullptr, L, nullptr, nullptr, L, c->cent_k, cstride, nullptr, c->n_k, 0, c->labels_k,
                         c->dmin_k, BH, d};
     make_fast(c, fin, K, false, c->cent_k, cstride, c->n_k, 0, c->labels_k, c->dmin_k);
-    CK(assign_pass(c, fin, true, s), "final assign");
+    CK(assign_pass(c, fin, false, s), "final assign");  // dmin: key statistics
     return AC_OK;
 }
 
@@ -375,7 +376,8 @@ ac_status cluster_k_warm(ac_ctx *c, const bf16 *K, cudaStream_t s) {
     k.up = UpdateArgs{K, nullptr, L, nullptr, c->perm_k, c->offs_k, c->Ccap + 1, c->cent_k, cstride, nullptr,
                       c->st_m, 0, BH, d, c->Ccap};
     make_fast(c, k, K, false, c->cent_k, cstride, c->st_m, 0, c->labels_k, c->dmin_k);
-    CK(run_lloyd(c, k, c->cfg.iters_warm, false, s), "warm lloyd");
+    // dmin of the final labels comes from the key statistics
+    CK(run_lloyd(c, k, c->cfg.iters_warm, false, s, false), "warm lloyd");
     return AC_OK;
 }
 
@@ -385,7 +387,8 @@ ac_status key_stats_impl(ac_ctx *c, const bf16 *K, cudaStream_t s) {
                 c->counts_k, c->Ccap, c->BH, c->sort_scratch};
     CK(launch_counting_sort(so, s), "k sort");
     StatsArgs st{K, c->L, c->perm_k, c->offs_k, c->Ccap + 1, c->dmin_k, c->n_k, c->Ccap, c->d, c->BH,
-                 c->counts_k, c->kmax, c->kmin, c->sse, c->mse, c->comp};
+                 c->counts_k, c->kmax, c->kmin, c->sse, c->mse, c->comp, c->cent_k, (int64_t)c->Ccap * c->d,
+                 c->err};
     CK(launch_key_stats(st, s), "k stats");
     c->have_k = true;
     return AC_OK;
@@ -542,7 +545,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->rowsq_k, BH * Lz));
     A(dalloc(&c->cand, BH * Lz));
     A(dalloc(&c->amb_list, BH * Lz));
-    A(dalloc(&c->amb_count, 1));
+    A(dalloc(&c->amb_count, 2));
     A(dalloc(&c->asg_stats, 2));
     A(dalloc(&c->Qp, BH * Lz * dz));
     A(dalloc(&c->Kp, BH * (size_t)c->Lpad * dz));

@@ -152,6 +152,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int3
         : "memory");
 }
 
+// Plain bulk copy of `bytes` contiguous bytes from global memory into this
+// CTA's shared memory (no tensor map, no cluster multicast), completion counted
+// on `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 // 4-D tiled bulk tensor load (coordinates x innermost).  No cluster multicast.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *tmap, int32_t x, int32_t y, int32_t z,
                                             int32_t w, uint32_t bar) {

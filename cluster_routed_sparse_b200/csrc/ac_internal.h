@@ -200,6 +200,7 @@ struct UpdateArgs {
     float *C; int64_t cstride; const int *coff;
     const int *ncent; int ncent_const;
     int BH, d, max_cent;
+    uint32_t *err = nullptr;  // bounded-wait failures are recorded here
 };
 cudaError_t launch_update(const UpdateArgs &a, cudaStream_t s);
 
@@ -227,10 +228,13 @@ cudaError_t launch_remove(const float *dist, const float *tau, int *u_idx, int *
                           const int *st_m, int *removed_stage, int stage, int64_t L, int BH,
                           cudaStream_t s);
 
+// Also writes dmin[h, t] = exact squared distance of key t to its centre.
 struct StatsArgs {
     const bf16 *K; int64_t L; const int *perm; const int *offs; int offs_stride;
-    const float *dmin; const int *n_k; int Ccap; int d; int BH;
+    float *dmin; const int *n_k; int Ccap; int d; int BH;
     int *counts; bf16 *kmax; bf16 *kmin; float *sse; float *mse; float *comp;
+    const float *C; int64_t cstride;  // key centres
+    uint32_t *err;
 };
 cudaError_t launch_key_stats(const StatsArgs &a, cudaStream_t s);
 

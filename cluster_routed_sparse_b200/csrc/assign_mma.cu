@@ -83,7 +83,8 @@ struct AsgParams {
     float e_tc;           // tensor-core error coefficient (see assign_bound)
     int *labels;
     int4 *cand;
-    int *amb_list, *amb_count;
+    int *amb_list, *amb_count;  // candidate rows from the front, every-centre rows from the back
+    int64_t amb_cap;            // entries of amb_list
     unsigned long long *stats;  // [0] ambiguous rows, [1] rows rescored against every centre
     uint32_t *err;
 };
@@ -449,12 +450,13 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                 // beyond the kept four are settled when the fourth is.
                 const bool beyond = m > 4 && (a4 || sqrtf(fmaxf(d4 + sq, 0.f) + 2.f * e) <= 2.f * delta);
                 p.labels[f] = i1;
-                if (a2 || a3 || a4 || beyond) {
+                if (beyond) {
+                    const int pos = atomicAdd(p.amb_count + 1, 1);
+                    p.amb_list[p.amb_cap - 1 - pos] = (int)f;
+                } else if (a2 || a3 || a4) {
                     const int pos = atomicAdd(p.amb_count, 1);
                     p.amb_list[pos] = (int)f;
-                    p.cand[pos] = beyond ? make_int4(-2, 0, 0, 0)
-                                         : make_int4(i1, a2 ? i2 : -1, a3 ? i3 : -1, a4 ? i4 : -1);
-                    if (beyond) atomicAdd(p.stats + 1, 1ull);
+                    p.cand[pos] = make_int4(i1, a2 ? i2 : -1, a3 ? i3 : -1, a4 ? i4 : -1);
                 }
             }
         }
@@ -502,41 +504,76 @@ __device__ __forceinline__ float exact_sqdist(const bf16 *__restrict__ xr, float
     return acc;
 }
 
-// One warp per uncertain row: exact distances of the candidates (lanes 0-3) or
-// of every centre (lane-strided, ascending per lane), argmin with the lowest
-// index among equal distances.
+// Rows with a few candidates: four consecutive lanes per row, lane j of the
+// group computes the exact distance of candidate j; the group's argmin takes
+// the lowest index among equal distances.
 template <bool NORM>
 __global__ void k_assign_resolve(const bf16 *__restrict__ X, const float *__restrict__ inv, int64_t L, int d,
-                                 const float *__restrict__ C, int64_t cstride, const int *__restrict__ ncent,
-                                 int ncent_const, const int4 *__restrict__ cand, const int *__restrict__ amb_list,
-                                 const int *__restrict__ amb_count, int *__restrict__ labels,
-                                 unsigned long long *__restrict__ stats) {
-    const int n = *amb_count;
-    const int lane = threadIdx.x & 31;
-    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, nw = (gridDim.x * blockDim.x) >> 5;
-    if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(stats, (unsigned long long)n);
-    for (int i = gw; i < n; i += nw) {
-        const int64_t f = amb_list[i];
+                                 const float *__restrict__ C, int64_t cstride, const int4 *__restrict__ cand,
+                                 const int *__restrict__ amb_list, const int *__restrict__ amb_count,
+                                 int *__restrict__ labels, unsigned long long *__restrict__ stats) {
+    const int n = amb_count[0];
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        atomicAdd(stats, (unsigned long long)(n + amb_count[1]));
+        atomicAdd(stats + 1, (unsigned long long)amb_count[1]);
+    }
+    const int lane = threadIdx.x & 31, j = lane & 3;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    // the loop bound is uniform per warp, so every lane takes part in the shuffles
+    for (int64_t base = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) - lane; base < 4 * (int64_t)n;
+         base += nthr) {
+        const int64_t t = base + lane;
+        const int i = (int)(t >> 2);
+        float best = INFINITY;
+        int arg = 0x7FFFFFFF;
+        int64_t f = 0;
+        if (i < n) {
+            f = amb_list[i];
+            const int4 cd = cand[i];
+            const int c = j == 0 ? cd.x : j == 1 ? cd.y : j == 2 ? cd.z : cd.w;
+            if (c >= 0) {
+                const int h = (int)(f / L);
+                best = exact_sqdist<NORM>(X + f * d, NORM ? inv[f] : 1.f, C + (int64_t)h * cstride + (int64_t)c * d, d);
+                arg = c;
+            }
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            const float ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+            const int oa = __shfl_xor_sync(0xFFFFFFFFu, arg, o);
+            if (ob < best || (ob == best && oa < arg)) {
+                best = ob;
+                arg = oa;
+            }
+        }
+        if (i < n && j == 0) labels[f] = arg;
+    }
+}
+
+// Rows whose every centre stays in doubt: one block per row, thread t scores
+// centres t, t + blockDim, ... in ascending order; lowest index on ties.
+template <bool NORM>
+__global__ void k_assign_resolve_all(const bf16 *__restrict__ X, const float *__restrict__ inv, int64_t L, int d,
+                                     const float *__restrict__ C, int64_t cstride, const int *__restrict__ ncent,
+                                     int ncent_const, const int *__restrict__ amb_list, int64_t amb_cap,
+                                     const int *__restrict__ amb_count, int *__restrict__ labels) {
+    __shared__ float sb[32];
+    __shared__ int sa[32];
+    const int n = amb_count[1];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+        const int64_t f = amb_list[amb_cap - 1 - i];
         const int h = (int)(f / L);
         const int m = ncent ? ncent[h] : ncent_const;
         const bf16 *xr = X + f * d;
         const float s = NORM ? inv[f] : 1.f;
         const float *Ch = C + (int64_t)h * cstride;
-        const int4 cd = cand[i];
         float best = INFINITY;
         int arg = 0x7FFFFFFF;
-        if (cd.x == -2) {
-            for (int c = lane; c < m; c += 32) {
-                const float v = exact_sqdist<NORM>(xr, s, Ch + (int64_t)c * d, d);
-                if (v < best) {
-                    best = v;
-                    arg = c;
-                }
-            }
-        } else if (lane < 4) {
-            const int c = lane == 0 ? cd.x : lane == 1 ? cd.y : lane == 2 ? cd.z : cd.w;
-            if (c >= 0) {
-                best = exact_sqdist<NORM>(xr, s, Ch + (int64_t)c * d, d);
+        for (int c = threadIdx.x; c < m; c += blockDim.x) {
+            const float v = exact_sqdist<NORM>(xr, s, Ch + (int64_t)c * d, d);
+            if (v < best) {
+                best = v;
                 arg = c;
             }
         }
@@ -549,11 +586,23 @@ __global__ void k_assign_resolve(const bf16 *__restrict__ X, const float *__rest
                 arg = oa;
             }
         }
-        if (lane == 0) labels[f] = arg == 0x7FFFFFFF ? 0 : arg;
+        if (lane == 0) {
+            sb[warp] = best;
+            sa[warp] = arg;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            for (int w = 1; w < nwarp; ++w)
+                if (sb[w] < best || (sb[w] == best && sa[w] < arg)) {
+                    best = sb[w];
+                    arg = sa[w];
+                }
+            labels[f] = arg == 0x7FFFFFFF ? 0 : arg;
+        }
+        __syncthreads();
     }
 }
 
-// dmin[f] = exact distance of row f to its labelled centre.
 template <bool NORM>
 __global__ void k_exact_dmin(const bf16 *__restrict__ X, const float *__restrict__ inv, int64_t L, int d,
                              const float *__restrict__ C, int64_t cstride, const int *__restrict__ nrows,
@@ -693,7 +742,7 @@ cudaError_t launch_assign_fast(const FastAssignArgs &a, cudaStream_t s) {
     if (BH <= 0 || a.L <= 0) return cudaSuccess;
     // 1. split the centres
     if ((e = cudaMemsetAsync(a.hstat, 0, sizeof(unsigned int) * 2 * BH, s)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(a.amb_count, 0, sizeof(int), s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.amb_count, 0, 2 * sizeof(int), s)) != cudaSuccess) return e;
     const bool fold = !a.two_term;
     k_centre_prep<<<dim3(a.Cpad, BH), 64, 0, s>>>(a.C, a.cstride, a.ncent, a.ncent_const, a.d, a.Cpad,
                                                   a.two_term ? 1 : 0, fold ? 1 : 0, a.Chi, a.cnp, a.cn, a.hstat);
@@ -722,6 +771,7 @@ cudaError_t launch_assign_fast(const FastAssignArgs &a, cudaStream_t s) {
     p.cand = a.cand;
     p.amb_list = a.amb_list;
     p.amb_count = a.amb_count;
+    p.amb_cap = (int64_t)BH * a.L;
     p.stats = a.stats;
     p.err = a.err;
     p.c_stage = (uint32_t)(a.two_term ? 2 * (a.d / 64) * a.CH * 128 : (a.d / 64) * a.CH * 128 + a.CH * 32);
@@ -736,14 +786,20 @@ cudaError_t launch_assign_fast(const FastAssignArgs &a, cudaStream_t s) {
     else e = a.d == 128 ? launch_mma<128, false>(a, p, grid, s) : launch_mma<64, false>(a, p, grid, s);
     if (e != cudaSuccess) return e;
     // 3. exact rescoring of the uncertain rows
-    if (a.inv)
-        k_assign_resolve<true><<<4 * a.num_sms, 256, 0, s>>>(a.X, a.inv, a.L, a.d, a.C, a.cstride, a.ncent,
-                                                             a.ncent_const, a.cand, a.amb_list, a.amb_count,
-                                                             a.labels, a.stats);
-    else
-        k_assign_resolve<false><<<4 * a.num_sms, 256, 0, s>>>(a.X, a.inv, a.L, a.d, a.C, a.cstride, a.ncent,
-                                                              a.ncent_const, a.cand, a.amb_list, a.amb_count,
-                                                              a.labels, a.stats);
+    if (a.inv) {
+        k_assign_resolve<true><<<4 * a.num_sms, 256, 0, s>>>(a.X, a.inv, a.L, a.d, a.C, a.cstride, a.cand,
+                                                             a.amb_list, a.amb_count, a.labels, a.stats);
+        k_assign_resolve_all<true><<<4 * a.num_sms, 256, 0, s>>>(a.X, a.inv, a.L, a.d, a.C, a.cstride, a.ncent,
+                                                                 a.ncent_const, a.amb_list, p.amb_cap, a.amb_count,
+                                                                 a.labels);
+    } else {
+        k_assign_resolve<false><<<4 * a.num_sms, 256, 0, s>>>(a.X, a.inv, a.L, a.d, a.C, a.cstride, a.cand,
+                                                              a.amb_list, a.amb_count, a.labels, a.stats);
+        k_assign_resolve_all<false><<<4 * a.num_sms, 256, 0, s>>>(a.X, a.inv, a.L, a.d, a.C, a.cstride, a.ncent,
+                                                                  a.ncent_const, a.amb_list, p.amb_cap,
+                                                                  a.amb_count, a.labels);
+    }
+    AC_NOTE_LAUNCH();
     AC_NOTE_LAUNCH();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 4. exact distance to the chosen centre

@@ -341,89 +341,330 @@ cudaError_t launch_counting_sort(const SortArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ member streaming
+// The centre update and the key statistics both walk the members of every
+// cluster in ascending member order.  Members are scattered over the unit, so
+// a producer warp gathers their rows with bulk copies (one row per lane, no
+// tensor map) into a ring of MS_STAGES shared-memory stages of MS_BATCH rows,
+// and d consumer threads (one per dimension) reduce the stages in order.  The
+// grid is persistent: block g takes the clusters g, g + G, ... of the flat
+// (unit, cluster) list, so the ring stays full across cluster boundaries.
+constexpr int MS_BATCH = 32;
+constexpr int MS_STAGES = 4;
+constexpr int MS_BLOCKS_PER_SM = 6;
+enum { MS_FIRST = 1, MS_LAST = 2, MS_EMPTY = 4, MS_END = 8 };
+enum { MS_UPDATE = 0, MS_UPDATE_NORM = 1, MS_STATS = 2 };
+
+struct MsArgs {
+    const bf16 *X; const float *inv; int64_t L;
+    const int *rows;                    // [BH, L] or null (update only)
+    const int *perm; const int *offs; int offs_stride;
+    const int *ncent; int ncent_const;  // clusters c < m(h) hold members
+    int maxc, BH;                       // flat list: f = h * maxc + c
+    float *C; int64_t cstride; const int *coff;  // update: centres written; stats: centres read
+    float *dmin; int *counts; bf16 *kmax; bf16 *kmin; float *sse;  // stats
+    uint32_t *err;
+};
+
+template <int D>
+struct MsLayout {
+    static constexpr uint32_t ROWB = D * 2 + 16;  // padded: per-row 16-byte reads hit distinct banks
+    static constexpr uint32_t STAGE = MS_BATCH * ROWB;
+    static constexpr uint32_t OFF_AUX = MS_STAGES * STAGE;                 // [STAGES][BATCH] inv or token
+    static constexpr uint32_t OFF_META = OFF_AUX + MS_STAGES * MS_BATCH * 4;  // [STAGES] int4
+    static constexpr uint32_t OFF_BAR = OFF_META + MS_STAGES * 16;          // full[STAGES], empty[STAGES]
+    static constexpr uint32_t OFF_CENT = OFF_BAR + 2 * MS_STAGES * 8;       // [D] fp32 (stats, warp 0)
+    static constexpr uint32_t OFF_DM = OFF_CENT + D * 4;                    // [BATCH] fp32 (stats, warp 0)
+    static constexpr uint32_t BYTES = OFF_DM + MS_BATCH * 4;
+};
+
+// The producer's queue of upcoming clusters: lane l examines the cluster
+// fbase + l G of the flat list (one latency for 32 clusters).  An item is a
+// cluster with members; the statistics also emit every other cluster
+// c < maxc (as an MS_EMPTY item), the update skips them (they keep their centre).
+struct MsQueue {
+    int f, beg, end;   // this lane's cluster
+    unsigned mask;     // lanes still holding an item
+    int fbase;
+};
+
+template <int MODE>
+__device__ __forceinline__ void ms_refill(const MsArgs &a, int total, int G, int lane, MsQueue &q) {
+    const int fl = q.fbase + lane * G;
+    bool v = false;
+    int b = 0, e = 0;
+    if (fl < total) {
+        const int h = fl / a.maxc, c = fl - h * a.maxc;
+        const int m = a.ncent ? a.ncent[h] : a.ncent_const;
+        if (c < m) {
+            const int *o = a.offs + (int64_t)h * a.offs_stride + c;
+            b = o[0];
+            e = o[1];
+            v = e > b || MODE == MS_STATS;
+        } else {
+            v = MODE == MS_STATS;
+        }
+    }
+    q.f = fl;
+    q.beg = b;
+    q.end = e;
+    q.mask = __ballot_sync(0xFFFFFFFFu, v);
+    q.fbase += 32 * G;
+}
+
+// Pops the next item into (f, beg, end); false when the block has no more.
+template <int MODE>
+__device__ __forceinline__ bool ms_pop(const MsArgs &a, int total, int G, int lane, MsQueue &q, int &f, int &beg,
+                                       int &end) {
+    while (q.mask == 0u && q.fbase < total) ms_refill<MODE>(a, total, G, lane, q);
+    if (q.mask == 0u) return false;
+    const int src = __ffs(q.mask) - 1;
+    q.mask &= q.mask - 1u;
+    f = __shfl_sync(0xFFFFFFFFu, q.f, src);
+    beg = __shfl_sync(0xFFFFFFFFu, q.beg, src);
+    end = __shfl_sync(0xFFFFFFFFu, q.end, src);
+    return true;
+}
+
+__device__ __forceinline__ void ms_cp16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void ms_cp4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrives on bar once every cp.async this thread issued so far has landed
+// (counted in the barrier's expected arrivals).
+__device__ __forceinline__ void ms_cp_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
+    using LY = MsLayout<D>;
+    extern __shared__ __align__(128) uint8_t ms_sm[];
+    const uint32_t sbase = smem_u32(ms_sm);
+    const uint32_t bar_full = sbase + LY::OFF_BAR, bar_empty = bar_full + MS_STAGES * 8;
+    int4 *meta = reinterpret_cast<int4 *>(ms_sm + LY::OFF_META);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NCW = D / 32;  // consumer warps
+    if (tid == 0) {
+        for (int i = 0; i < MS_STAGES; ++i) {
+            mbar_init(bar_full + 8 * i, 33);  // 32 cp.async arrivals + lane 0's
+            mbar_init(bar_empty + 8 * i, NCW);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int total = a.BH * a.maxc, G = gridDim.x;
+    if (warp == NCW) {
+        // ---------------- producer warp: 16-byte cp.async pieces, PPR lanes per
+        // row, RPI rows per instruction; lane r keeps member r's row index
+        constexpr int PPR = D / 8, RPI = 32 / PPR;
+        MsQueue q{0, 0, 0, 0u, (int)blockIdx.x};
+        int f = 0, beg = 0, end = 0;
+        bool have = ms_pop<MODE>(a, total, G, lane, q, f, beg, end);
+        int j0 = beg;
+        int pn = 0;
+        if (have && lane < min(MS_BATCH, end - j0)) pn = a.perm[(int64_t)(f / a.maxc) * a.L + j0 + lane];
+        uint32_t it = 0;
+        bool ok = true;
+        while (have) {
+            const int cf = f, cbeg = beg, cend = end, cj0 = j0;
+            const int cnt = min(MS_BATCH, cend - cj0);  // 0 for an empty cluster
+            const int p = pn;
+            // advance, and start the next batch's member indices
+            j0 += MS_BATCH;
+            if (j0 >= end) {
+                have = ms_pop<MODE>(a, total, G, lane, q, f, beg, end);
+                j0 = beg;
+            }
+            if (have && lane < min(MS_BATCH, end - j0)) pn = a.perm[(int64_t)(f / a.maxc) * a.L + j0 + lane];
+            const int hh = cf / a.maxc;
+            const int t = (lane < cnt && a.rows) ? a.rows[(int64_t)hh * a.L + p] : p;
+            const uint32_t slot = it % MS_STAGES;
+            if (it >= MS_STAGES && !mbar_wait(bar_empty + 8 * slot, ((it / MS_STAGES) - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            const uint32_t full = bar_full + 8 * slot;
+            if (lane == 0) {
+                const int fl = (cj0 == cbeg ? MS_FIRST : 0) | (cj0 + MS_BATCH >= cend ? MS_LAST : 0) |
+                               (cnt <= 0 ? MS_EMPTY : 0);
+                meta[slot] = make_int4(cf, cnt, fl, cend - cbeg);
+            }
+            const uint32_t dst = sbase + slot * LY::STAGE + (lane % PPR) * 16;
+            const bf16 *src = a.X + (int64_t)hh * a.L * D + (lane % PPR) * 8;
+#pragma unroll
+            for (int i = 0; i < MS_BATCH / RPI; ++i) {
+                const int r = i * RPI + lane / PPR;
+                const int tr = __shfl_sync(0xFFFFFFFFu, t, r);
+                if (r < cnt) ms_cp16(dst + r * LY::ROWB, src + (int64_t)tr * D);
+            }
+            if (lane < cnt) {
+                const uint32_t ad = sbase + LY::OFF_AUX + (slot * MS_BATCH + lane) * 4;
+                if (MODE == MS_UPDATE_NORM) ms_cp4(ad, a.inv + (int64_t)hh * a.L + t);
+                if (MODE == MS_STATS) ms_cp4(ad, a.perm + (int64_t)hh * a.L + cj0 + lane);
+            }
+            ms_cp_arrive(full);
+            if (lane == 0) mbar_arrive(full);  // publishes meta
+            ++it;
+        }
+        // end marker
+        if (ok) {
+            const uint32_t slot = it % MS_STAGES;
+            if (it >= MS_STAGES && !mbar_wait(bar_empty + 8 * slot, ((it / MS_STAGES) - 1) & 1)) ok = false;
+            if (ok) {
+                if (lane == 0) meta[slot] = make_int4(0, 0, MS_END, 0);
+                ms_cp_arrive(bar_full + 8 * slot);
+                if (lane == 0) mbar_arrive(bar_full + 8 * slot);
+            }
+        }
+        if (!ok && lane == 0 && a.err) set_err(a.err, DEV_ERR_TIMEOUT);
+        // the copies of a producer that gave up still land before the block exits
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        return;
+    }
+    // ---------------- consumers: thread k owns dimension k
+    const int k = tid;
+    const float *aux_s = reinterpret_cast<const float *>(ms_sm + LY::OFF_AUX);  // inv (update) or token (stats)
+    float *cent_s = reinterpret_cast<float *>(ms_sm + LY::OFF_CENT);
+    float *dm_s = reinterpret_cast<float *>(ms_sm + LY::OFF_DM);
+    float s = 0.f, mx = 0.f, mn = 0.f, se = 0.f;
+    for (uint32_t it = 0;; ++it) {
+        const uint32_t slot = it % MS_STAGES;
+        if (!mbar_wait(bar_full + 8 * slot, (it / MS_STAGES) & 1)) {
+            if (lane == 0 && a.err) set_err(a.err, DEV_ERR_TIMEOUT);
+            break;
+        }
+        const int4 mt = meta[slot];
+        if (mt.z & MS_END) break;
+        const int h = mt.x / a.maxc, c = mt.x - h * a.maxc, cnt = mt.y;
+        const uint8_t *rs = ms_sm + slot * LY::STAGE;
+        if (MODE != MS_STATS) {
+            if (mt.z & MS_FIRST) s = 0.f;
+            const bf16 *col = reinterpret_cast<const bf16 *>(rs) + k;
+            constexpr int RS = LY::ROWB / 2;  // row stride in elements
+            if (cnt == MS_BATCH) {
+                float v[MS_BATCH];
+#pragma unroll
+                for (int r = 0; r < MS_BATCH; ++r) {
+                    v[r] = bf2f(col[r * RS]);
+                    if (MODE == MS_UPDATE_NORM) v[r] = __fmul_rn(v[r], aux_s[slot * MS_BATCH + r]);
+                }
+#pragma unroll
+                for (int r = 0; r < MS_BATCH; ++r) s = __fadd_rn(s, v[r]);
+            } else {
+                for (int r = 0; r < cnt; ++r) {
+                    float v = bf2f(col[r * RS]);
+                    if (MODE == MS_UPDATE_NORM) v = __fmul_rn(v, aux_s[slot * MS_BATCH + r]);
+                    s = __fadd_rn(s, v);
+                }
+            }
+            if (mt.z & MS_LAST) {
+                const int off = a.coff ? a.coff[h] : 0;
+                a.C[(int64_t)h * a.cstride + (int64_t)(off + c) * D + k] = __fdiv_rn(s, (float)mt.w);
+            }
+        } else {
+            const int64_t ci = (int64_t)h * a.maxc + c;
+            if (mt.z & MS_EMPTY) {
+                a.kmax[ci * D + k] = __float2bfloat16(0.f);
+                a.kmin[ci * D + k] = __float2bfloat16(0.f);
+                if (k == 0) {
+                    a.counts[ci] = 0;
+                    a.sse[ci] = 0.f;
+                }
+            } else {
+                if (mt.z & MS_FIRST) {
+                    if (warp == 0) {  // only warp 0 reads the centre
+                        const float *cg = a.C + (int64_t)h * a.cstride + (int64_t)c * D;
+#pragma unroll
+                        for (int q = 0; q < D / 32; ++q) cent_s[q * 32 + lane] = cg[q * 32 + lane];
+                        __syncwarp();
+                    }
+                    const float v0 = bf2f(reinterpret_cast<const bf16 *>(rs)[k]);
+                    mx = mn = v0;
+                    se = 0.f;
+                }
+                const bf16 *col = reinterpret_cast<const bf16 *>(rs) + k;
+                constexpr int RS = LY::ROWB / 2;
+                for (int r = 0; r < cnt; ++r) {
+                    const float v = bf2f(col[r * RS]);
+                    mx = v > mx ? v : mx;
+                    mn = v < mn ? v : mn;
+                }
+                if (warp == 0) {
+                    // exact squared distance of member row `lane` to the centre,
+                    // summed over dimensions in order
+                    float acc = 0.f;
+                    if (lane < cnt) {
+                        const uint4 *xr = reinterpret_cast<const uint4 *>(rs + lane * LY::ROWB);
+#pragma unroll 4
+                        for (int q = 0; q < D / 8; ++q) {
+                            const uint4 xv = xr[q];
+                            const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                            for (int jj = 0; jj < 8; ++jj) {
+                                const float x = __uint_as_float((jj & 1) ? (w[jj >> 1] & 0xFFFF0000u) : (w[jj >> 1] << 16));
+                                const float tt = __fsub_rn(x, cent_s[q * 8 + jj]);
+                                acc = __fadd_rn(acc, __fmul_rn(tt, tt));
+                            }
+                        }
+                        const int tok = reinterpret_cast<const int *>(aux_s)[slot * MS_BATCH + lane];
+                        a.dmin[(int64_t)h * a.L + tok] = acc;
+                        dm_s[lane] = acc;
+                    }
+                    __syncwarp();
+                    if (lane == 0)
+                        for (int r = 0; r < cnt; ++r) se = __fadd_rn(se, dm_s[r]);
+                    __syncwarp();
+                    if (lane == 0 && (mt.z & MS_LAST)) {
+                        a.sse[ci] = se;
+                        a.counts[ci] = mt.w;
+                    }
+                }
+                if (mt.z & MS_LAST) {
+                    a.kmax[ci * D + k] = __float2bfloat16(mx);
+                    a.kmin[ci * D + k] = __float2bfloat16(mn);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
+    }
+}
+
+template <int D, int MODE>
+cudaError_t launch_member_stream(const MsArgs &a, cudaStream_t s) {
+    const int total = a.BH * a.maxc;
+    if (total <= 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int G = std::min(total, sms * MS_BLOCKS_PER_SM);
+    const size_t smem = MsLayout<D>::BYTES;
+    cudaError_t e = cudaFuncSetAttribute(k_member_stream<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    k_member_stream<D, MODE><<<G, D + 32, smem, s>>>(a);
+    AC_NOTE_LAUNCH();
+    return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_member_stream_d(const MsArgs &a, int d, cudaStream_t s) {
+    return d == 128 ? launch_member_stream<128, MODE>(a, s) : launch_member_stream<64, MODE>(a, s);
+}
+
+// Bulk copies need 16-byte aligned rows.
+inline bool ms_aligned(const bf16 *X) { return (reinterpret_cast<uintptr_t>(X) & 15u) == 0; }
+
 // ------------------------------------------------------------------ update
-// One block per (cluster, unit), one thread per dimension; members summed in
-// ascending order in fp32, then divided by the count.  The members' rows are
-// scattered over the unit, so they are staged in shared memory by cp.async,
-// UPD_BATCH rows per batch and UPD_STAGES batches in flight, while the
-// threads add the rows of the oldest batch in order.
-constexpr int UPD_BATCH = 32;
-constexpr int UPD_STAGES = 4;
-
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-template <bool NORM>
-__global__ void k_update(UpdateArgs a) {
-    extern __shared__ __align__(16) uint8_t upd_sm[];
-    bf16 *rows_s = reinterpret_cast<bf16 *>(upd_sm);                                    // [STAGES][BATCH][d]
-    float *inv_s = reinterpret_cast<float *>(upd_sm + UPD_STAGES * UPD_BATCH * a.d * 2);  // [STAGES][BATCH]
-    const int c = blockIdx.x, h = blockIdx.y, k = threadIdx.x;
-    const int m = a.ncent ? a.ncent[h] : a.ncent_const;
-    if (c >= m) return;
-    const int *offs = a.offs + (int64_t)h * a.offs_stride;
-    const int beg = offs[c], end = offs[c + 1];
-    if (end <= beg) return;  // empty: keep the previous centre
-    const int *perm = a.perm + (int64_t)h * a.L;
-    const int *rows = a.rows ? a.rows + (int64_t)h * a.L : nullptr;
-    const bf16 *X = a.X + (int64_t)h * a.L * a.d;
-    const float *inv = NORM ? a.inv + (int64_t)h * a.L : nullptr;
-    const int nthr = blockDim.x, pieces = a.d / 8;  // 16-byte pieces per row
-    const int nb = (end - beg + UPD_BATCH - 1) / UPD_BATCH;
-    // batch b: members beg + b*BATCH .. into stage b % STAGES
-    auto issue = [&](int b) {
-        if (b < nb) {
-            const int st = b % UPD_STAGES;
-            const int j0 = beg + b * UPD_BATCH;
-            const int cnt = min(UPD_BATCH, end - j0);
-            for (int q = k; q < cnt * pieces; q += nthr) {
-                const int r = q / pieces, part = q % pieces;
-                const int p = perm[j0 + r];
-                const int t = rows ? rows[p] : p;
-                cp_async16(rows_s + ((size_t)st * UPD_BATCH + r) * a.d + part * 8, X + (int64_t)t * a.d + part * 8);
-            }
-            if (NORM && k < cnt) {
-                const int p = perm[j0 + k];
-                inv_s[st * UPD_BATCH + k] = inv[rows ? rows[p] : p];
-            }
-        }
-        cp_async_commit();  // an empty group past the last batch keeps the count uniform
-    };
-#pragma unroll 1
-    for (int b = 0; b < UPD_STAGES - 1; ++b) issue(b);
-    float s = 0.f;
-#pragma unroll 1
-    for (int b = 0; b < nb; ++b) {
-        issue(b + UPD_STAGES - 1);
-        cp_async_wait<UPD_STAGES - 1>();  // batch b has landed (this thread's copies)
-        __syncthreads();                  // ... and every thread's
-        const int st = b % UPD_STAGES;
-        const int cnt = min(UPD_BATCH, end - beg - b * UPD_BATCH);
-        if (k < a.d) {
-            const bf16 *rs = rows_s + (size_t)st * UPD_BATCH * a.d + k;
-            for (int r = 0; r < cnt; ++r) {
-                float v = bf2f(rs[(size_t)r * a.d]);
-                if (NORM) v = __fmul_rn(v, inv_s[st * UPD_BATCH + r]);
-                s = __fadd_rn(s, v);
-            }
-        }
-        __syncthreads();  // stage st is refilled by the next issue
-    }
-    cp_async_wait<0>();
-    if (k < a.d) {
-        const int off = a.coff ? a.coff[h] : 0;
-        a.C[(int64_t)h * a.cstride + (int64_t)(off + c) * a.d + k] = __fdiv_rn(s, (float)(end - beg));
-    }
-}
-
-// The same sums for small clusters (a few dozen members): each thread loads
-// 32 members ahead from global memory, no staging.
+// Centre = mean of the members, summed in ascending member order in fp32 and
+// divided by the count (one thread per dimension).  Normally the members
+// stream through k_member_stream below; k_update_direct serves rows that are
+// not 16-byte aligned.
+// One block per (cluster, unit): each thread loads 32 members ahead from
+// global memory.
 template <bool NORM>
 __global__ void k_update_direct(UpdateArgs a) {
     const int c = blockIdx.x, h = blockIdx.y, k = threadIdx.x;
@@ -468,16 +709,28 @@ __global__ void k_update_direct(UpdateArgs a) {
 }
 
 cudaError_t launch_update(const UpdateArgs &a, cudaStream_t s) {
-    dim3 grid((unsigned)a.max_cent, (unsigned)a.BH);
-    // few, large clusters (queries): staged batches; many small ones: direct
-    if ((int64_t)a.max_cent * 256 <= a.L) {
-        const size_t smem = (size_t)UPD_STAGES * UPD_BATCH * (a.d * 2 + 4);
-        if (a.inv) k_update<true><<<grid, a.d, smem, s>>>(a);
-        else k_update<false><<<grid, a.d, smem, s>>>(a);
-    } else {
-        if (a.inv) k_update_direct<true><<<grid, a.d, 0, s>>>(a);
-        else k_update_direct<false><<<grid, a.d, 0, s>>>(a);
+    if (ms_aligned(a.X) && (a.d == 64 || a.d == 128)) {
+        MsArgs m{};
+        m.X = a.X;
+        m.inv = a.inv;
+        m.L = a.L;
+        m.rows = a.rows;
+        m.perm = a.perm;
+        m.offs = a.offs;
+        m.offs_stride = a.offs_stride;
+        m.ncent = a.ncent;
+        m.ncent_const = a.ncent_const;
+        m.maxc = a.max_cent;
+        m.BH = a.BH;
+        m.C = a.C;
+        m.cstride = a.cstride;
+        m.coff = a.coff;
+        m.err = a.err;
+        return a.inv ? launch_member_stream_d<MS_UPDATE_NORM>(m, a.d, s) : launch_member_stream_d<MS_UPDATE>(m, a.d, s);
     }
+    dim3 grid((unsigned)a.max_cent, (unsigned)a.BH);
+    if (a.inv) k_update_direct<true><<<grid, a.d, 0, s>>>(a);
+    else k_update_direct<false><<<grid, a.d, 0, s>>>(a);
     AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
@@ -670,42 +923,26 @@ cudaError_t launch_remove(const float *dist, const float *tau, int *u_idx, int *
 }
 
 // ------------------------------------------------------------------ Sec. 3.2.1 stats
-// One block per (cluster, unit), one thread per dimension: count, exact
-// per-dimension max/min, and (thread 0) SSE over members in ascending order.
+// Per key cluster: count, exact per-dimension max/min, and the SSE: the exact
+// squared distance of every member to the centre (summed over dimensions in
+// order, written to dmin as well), summed over the members in ascending order.
+// Normally k_member_stream<MS_STATS> computes them; this one-block-per-cluster
+// kernel serves rows that are not 16-byte aligned.
 __global__ void k_key_stats(StatsArgs a) {
     const int c = blockIdx.x, h = blockIdx.y, k = threadIdx.x;
     const int nk = a.n_k[h];
     const int64_t ci = (int64_t)h * a.Ccap + c;
-    if (c >= nk) {
-        if (k == 0) {
-            a.counts[ci] = 0;
-            a.sse[ci] = 0.f;
-        }
-        a.kmax[ci * a.d + k] = __float2bfloat16(0.f);
-        a.kmin[ci * a.d + k] = __float2bfloat16(0.f);
-        return;
+    int beg = 0, end = 0;
+    if (c < nk) {
+        const int *offs = a.offs + (int64_t)h * a.offs_stride;
+        beg = offs[c];
+        end = offs[c + 1];
     }
-    const int *offs = a.offs + (int64_t)h * a.offs_stride;
-    const int beg = offs[c], end = offs[c + 1];
     const int *perm = a.perm + (int64_t)h * a.L;
     const bf16 *K = a.K + (int64_t)h * a.L * a.d;
-    // 16 members in flight per step (scattered rows); max and min are exact
-    // in any order, the SSE is summed in member order
-    constexpr int U = 16;
     float mx = 0.f, mn = 0.f;  // an empty cluster keeps 0 (and count 0)
     if (end > beg) mx = mn = bf2f(K[(int64_t)perm[beg] * a.d + k]);
-    int j = beg + 1;
-    for (; j + U <= end; j += U) {
-        float v[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) v[u] = bf2f(K[(int64_t)perm[j + u] * a.d + k]);
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            mx = v[u] > mx ? v[u] : mx;
-            mn = v[u] < mn ? v[u] : mn;
-        }
-    }
-    for (; j < end; ++j) {
+    for (int j = beg + 1; j < end; ++j) {
         const float v = bf2f(K[(int64_t)perm[j] * a.d + k]);
         mx = v > mx ? v : mx;
         mn = v < mn ? v : mn;
@@ -713,17 +950,19 @@ __global__ void k_key_stats(StatsArgs a) {
     a.kmax[ci * a.d + k] = __float2bfloat16(mx);
     a.kmin[ci * a.d + k] = __float2bfloat16(mn);
     if (k == 0) {
+        const float *cc = a.C + (int64_t)h * a.cstride + (int64_t)c * a.d;
         float se = 0.f;
-        const float *dm = a.dmin + (int64_t)h * a.L;
-        int i = beg;
-        for (; i + U <= end; i += U) {
-            float v[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) v[u] = dm[perm[i + u]];
-#pragma unroll
-            for (int u = 0; u < U; ++u) se = __fadd_rn(se, v[u]);
+        for (int j = beg; j < end; ++j) {
+            const int t = perm[j];
+            const bf16 *x = K + (int64_t)t * a.d;
+            float acc = 0.f;
+            for (int q = 0; q < a.d; ++q) {
+                const float tt = __fsub_rn(bf2f(x[q]), cc[q]);
+                acc = __fadd_rn(acc, __fmul_rn(tt, tt));
+            }
+            a.dmin[(int64_t)h * a.L + t] = acc;
+            se = __fadd_rn(se, acc);
         }
-        for (; i < end; ++i) se = __fadd_rn(se, dm[perm[i]]);
         a.sse[ci] = se;
         a.counts[ci] = end - beg;
     }
@@ -741,9 +980,31 @@ __global__ void k_head_comp(StatsArgs a) {
 }
 
 cudaError_t launch_key_stats(const StatsArgs &a, cudaStream_t s) {
-    k_key_stats<<<dim3(a.Ccap, a.BH), a.d, 0, s>>>(a);
-    AC_NOTE_LAUNCH();
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    if (ms_aligned(a.K) && (a.d == 64 || a.d == 128)) {
+        MsArgs m{};
+        m.X = a.K;
+        m.L = a.L;
+        m.perm = a.perm;
+        m.offs = a.offs;
+        m.offs_stride = a.offs_stride;
+        m.ncent = a.n_k;
+        m.maxc = a.Ccap;
+        m.BH = a.BH;
+        m.C = const_cast<float *>(a.C);
+        m.cstride = a.cstride;
+        m.dmin = a.dmin;
+        m.counts = a.counts;
+        m.kmax = a.kmax;
+        m.kmin = a.kmin;
+        m.sse = a.sse;
+        m.err = a.err;
+        e = launch_member_stream_d<MS_STATS>(m, a.d, s);
+    } else {
+        k_key_stats<<<dim3(a.Ccap, a.BH), a.d, 0, s>>>(a);
+        AC_NOTE_LAUNCH();
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
     k_head_comp<<<(a.BH + 127) / 128, 128, 0, s>>>(a);
     AC_NOTE_LAUNCH();
