@@ -344,14 +344,18 @@ cudaError_t launch_counting_sort(const SortArgs &a, cudaStream_t s) {
 // ------------------------------------------------------------------ member streaming
 // The centre update and the key statistics both walk the members of every
 // cluster in ascending member order.  Members are scattered over the unit, so
-// a producer warp gathers their rows with bulk copies (one row per lane, no
-// tensor map) into a ring of MS_STAGES shared-memory stages of MS_BATCH rows,
-// and d consumer threads (one per dimension) reduce the stages in order.  The
-// grid is persistent: block g takes the clusters g, g + G, ... of the flat
-// (unit, cluster) list, so the ring stays full across cluster boundaries.
-constexpr int MS_BATCH = 32;
+// a producer warp gathers their rows (16-byte cp.async pieces, completion on
+// an mbarrier) into a ring of MS_STAGES shared-memory stages of BATCH rows,
+// and d consumer threads (one per dimension) reduce the stages in order.
+// The grid is persistent: block g takes a contiguous range of the flat
+// (unit, cluster) list holding about 1/G of the work (members plus MS_W per
+// cluster for its partly filled last batch), so the member indices it reads
+// (perm) are contiguous too; the producer fetches them in windows of MS_WIN,
+// three windows ahead.
 constexpr int MS_STAGES = 4;
-constexpr int MS_BLOCKS_PER_SM = 6;
+constexpr int MS_WIN = 256;   // member indices per window
+constexpr int MS_WSLOTS = 4;  // window ring
+constexpr int MS_W = 16;      // work of one cluster beyond its members, in rows
 enum { MS_FIRST = 1, MS_LAST = 2, MS_EMPTY = 4, MS_END = 8 };
 enum { MS_UPDATE = 0, MS_UPDATE_NORM = 1, MS_STATS = 2 };
 
@@ -362,38 +366,89 @@ struct MsArgs {
     const int *ncent; int ncent_const;  // clusters c < m(h) hold members
     int maxc, BH;                       // flat list: f = h * maxc + c
     float *C; int64_t cstride; const int *coff;  // update: centres written; stats: centres read
-    float *dmin; int *counts; bf16 *kmax; bf16 *kmin; float *sse;  // stats
+    float *dmin; bf16 *kmax; bf16 *kmin;         // stats
     uint32_t *err;
 };
 
-template <int D>
+template <int D, int MODE>
 struct MsLayout {
-    static constexpr uint32_t ROWB = D * 2 + 16;  // padded: per-row 16-byte reads hit distinct banks
-    static constexpr uint32_t STAGE = MS_BATCH * ROWB;
-    static constexpr uint32_t OFF_AUX = MS_STAGES * STAGE;                 // [STAGES][BATCH] inv or token
-    static constexpr uint32_t OFF_META = OFF_AUX + MS_STAGES * MS_BATCH * 4;  // [STAGES] int4
+    // the query update takes 64-row stages: its clusters are few and large
+    static constexpr int BATCH = MODE == MS_UPDATE_NORM ? 64 : 32;
+    // stats rows are padded: per-row 16-byte reads then hit distinct banks
+    static constexpr uint32_t ROWB = MODE == MS_STATS ? D * 2 + 16 : D * 2;
+    static constexpr uint32_t STAGE = BATCH * ROWB;
+    static constexpr uint32_t OFF_AUX = MS_STAGES * STAGE;                   // [STAGES][BATCH] inv or token
+    static constexpr uint32_t OFF_META = OFF_AUX + MS_STAGES * BATCH * 4;   // [STAGES] int4
     static constexpr uint32_t OFF_BAR = OFF_META + MS_STAGES * 16;          // full[STAGES], empty[STAGES]
-    static constexpr uint32_t OFF_CENT = OFF_BAR + 2 * MS_STAGES * 8;       // [D] fp32 (stats, warp 0)
-    static constexpr uint32_t OFF_DM = OFF_CENT + D * 4;                    // [BATCH] fp32 (stats, warp 0)
-    static constexpr uint32_t BYTES = OFF_DM + MS_BATCH * 4;
+    static constexpr uint32_t OFF_CENT = OFF_BAR + 2 * MS_STAGES * 8;       // [STAGES][D] fp32 centre (stats)
+    static constexpr uint32_t OFF_WDESC = OFF_CENT + (MODE == MS_STATS ? MS_STAGES * D * 4 : 0);
+    static constexpr uint32_t OFF_WIN = OFF_WDESC + MS_WSLOTS * 16;         // [WSLOTS][WIN] int (producer)
+    static constexpr uint32_t BYTES = OFF_WIN + MS_WSLOTS * MS_WIN * 4;
 };
 
-// The producer's queue of upcoming clusters: lane l examines the cluster
-// fbase + l G of the flat list (one latency for 32 clusters).  An item is a
-// cluster with members; the statistics also emit every other cluster
-// c < maxc (as an MS_EMPTY item), the update skips them (they keep their centre).
+// Work position of flat cluster f: h S + (start of cluster c + MS_W c) with
+// S = L + MS_W maxc, or (h + 1) S for a slot c >= m(h).  Non-decreasing in f.
+__device__ __forceinline__ int64_t ms_key(const MsArgs &a, int f) {
+    const int h = f / a.maxc, c = f - h * a.maxc;
+    const int m = a.ncent ? a.ncent[h] : a.ncent_const;
+    const int64_t S = a.L + (int64_t)MS_W * a.maxc;
+    return (int64_t)h * S + (c < m ? a.offs[(int64_t)h * a.offs_stride + c] + (int64_t)MS_W * c : S);
+}
+
+// Block g's range [fs, fe): fs(g) = the first f whose key reaches g M / G
+// (M = BH S), found by a 16-ary search per half warp (lanes 0-15: g,
+// lanes 16-31: g + 1).  Every cluster lands in exactly one range.
+__device__ __forceinline__ void ms_range(const MsArgs &a, int total, int G, int lane, int &fs, int &fe) {
+    const int half = lane >> 4, hl = lane & 15;
+    const int g = (int)blockIdx.x + half;
+    const int64_t S = a.L + (int64_t)MS_W * a.maxc;
+    const int64_t T = (int64_t)a.BH * S * g / G;
+    int lo = total, hi = total;  // the answer lies in [lo, hi]
+    if (g < G) {
+        const int64_t h0 = min(T / S, (int64_t)a.BH - 1);
+        lo = (int)max((int64_t)0, (h0 - 1) * a.maxc);
+        hi = (int)min((int64_t)total, (h0 + 1) * a.maxc);
+    }
+    while (__any_sync(0xFFFFFFFFu, hi > lo)) {
+        const int step = hi > lo ? (hi - lo + 15) / 16 : 1;
+        const int fp = lo + hl * step;
+        const bool ge = hi <= lo || fp >= hi || ms_key(a, fp) >= T;
+        const unsigned b = (__ballot_sync(0xFFFFFFFFu, ge) >> (16 * half)) & 0xFFFFu;
+        if (hi > lo) {
+            if (b == 0u) {
+                lo = lo + 15 * step + 1;
+            } else {
+                const int first = __ffs(b) - 1;
+                if (first == 0) {
+                    hi = lo;
+                } else {
+                    hi = lo + first * step;
+                    lo = lo + (first - 1) * step + 1;
+                }
+            }
+        }
+    }
+    fs = __shfl_sync(0xFFFFFFFFu, lo, 0);
+    fe = __shfl_sync(0xFFFFFFFFu, lo, 16);
+}
+
+// The producer's queue of upcoming clusters: lane l examines cluster fbase + l
+// (one latency for 32 clusters).  An item is a cluster with members; the
+// statistics also emit the empty clusters c < m(h) (as MS_EMPTY items; the
+// slots c >= m(h) are zeroed apart), the update skips them (they keep their
+// centre).
 struct MsQueue {
-    int f, beg, end;   // this lane's cluster
-    unsigned mask;     // lanes still holding an item
-    int fbase;
+    int f, beg, end;  // this lane's cluster
+    unsigned mask;    // lanes still holding an item
+    int fbase, fend;
 };
 
 template <int MODE>
-__device__ __forceinline__ void ms_refill(const MsArgs &a, int total, int G, int lane, MsQueue &q) {
-    const int fl = q.fbase + lane * G;
+__device__ __forceinline__ void ms_refill(const MsArgs &a, int lane, MsQueue &q) {
+    const int fl = q.fbase + lane;
     bool v = false;
     int b = 0, e = 0;
-    if (fl < total) {
+    if (fl < q.fend) {
         const int h = fl / a.maxc, c = fl - h * a.maxc;
         const int m = a.ncent ? a.ncent[h] : a.ncent_const;
         if (c < m) {
@@ -401,22 +456,18 @@ __device__ __forceinline__ void ms_refill(const MsArgs &a, int total, int G, int
             b = o[0];
             e = o[1];
             v = e > b || MODE == MS_STATS;
-        } else {
-            v = MODE == MS_STATS;
         }
     }
     q.f = fl;
     q.beg = b;
     q.end = e;
     q.mask = __ballot_sync(0xFFFFFFFFu, v);
-    q.fbase += 32 * G;
+    q.fbase += 32;
 }
 
-// Pops the next item into (f, beg, end); false when the block has no more.
 template <int MODE>
-__device__ __forceinline__ bool ms_pop(const MsArgs &a, int total, int G, int lane, MsQueue &q, int &f, int &beg,
-                                       int &end) {
-    while (q.mask == 0u && q.fbase < total) ms_refill<MODE>(a, total, G, lane, q);
+__device__ __forceinline__ bool ms_pop(const MsArgs &a, int lane, MsQueue &q, int &f, int &beg, int &end) {
+    while (q.mask == 0u && q.fbase < q.fend) ms_refill<MODE>(a, lane, q);
     if (q.mask == 0u) return false;
     const int src = __ffs(q.mask) - 1;
     q.mask &= q.mask - 1u;
@@ -432,15 +483,45 @@ __device__ __forceinline__ void ms_cp16(uint32_t dst, const void *src) {
 __device__ __forceinline__ void ms_cp4(uint32_t dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void ms_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void ms_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
 // Arrives on bar once every cp.async this thread issued so far has landed
 // (counted in the barrier's expected arrivals).
 __device__ __forceinline__ void ms_cp_arrive(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// Exact squared distance of a bf16 row (in shared memory) to an fp32 centre
+// (in shared memory): per dimension the difference and its square are
+// rounded to fp32, then added over the dimensions in order.
+template <int D>
+__device__ __forceinline__ float ms_sqdist(const uint8_t *row, const float *cent) {
+    const uint4 *xr = reinterpret_cast<const uint4 *>(row);
+    const float4 *c4 = reinterpret_cast<const float4 *>(cent);
+    float acc = 0.f;
+#pragma unroll
+    for (int q = 0; q < D / 8; ++q) {
+        const uint4 xv = xr[q];
+        const float4 ca = c4[2 * q], cb = c4[2 * q + 1];
+        const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+        const float cc[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr) {
+            const uint64_t x2 = f2_pack(__uint_as_float(w[pr] << 16), __uint_as_float(w[pr] & 0xFFFF0000u));
+            const uint64_t d2 = f2_sub(x2, f2_pack(cc[2 * pr], cc[2 * pr + 1]));
+            float s0, s1;
+            f2_unpack(f2_mul(d2, d2), s0, s1);
+            acc = __fadd_rn(acc, s0);
+            acc = __fadd_rn(acc, s1);
+        }
+    }
+    return acc;
+}
+
 template <int D, int MODE>
 __global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
-    using LY = MsLayout<D>;
+    using LY = MsLayout<D, MODE>;
+    constexpr int BATCH = LY::BATCH;
     extern __shared__ __align__(128) uint8_t ms_sm[];
     const uint32_t sbase = smem_u32(ms_sm);
     const uint32_t bar_full = sbase + LY::OFF_BAR, bar_empty = bar_full + MS_STAGES * 8;
@@ -456,58 +537,110 @@ __global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
     }
     __syncthreads();
     const int total = a.BH * a.maxc, G = gridDim.x;
+    if (MODE == MS_STATS && warp < NCW) {
+        // slots without a cluster (c >= m(h)): bounds 0
+        for (int f = blockIdx.x; f < total; f += G) {
+            const int h = f / a.maxc, c = f - h * a.maxc;
+            if (c < a.ncent[h]) continue;
+            a.kmax[(int64_t)f * D + tid] = __float2bfloat16(0.f);
+            a.kmin[(int64_t)f * D + tid] = __float2bfloat16(0.f);
+        }
+    }
     if (warp == NCW) {
-        // ---------------- producer warp: 16-byte cp.async pieces, PPR lanes per
-        // row, RPI rows per instruction; lane r keeps member r's row index
+        // ---------------- producer warp: 16-byte pieces, PPR lanes per row,
+        // RPI rows per instruction
         constexpr int PPR = D / 8, RPI = 32 / PPR;
-        MsQueue q{0, 0, 0, 0u, (int)blockIdx.x};
-        int f = 0, beg = 0, end = 0;
-        bool have = ms_pop<MODE>(a, total, G, lane, q, f, beg, end);
-        int j0 = beg;
-        int pn = 0;
-        if (have && lane < min(MS_BATCH, end - j0)) pn = a.perm[(int64_t)(f / a.maxc) * a.L + j0 + lane];
+        int4 *wdesc = reinterpret_cast<int4 *>(ms_sm + LY::OFF_WDESC);
+        const int *win = reinterpret_cast<const int *>(ms_sm + LY::OFF_WIN);
+        const uint32_t win_s = sbase + LY::OFF_WIN;
+        MsQueue q{0, 0, 0, 0u, 0, 0};
+        ms_range(a, total, G, lane, q.fbase, q.fend);
+        // window frontier: (f, beg, end) and the window start ws
+        int ff = 0, fbeg = 0, fend = 0, ws = 0;
+        bool fhave = ms_pop<MODE>(a, lane, q, ff, fbeg, fend);
+        ws = fbeg;
+        // window n -> slot n % WSLOTS: descriptor and member indices, one commit group
+        auto issue_window = [&](uint32_t n) {
+            const uint32_t sl = n % MS_WSLOTS;
+            if (lane == 0) wdesc[sl] = fhave ? make_int4(ff, fbeg, fend, ws) : make_int4(-1, 0, 0, 0);
+            if (fhave) {
+                const int *src = a.perm + (int64_t)(ff / a.maxc) * a.L;
+#pragma unroll
+                for (int i = 0; i < MS_WIN / 32; ++i) {
+                    const int pos = ws + 32 * i + lane;
+                    if (pos < fend) ms_cp4(win_s + (sl * MS_WIN + 32 * i + lane) * 4, src + pos);
+                }
+                // advance the frontier
+                if (ws + MS_WIN < fend) {
+                    ws += MS_WIN;
+                } else {
+                    fhave = ms_pop<MODE>(a, lane, q, ff, fbeg, fend);
+                    ws = fbeg;
+                }
+            }
+            ms_commit();
+        };
+        issue_window(0);
+        issue_window(1);
+        issue_window(2);
         uint32_t it = 0;
         bool ok = true;
-        while (have) {
-            const int cf = f, cbeg = beg, cend = end, cj0 = j0;
-            const int cnt = min(MS_BATCH, cend - cj0);  // 0 for an empty cluster
-            const int p = pn;
-            // advance, and start the next batch's member indices
-            j0 += MS_BATCH;
-            if (j0 >= end) {
-                have = ms_pop<MODE>(a, total, G, lane, q, f, beg, end);
-                j0 = beg;
-            }
-            if (have && lane < min(MS_BATCH, end - j0)) pn = a.perm[(int64_t)(f / a.maxc) * a.L + j0 + lane];
-            const int hh = cf / a.maxc;
-            const int t = (lane < cnt && a.rows) ? a.rows[(int64_t)hh * a.L + p] : p;
-            const uint32_t slot = it % MS_STAGES;
-            if (it >= MS_STAGES && !mbar_wait(bar_empty + 8 * slot, ((it / MS_STAGES) - 1) & 1)) {
-                ok = false;
-                break;
-            }
-            const uint32_t full = bar_full + 8 * slot;
-            if (lane == 0) {
-                const int fl = (cj0 == cbeg ? MS_FIRST : 0) | (cj0 + MS_BATCH >= cend ? MS_LAST : 0) |
-                               (cnt <= 0 ? MS_EMPTY : 0);
-                meta[slot] = make_int4(cf, cnt, fl, cend - cbeg);
-            }
-            const uint32_t dst = sbase + slot * LY::STAGE + (lane % PPR) * 16;
+        for (uint32_t w = 0; ok; ++w) {
+            issue_window(w + 3);
+            ms_wait2();  // window w has landed (each lane reads the entries it loaded)
+            __syncwarp();
+            const int4 dw = wdesc[w % MS_WSLOTS];
+            if (dw.x < 0) break;
+            const int hh = dw.x / a.maxc;
+            const int *wc = win + (w % MS_WSLOTS) * MS_WIN;
             const bf16 *src = a.X + (int64_t)hh * a.L * D + (lane % PPR) * 8;
+            for (int i = 0; i < MS_WIN / BATCH; ++i) {
+                const int j0 = dw.w + BATCH * i;
+                if (j0 >= dw.z && !(i == 0 && dw.y == dw.z)) break;
+                const int cnt = min(BATCH, dw.z - j0);  // 0 for an empty cluster
+                // member indices of rows lane and lane + 32 of the batch
+                int t0 = 0, t1 = 0;
+                if (lane < cnt) t0 = wc[BATCH * i + lane];
+                if (BATCH > 32 && lane + 32 < cnt) t1 = wc[BATCH * i + 32 + lane];
+                if (a.rows) {
+                    if (lane < cnt) t0 = a.rows[(int64_t)hh * a.L + t0];
+                    if (BATCH > 32 && lane + 32 < cnt) t1 = a.rows[(int64_t)hh * a.L + t1];
+                }
+                const uint32_t slot = it % MS_STAGES;
+                if (it >= MS_STAGES && !mbar_wait(bar_empty + 8 * slot, ((it / MS_STAGES) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t full = bar_full + 8 * slot;
+                if (lane == 0) {
+                    const int fl = (j0 == dw.y ? MS_FIRST : 0) | (j0 + BATCH >= dw.z ? MS_LAST : 0) |
+                                   (cnt <= 0 ? MS_EMPTY : 0);
+                    meta[slot] = make_int4(dw.x, cnt, fl, dw.z - dw.y);
+                }
+                const uint32_t dst = sbase + slot * LY::STAGE + (lane % PPR) * 16;
 #pragma unroll
-            for (int i = 0; i < MS_BATCH / RPI; ++i) {
-                const int r = i * RPI + lane / PPR;
-                const int tr = __shfl_sync(0xFFFFFFFFu, t, r);
-                if (r < cnt) ms_cp16(dst + r * LY::ROWB, src + (int64_t)tr * D);
+                for (int r0 = 0; r0 < BATCH; r0 += RPI) {
+                    // the RPI rows of one instruction lie in the same half (r0 is a multiple of RPI)
+                    const int r = r0 + lane / PPR;
+                    const int tr = __shfl_sync(0xFFFFFFFFu, r0 < 32 ? t0 : t1, r & 31);
+                    if (r < cnt) ms_cp16(dst + r * LY::ROWB, src + (int64_t)tr * D);
+                }
+                const uint32_t ad = sbase + LY::OFF_AUX + (slot * BATCH + lane) * 4;
+                if (lane < cnt) {
+                    if (MODE == MS_UPDATE_NORM) ms_cp4(ad, a.inv + (int64_t)hh * a.L + t0);
+                    if (MODE == MS_STATS) ms_cp4(ad, a.perm + (int64_t)hh * a.L + j0 + lane);
+                }
+                if (MODE == MS_UPDATE_NORM && BATCH > 32 && lane + 32 < cnt)
+                    ms_cp4(ad + 128, a.inv + (int64_t)hh * a.L + t1);
+                if (MODE == MS_STATS && cnt > 0 && lane < D / 4) {  // the centre, with every batch
+                    const int c = dw.x - hh * a.maxc;
+                    ms_cp16(sbase + LY::OFF_CENT + slot * D * 4 + lane * 16,
+                            a.C + (int64_t)hh * a.cstride + (int64_t)c * D + lane * 4);
+                }
+                ms_cp_arrive(full);
+                if (lane == 0) mbar_arrive(full);  // publishes meta
+                ++it;
             }
-            if (lane < cnt) {
-                const uint32_t ad = sbase + LY::OFF_AUX + (slot * MS_BATCH + lane) * 4;
-                if (MODE == MS_UPDATE_NORM) ms_cp4(ad, a.inv + (int64_t)hh * a.L + t);
-                if (MODE == MS_STATS) ms_cp4(ad, a.perm + (int64_t)hh * a.L + cj0 + lane);
-            }
-            ms_cp_arrive(full);
-            if (lane == 0) mbar_arrive(full);  // publishes meta
-            ++it;
         }
         // end marker
         if (ok) {
@@ -520,16 +653,16 @@ __global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
             }
         }
         if (!ok && lane == 0 && a.err) set_err(a.err, DEV_ERR_TIMEOUT);
-        // the copies of a producer that gave up still land before the block exits
+        // every copy this warp issued lands before the block exits
         asm volatile("cp.async.wait_all;" ::: "memory");
         return;
     }
     // ---------------- consumers: thread k owns dimension k
     const int k = tid;
     const float *aux_s = reinterpret_cast<const float *>(ms_sm + LY::OFF_AUX);  // inv (update) or token (stats)
-    float *cent_s = reinterpret_cast<float *>(ms_sm + LY::OFF_CENT);
-    float *dm_s = reinterpret_cast<float *>(ms_sm + LY::OFF_DM);
-    float s = 0.f, mx = 0.f, mn = 0.f, se = 0.f;
+    const float *cent_s = reinterpret_cast<const float *>(ms_sm + LY::OFF_CENT);
+    constexpr int RS = LY::ROWB / 2;  // row stride in elements
+    float s = 0.f, mx = 0.f, mn = 0.f;
     for (uint32_t it = 0;; ++it) {
         const uint32_t slot = it % MS_STAGES;
         if (!mbar_wait(bar_full + 8 * slot, (it / MS_STAGES) & 1)) {
@@ -540,25 +673,25 @@ __global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
         if (mt.z & MS_END) break;
         const int h = mt.x / a.maxc, c = mt.x - h * a.maxc, cnt = mt.y;
         const uint8_t *rs = ms_sm + slot * LY::STAGE;
+        const bf16 *col = reinterpret_cast<const bf16 *>(rs) + k;
         if (MODE != MS_STATS) {
             if (mt.z & MS_FIRST) s = 0.f;
-            const bf16 *col = reinterpret_cast<const bf16 *>(rs) + k;
-            constexpr int RS = LY::ROWB / 2;  // row stride in elements
-            if (cnt == MS_BATCH) {
-                float v[MS_BATCH];
+            const float *inv_s = aux_s + slot * BATCH;
+            int r = 0;
+            for (; r + 32 <= cnt; r += 32) {
+                float v[32];
 #pragma unroll
-                for (int r = 0; r < MS_BATCH; ++r) {
-                    v[r] = bf2f(col[r * RS]);
-                    if (MODE == MS_UPDATE_NORM) v[r] = __fmul_rn(v[r], aux_s[slot * MS_BATCH + r]);
+                for (int u = 0; u < 32; ++u) {
+                    v[u] = bf2f(col[(r + u) * RS]);
+                    if (MODE == MS_UPDATE_NORM) v[u] = __fmul_rn(v[u], inv_s[r + u]);
                 }
 #pragma unroll
-                for (int r = 0; r < MS_BATCH; ++r) s = __fadd_rn(s, v[r]);
-            } else {
-                for (int r = 0; r < cnt; ++r) {
-                    float v = bf2f(col[r * RS]);
-                    if (MODE == MS_UPDATE_NORM) v = __fmul_rn(v, aux_s[slot * MS_BATCH + r]);
-                    s = __fadd_rn(s, v);
-                }
+                for (int u = 0; u < 32; ++u) s = __fadd_rn(s, v[u]);
+            }
+            for (; r < cnt; ++r) {
+                float v = bf2f(col[r * RS]);
+                if (MODE == MS_UPDATE_NORM) v = __fmul_rn(v, inv_s[r]);
+                s = __fadd_rn(s, v);
             }
             if (mt.z & MS_LAST) {
                 const int off = a.coff ? a.coff[h] : 0;
@@ -567,65 +700,24 @@ __global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
         } else {
             const int64_t ci = (int64_t)h * a.maxc + c;
             if (mt.z & MS_EMPTY) {
-                a.kmax[ci * D + k] = __float2bfloat16(0.f);
-                a.kmin[ci * D + k] = __float2bfloat16(0.f);
-                if (k == 0) {
-                    a.counts[ci] = 0;
-                    a.sse[ci] = 0.f;
-                }
+                mx = mn = 0.f;
             } else {
-                if (mt.z & MS_FIRST) {
-                    if (warp == 0) {  // only warp 0 reads the centre
-                        const float *cg = a.C + (int64_t)h * a.cstride + (int64_t)c * D;
-#pragma unroll
-                        for (int q = 0; q < D / 32; ++q) cent_s[q * 32 + lane] = cg[q * 32 + lane];
-                        __syncwarp();
-                    }
-                    const float v0 = bf2f(reinterpret_cast<const bf16 *>(rs)[k]);
-                    mx = mn = v0;
-                    se = 0.f;
-                }
-                const bf16 *col = reinterpret_cast<const bf16 *>(rs) + k;
-                constexpr int RS = LY::ROWB / 2;
+                if (mt.z & MS_FIRST) mx = mn = bf2f(col[0]);
                 for (int r = 0; r < cnt; ++r) {
                     const float v = bf2f(col[r * RS]);
                     mx = v > mx ? v : mx;
                     mn = v < mn ? v : mn;
                 }
-                if (warp == 0) {
-                    // exact squared distance of member row `lane` to the centre,
-                    // summed over dimensions in order
-                    float acc = 0.f;
-                    if (lane < cnt) {
-                        const uint4 *xr = reinterpret_cast<const uint4 *>(rs + lane * LY::ROWB);
-#pragma unroll 4
-                        for (int q = 0; q < D / 8; ++q) {
-                            const uint4 xv = xr[q];
-                            const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                            for (int jj = 0; jj < 8; ++jj) {
-                                const float x = __uint_as_float((jj & 1) ? (w[jj >> 1] & 0xFFFF0000u) : (w[jj >> 1] << 16));
-                                const float tt = __fsub_rn(x, cent_s[q * 8 + jj]);
-                                acc = __fadd_rn(acc, __fmul_rn(tt, tt));
-                            }
-                        }
-                        const int tok = reinterpret_cast<const int *>(aux_s)[slot * MS_BATCH + lane];
-                        a.dmin[(int64_t)h * a.L + tok] = acc;
-                        dm_s[lane] = acc;
-                    }
-                    __syncwarp();
-                    if (lane == 0)
-                        for (int r = 0; r < cnt; ++r) se = __fadd_rn(se, dm_s[r]);
-                    __syncwarp();
-                    if (lane == 0 && (mt.z & MS_LAST)) {
-                        a.sse[ci] = se;
-                        a.counts[ci] = mt.w;
-                    }
+                // the batches take turns among the consumer warps for the
+                // exact distances: member row `lane` to the centre
+                if (warp == (int)(it % NCW) && lane < cnt) {
+                    const int tok = reinterpret_cast<const int *>(aux_s)[slot * BATCH + lane];
+                    a.dmin[(int64_t)h * a.L + tok] = ms_sqdist<D>(rs + lane * LY::ROWB, cent_s + slot * D);
                 }
-                if (mt.z & MS_LAST) {
-                    a.kmax[ci * D + k] = __float2bfloat16(mx);
-                    a.kmin[ci * D + k] = __float2bfloat16(mn);
-                }
+            }
+            if (mt.z & MS_LAST) {
+                a.kmax[ci * D + k] = __float2bfloat16(mx);
+                a.kmin[ci * D + k] = __float2bfloat16(mn);
             }
         }
         __syncwarp();
@@ -640,8 +732,10 @@ cudaError_t launch_member_stream(const MsArgs &a, cudaStream_t s) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int G = std::min(total, sms * MS_BLOCKS_PER_SM);
-    const size_t smem = MsLayout<D>::BYTES;
+    const size_t smem = MsLayout<D, MODE>::BYTES;
+    // resident blocks per SM: shared memory (about 220 KB usable), at most 5
+    const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(5, (220u << 10) / (smem + 1024)));
+    const int G = std::min(total, sms * per_sm);
     cudaError_t e = cudaFuncSetAttribute(k_member_stream<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
@@ -653,6 +747,36 @@ cudaError_t launch_member_stream(const MsArgs &a, cudaStream_t s) {
 template <int MODE>
 cudaError_t launch_member_stream_d(const MsArgs &a, int d, cudaStream_t s) {
     return d == 128 ? launch_member_stream<128, MODE>(a, s) : launch_member_stream<64, MODE>(a, s);
+}
+
+// Per key cluster: count and SSE = the members' exact distances (dmin, from
+// the statistics pass) summed in ascending member order; 0 for the slots
+// c >= n_k.  One thread per cluster.
+__global__ void k_cluster_sse(const int *__restrict__ perm, const int *__restrict__ offs, int offs_stride,
+                              const float *__restrict__ dmin, const int *__restrict__ n_k, int Ccap, int64_t L,
+                              int BH, int *__restrict__ counts, float *__restrict__ sse) {
+    const int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (f >= (int64_t)BH * Ccap) return;
+    const int h = (int)(f / Ccap), c = (int)(f - (int64_t)h * Ccap);
+    int beg = 0, end = 0;
+    if (c < n_k[h]) {
+        beg = offs[(int64_t)h * offs_stride + c];
+        end = offs[(int64_t)h * offs_stride + c + 1];
+    }
+    const int *pm = perm + (int64_t)h * L;
+    const float *dm = dmin + (int64_t)h * L;
+    float se = 0.f;
+    int j = beg;
+    for (; j + 8 <= end; j += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = dm[pm[j + u]];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) se = __fadd_rn(se, v[u]);
+    }
+    for (; j < end; ++j) se = __fadd_rn(se, dm[pm[j]]);
+    sse[f] = se;
+    counts[f] = end - beg;
 }
 
 // Bulk copies need 16-byte aligned rows.
@@ -994,12 +1118,16 @@ cudaError_t launch_key_stats(const StatsArgs &a, cudaStream_t s) {
         m.C = const_cast<float *>(a.C);
         m.cstride = a.cstride;
         m.dmin = a.dmin;
-        m.counts = a.counts;
         m.kmax = a.kmax;
         m.kmin = a.kmin;
-        m.sse = a.sse;
         m.err = a.err;
         e = launch_member_stream_d<MS_STATS>(m, a.d, s);
+        if (e != cudaSuccess) return e;
+        const int64_t n = (int64_t)a.BH * a.Ccap;
+        k_cluster_sse<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.perm, a.offs, a.offs_stride, a.dmin, a.n_k,
+                                                                   a.Ccap, a.L, a.BH, a.counts, a.sse);
+        AC_NOTE_LAUNCH();
+        e = cudaGetLastError();
     } else {
         k_key_stats<<<dim3(a.Ccap, a.BH), a.d, 0, s>>>(a);
         AC_NOTE_LAUNCH();
