@@ -212,7 +212,7 @@ def workload_config():
 # DRAM bytes (read + write) of one k_sparse_attn launch per head, from the ncu capture summarised
 # in profiles/k_sparse_attn_wan14b_h8.md (8 heads, scaled by heads), valid only for the kernel
 # source it was taken on: any change to attn_kernel.cu turns the figure into null.
-ATTN_TRAFFIC = {"sha256_prefix": "e2bc600c81be3bda", "bytes_per_head": (313.696512e6 + 133.403648e6) / 8}
+ATTN_TRAFFIC = {"sha256_prefix": "f0e4b1ad3dc6ebe4", "bytes_per_head": (313.705472e6 + 132.507648e6) / 8}
 
 
 def attn_traffic_bytes(heads):
