@@ -155,15 +155,61 @@ struct Lloyd {
     UpdateArgs up;
     bool fast = false;  // assignment on the tensor cores (fa) instead of the exact kernel (as)
     FastAssignArgs fa;
+    bool stage_copy = false;  // copy the stage centres out of cent_k before each tensor-core pass
+    long long rows = -1;      // rows one pass assigns (for the counters), when not every row of every unit
 };
+
+// Stage centres of unit h (cent_k rows n_k[h] .. n_k[h] + m[h] - 1) into the
+// compact [BH, m0, d] buffer the tensor-core assignment reads.
+__global__ void k_stage_centres(const float *__restrict__ C, int64_t cstride, const int *__restrict__ n_k,
+                                const int *__restrict__ m, int m0, int d, float *__restrict__ out) {
+    const int c = blockIdx.x, h = blockIdx.y;
+    if (c >= m[h]) return;
+    const float *src = C + (int64_t)h * cstride + (int64_t)(n_k[h] + c) * d;
+    float *dst = out + ((int64_t)h * m0 + c) * d;
+    for (int k = threadIdx.x; k < d; k += blockDim.x) dst[k] = src[k];
+}
+
+// Xg[h, pos] = X[h, idx[h, pos]] for pos < cnt[h], and sq[h, pos] = |Xg[h, pos]|^2
+// (fp32; it only enters the assignment's error bound).  d / 8 lanes per row.
+__global__ void k_gather_rows_sq(const bf16 *__restrict__ X, const int *__restrict__ idx, const int *__restrict__ cnt,
+                                 bf16 *__restrict__ Xg, float *__restrict__ sq, int64_t L, int d) {
+    const int h = blockIdx.y;
+    const int lpr = d / 8;  // lanes per row (8 or 16), a power of two dividing 32
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t pos = g / lpr;
+    const int part = (int)(g % lpr);
+    const bool v = pos < cnt[h];
+    float ss = 0.f;
+    if (v) {
+        const int64_t src = (int64_t)h * L + idx[(int64_t)h * L + pos];
+        const uint4 w = reinterpret_cast<const uint4 *>(X + src * d)[part];
+        reinterpret_cast<uint4 *>(Xg + ((int64_t)h * L + pos) * d)[part] = w;
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        for (int t = 0; t < 4; ++t) {
+            const float a = __uint_as_float(ws[t] << 16), b = __uint_as_float(ws[t] & 0xFFFF0000u);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+        }
+    }
+    for (int o = lpr / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    if (v && part == 0) sq[(int64_t)h * L + pos] = ss;
+}
 
 // One assignment pass; dmin (where the caller asked for it) only when wanted.
 cudaError_t assign_pass(ac_ctx *c, const Lloyd &k, bool want_dmin, cudaStream_t s) {
     if (k.fast) {
+        if (k.stage_copy) {
+            k_stage_centres<<<dim3(c->cfg.m0, c->BH), 128, 0, s>>>(c->cent_k, (int64_t)c->Ccap * c->d, c->n_k,
+                                                                   c->st_m, c->cfg.m0, c->d, c->cent_st);
+            AC_NOTE_LAUNCH();
+            cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
         FastAssignArgs a = k.fa;
         if (!want_dmin) a.dmin = nullptr;
         ++c->n_fast;
-        c->n_fast_rows += (long long)a.BH * a.L;
+        c->n_fast_rows += k.rows >= 0 ? k.rows : (long long)a.BH * a.L;
         return launch_assign_fast(a, s);
     }
     ++c->n_exact;
@@ -189,7 +235,7 @@ cudaError_t run_lloyd(ac_ctx *c, Lloyd &k, int T, bool final_sort, cudaStream_t 
 bool make_fast(ac_ctx *c, Lloyd &k, const bf16 *X, bool queries, const float *C, int64_t cstride,
                const int *ncent, int ncent_const, int *labels, float *dmin) {
     if (!c->fast_assign || (reinterpret_cast<uintptr_t>(X) & 15u) != 0) return false;
-    CUtensorMap *tmx = queries ? &c->tm_xq : &c->tm_xk;
+    CUtensorMap *tmx = queries ? &c->tm_xq : (X == c->Qp ? &c->tm_xu : &c->tm_xk);
     if (make_tmap(c, tmx, const_cast<bf16 *>(X), (int64_t)c->BH * c->L, c->d, 128) != AC_OK) return false;
     FastAssignArgs &a = k.fa;
     a.tm_x = tmx;
@@ -313,8 +359,26 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
                         0, BH, c->sort_scratch};
         k.up = UpdateArgs{K, nullptr, L, c->u_idx, c->st_perm, c->st_offs, m0 + 1, c->cent_k, cstride, c->n_k,
                           c->st_m, 0, BH, d, max_m};
-        // stage 0: U is every key in order and the stage's centres start at 0
-        if (t == 0) make_fast(c, k, K, false, c->cent_k, cstride, c->st_m, 0, c->st_labels, c->dmin_k);
+        // stage 0: U is every key in order and the stage's centres start at 0;
+        // later stages: the GEMM runs on a gathered copy of U and a compact copy
+        // of the stage's centres (labels and distances by position in U, as the
+        // exact kernel gives them)
+        if (t == 0) {
+            make_fast(c, k, K, false, c->cent_k, cstride, c->st_m, 0, c->st_labels, c->dmin_k);
+        } else if (c->fast_assign && (reinterpret_cast<uintptr_t>(K) & 15u) == 0) {
+            const int64_t per = (int64_t)L * (d / 8);
+            k_gather_rows_sq<<<dim3((unsigned)((per + 255) / 256), BH), 256, 0, s>>>(K, c->u_idx, c->u_cnt, c->Qp,
+                                                                                  c->rowsq_u, L, d);
+            AC_NOTE_LAUNCH();
+            CK(cudaGetLastError(), "gather stage keys");
+            if (make_fast(c, k, c->Qp, false, c->cent_st, (int64_t)m0 * d, c->st_m, 0, c->st_labels, c->dmin_k)) {
+                k.fa.rowsq = c->rowsq_u;
+                k.fa.nrows = c->u_cnt;
+                k.stage_copy = true;
+                k.rows = 0;
+                for (int h = 0; h < BH; ++h) k.rows += m[h] > 0 ? ucnt[h] : 0;
+            }
+        }
         CK(run_lloyd(c, k, c->cfg.iters_k, false, s), "k stage lloyd");
         // line 14: d_i = ||k_i - c(k_i)||
         CK(launch_stage_dist(c->dmin_k, c->st_dist, c->u_cnt, c->st_m, L, BH, t == 0 ? c->tau_acc : nullptr, s),
@@ -388,7 +452,7 @@ ac_status key_stats_impl(ac_ctx *c, const bf16 *K, cudaStream_t s) {
     CK(launch_counting_sort(so, s), "k sort");
     StatsArgs st{K, c->L, c->perm_k, c->offs_k, c->Ccap + 1, c->dmin_k, c->n_k, c->Ccap, c->d, c->BH,
                  c->counts_k, c->kmax, c->kmin, c->sse, c->mse, c->comp, c->cent_k, (int64_t)c->Ccap * c->d,
-                 c->err};
+                 c->err, c->st_dist};
     CK(launch_key_stats(st, s), "k stats");
     c->have_k = true;
     return AC_OK;
@@ -425,7 +489,7 @@ void free_all(ac_ctx *c) {
                    c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->Qp, c->Kp, c->Vp,
                    c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err, c->chi_q, c->chi_k, c->cn,
                    c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats, c->rbox, c->pgoff, c->nrange,
-                   c->sort_scratch, c->cnp_k};
+                   c->sort_scratch, c->cnp_k, c->rowsq_u, c->cent_st};
     for (void *p : dev)
         if (p) cudaFree(p);
     void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err};
@@ -543,6 +607,8 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->cn, BH * std::max(c->Cpad_q, c->Cpad_k)));
     A(dalloc(&c->hstat, 2 * BH));
     A(dalloc(&c->rowsq_k, BH * Lz));
+    A(dalloc(&c->rowsq_u, BH * Lz));
+    A(dalloc(&c->cent_st, BH * (size_t)m0 * dz));
     A(dalloc(&c->cand, BH * Lz));
     A(dalloc(&c->amb_list, BH * Lz));
     A(dalloc(&c->amb_count, 2));

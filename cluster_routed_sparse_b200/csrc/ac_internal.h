@@ -80,6 +80,9 @@ struct ac_ctx {
     bf16 *cnp_k;       // [BH, Cpad_k, 16] |c'|^2 of the key centres as three bf16 parts
     CUtensorMap tm_cnp_k;
     CUtensorMap tm_xq, tm_xk;  // caller's Q / K of the current call
+    CUtensorMap tm_xu;         // gathered keys of a stage t >= 1 (rows of Qp, which is free then)
+    float *rowsq_u;            // [BH, L] |k|^2 of the gathered keys, by position in U
+    float *cent_st;            // [BH, m0, d] the stage's centres, copied out of cent_k for the GEMM
     int num_sms;
     bool fast_assign;
     long long n_fast, n_exact, n_fast_rows;
@@ -235,6 +238,7 @@ struct StatsArgs {
     int *counts; bf16 *kmax; bf16 *kmin; float *sse; float *mse; float *comp;
     const float *C; int64_t cstride;  // key centres
     uint32_t *err;
+    float *dsorted;                   // [BH, L] scratch: the distances in member order
 };
 cudaError_t launch_key_stats(const StatsArgs &a, cudaStream_t s);
 

@@ -169,22 +169,24 @@ __global__ void __launch_bounds__(SORT_WARPS * 32) k_sort_hist(SortArgs a) {
     for (int l = lane; l < m; l += 32) H[l] = hist[w * m + l];
 }
 
-__global__ void __launch_bounds__(256) k_sort_offsets(SortArgs a) {
+constexpr int SORT_OFF_THREADS = 1024;
+__global__ void __launch_bounds__(SORT_OFF_THREADS) k_sort_offsets(SortArgs a) {
     extern __shared__ int tot[];  // [max_lab]
-    typedef cub::BlockScan<int, 256> Scan;
+    typedef cub::BlockScan<int, SORT_OFF_THREADS> Scan;
     __shared__ typename Scan::TempStorage scan_tmp;
     const int h = blockIdx.x, tid = threadIdx.x;
     const int n = a.nrows ? a.nrows[h] : a.nrows_const;
     const int m = a.nlab ? a.nlab[h] : a.nlab_const;
     if (m <= 0) return;
     int *H = a.scratch + (int64_t)h * SORT_CHUNKS * a.max_lab;
-    for (int l = tid; l < m; l += 256) {
+    for (int l = tid; l < m; l += SORT_OFF_THREADS) {
         int t = 0;
+#pragma unroll 8
         for (int ci = 0; ci < SORT_CHUNKS; ++ci) t += H[(int64_t)ci * a.max_lab + l];
         tot[l] = t;
     }
     __syncthreads();
-    const int sg = (m + 255) / 256;
+    const int sg = (m + SORT_OFF_THREADS - 1) / SORT_OFF_THREADS;
     const int l0 = min(m, tid * sg), l1 = min(m, l0 + sg);
     int local = 0;
     for (int l = l0; l < l1; ++l) local += tot[l];
@@ -198,14 +200,19 @@ __global__ void __launch_bounds__(256) k_sort_offsets(SortArgs a) {
     }
     __syncthreads();
     int *offs = a.offs + (int64_t)h * a.offs_stride;
-    for (int l = tid; l < m; l += 256) {
+    for (int l = tid; l < m; l += SORT_OFF_THREADS) {
         int slot = tot[l];
         offs[l] = slot;
         const int first = slot;
-        for (int ci = 0; ci < SORT_CHUNKS; ++ci) {
-            const int c = H[(int64_t)ci * a.max_lab + l];
-            H[(int64_t)ci * a.max_lab + l] = slot;  // first slot of chunk ci for label l
-            slot += c;
+        for (int c0 = 0; c0 < SORT_CHUNKS; c0 += 8) {
+            int cv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) cv[u] = H[(int64_t)(c0 + u) * a.max_lab + l];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                H[(int64_t)(c0 + u) * a.max_lab + l] = slot;  // first slot of chunk c0 + u for label l
+                slot += cv[u];
+            }
         }
         if (a.counts) a.counts[(int64_t)h * a.counts_stride + l] = slot - first;
     }
@@ -333,7 +340,7 @@ cudaError_t launch_counting_sort(const SortArgs &a, cudaStream_t s) {
     k_sort_hist<<<grid, SORT_WARPS * 32, smem, s>>>(a);
     AC_NOTE_LAUNCH();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_sort_offsets<<<a.BH, 256, (size_t)a.max_lab * sizeof(int), s>>>(a);
+    k_sort_offsets<<<a.BH, SORT_OFF_THREADS, (size_t)a.max_lab * sizeof(int), s>>>(a);
     AC_NOTE_LAUNCH();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_sort_scatter<<<grid, SORT_WARPS * 32, smem, s>>>(a);
@@ -366,7 +373,7 @@ struct MsArgs {
     const int *ncent; int ncent_const;  // clusters c < m(h) hold members
     int maxc, BH;                       // flat list: f = h * maxc + c
     float *C; int64_t cstride; const int *coff;  // update: centres written; stats: centres read
-    float *dmin; bf16 *kmax; bf16 *kmin;         // stats
+    float *dmin; float *dsorted; bf16 *kmax; bf16 *kmin;  // stats
     uint32_t *err;
 };
 
@@ -615,7 +622,7 @@ __global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
                 if (lane == 0) {
                     const int fl = (j0 == dw.y ? MS_FIRST : 0) | (j0 + BATCH >= dw.z ? MS_LAST : 0) |
                                    (cnt <= 0 ? MS_EMPTY : 0);
-                    meta[slot] = make_int4(dw.x, cnt, fl, dw.z - dw.y);
+                    meta[slot] = make_int4(dw.x, cnt | (fl << 8), dw.z - dw.y, j0);
                 }
                 const uint32_t dst = sbase + slot * LY::STAGE + (lane % PPR) * 16;
 #pragma unroll
@@ -647,7 +654,7 @@ __global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
             const uint32_t slot = it % MS_STAGES;
             if (it >= MS_STAGES && !mbar_wait(bar_empty + 8 * slot, ((it / MS_STAGES) - 1) & 1)) ok = false;
             if (ok) {
-                if (lane == 0) meta[slot] = make_int4(0, 0, MS_END, 0);
+                if (lane == 0) meta[slot] = make_int4(0, MS_END << 8, 0, 0);
                 ms_cp_arrive(bar_full + 8 * slot);
                 if (lane == 0) mbar_arrive(bar_full + 8 * slot);
             }
@@ -669,13 +676,14 @@ __global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
             if (lane == 0 && a.err) set_err(a.err, DEV_ERR_TIMEOUT);
             break;
         }
-        const int4 mt = meta[slot];
-        if (mt.z & MS_END) break;
-        const int h = mt.x / a.maxc, c = mt.x - h * a.maxc, cnt = mt.y;
+        const int4 mt = meta[slot];  // cluster, count | flags << 8, members, first position
+        const int fl = mt.y >> 8, cnt = mt.y & 0xFF;
+        if (fl & MS_END) break;
+        const int h = mt.x / a.maxc, c = mt.x - h * a.maxc;
         const uint8_t *rs = ms_sm + slot * LY::STAGE;
         const bf16 *col = reinterpret_cast<const bf16 *>(rs) + k;
         if (MODE != MS_STATS) {
-            if (mt.z & MS_FIRST) s = 0.f;
+            if (fl & MS_FIRST) s = 0.f;
             const float *inv_s = aux_s + slot * BATCH;
             int r = 0;
             for (; r + 32 <= cnt; r += 32) {
@@ -693,16 +701,16 @@ __global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
                 if (MODE == MS_UPDATE_NORM) v = __fmul_rn(v, inv_s[r]);
                 s = __fadd_rn(s, v);
             }
-            if (mt.z & MS_LAST) {
+            if (fl & MS_LAST) {
                 const int off = a.coff ? a.coff[h] : 0;
-                a.C[(int64_t)h * a.cstride + (int64_t)(off + c) * D + k] = __fdiv_rn(s, (float)mt.w);
+                a.C[(int64_t)h * a.cstride + (int64_t)(off + c) * D + k] = __fdiv_rn(s, (float)mt.z);
             }
         } else {
             const int64_t ci = (int64_t)h * a.maxc + c;
-            if (mt.z & MS_EMPTY) {
+            if (fl & MS_EMPTY) {
                 mx = mn = 0.f;
             } else {
-                if (mt.z & MS_FIRST) mx = mn = bf2f(col[0]);
+                if (fl & MS_FIRST) mx = mn = bf2f(col[0]);
                 for (int r = 0; r < cnt; ++r) {
                     const float v = bf2f(col[r * RS]);
                     mx = v > mx ? v : mx;
@@ -712,10 +720,12 @@ __global__ void __launch_bounds__(D + 32) k_member_stream(MsArgs a) {
                 // exact distances: member row `lane` to the centre
                 if (warp == (int)(it % NCW) && lane < cnt) {
                     const int tok = reinterpret_cast<const int *>(aux_s)[slot * BATCH + lane];
-                    a.dmin[(int64_t)h * a.L + tok] = ms_sqdist<D>(rs + lane * LY::ROWB, cent_s + slot * D);
+                    const float dd = ms_sqdist<D>(rs + lane * LY::ROWB, cent_s + slot * D);
+                    a.dmin[(int64_t)h * a.L + tok] = dd;
+                    a.dsorted[(int64_t)h * a.L + mt.w + lane] = dd;  // member order, for the SSE
                 }
             }
-            if (mt.z & MS_LAST) {
+            if (fl & MS_LAST) {
                 a.kmax[ci * D + k] = __float2bfloat16(mx);
                 a.kmin[ci * D + k] = __float2bfloat16(mn);
             }
@@ -749,34 +759,36 @@ cudaError_t launch_member_stream_d(const MsArgs &a, int d, cudaStream_t s) {
     return d == 128 ? launch_member_stream<128, MODE>(a, s) : launch_member_stream<64, MODE>(a, s);
 }
 
-// Per key cluster: count and SSE = the members' exact distances (dmin, from
-// the statistics pass) summed in ascending member order; 0 for the slots
-// c >= n_k.  One thread per cluster.
-__global__ void k_cluster_sse(const int *__restrict__ perm, const int *__restrict__ offs, int offs_stride,
-                              const float *__restrict__ dmin, const int *__restrict__ n_k, int Ccap, int64_t L,
-                              int BH, int *__restrict__ counts, float *__restrict__ sse) {
-    const int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (f >= (int64_t)BH * Ccap) return;
-    const int h = (int)(f / Ccap), c = (int)(f - (int64_t)h * Ccap);
-    int beg = 0, end = 0;
-    if (c < n_k[h]) {
-        beg = offs[(int64_t)h * offs_stride + c];
-        end = offs[(int64_t)h * offs_stride + c + 1];
+// Per key cluster: count and SSE = the members' exact distances (written in
+// member order by the statistics pass) summed in ascending member order; 0
+// for the slots c >= n_k.  One warp per cluster: 32 distances per load, the
+// next 32 in flight while every lane adds the current ones in order.
+__global__ void k_cluster_sse(const int *__restrict__ offs, int offs_stride, const float *__restrict__ dsorted,
+                              const int *__restrict__ n_k, int Ccap, int64_t L, int BH, int *__restrict__ counts,
+                              float *__restrict__ sse) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t f = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; f < (int64_t)BH * Ccap; f += nw) {
+        const int h = (int)(f / Ccap), c = (int)(f - (int64_t)h * Ccap);
+        int beg = 0, end = 0;
+        if (c < n_k[h]) {
+            beg = offs[(int64_t)h * offs_stride + c];
+            end = offs[(int64_t)h * offs_stride + c + 1];
+        }
+        const float *ds = dsorted + (int64_t)h * L;
+        float se = 0.f;
+        float v = beg + lane < end ? ds[beg + lane] : 0.f;
+        for (int j = beg; j < end; j += 32) {
+            const float vn = j + 32 + lane < end ? ds[j + 32 + lane] : 0.f;
+            const int n = min(32, end - j);
+            for (int r = 0; r < n; ++r) se = __fadd_rn(se, __shfl_sync(0xFFFFFFFFu, v, r));
+            v = vn;
+        }
+        if (lane == 0) {
+            sse[f] = se;
+            counts[f] = end - beg;
+        }
     }
-    const int *pm = perm + (int64_t)h * L;
-    const float *dm = dmin + (int64_t)h * L;
-    float se = 0.f;
-    int j = beg;
-    for (; j + 8 <= end; j += 8) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = dm[pm[j + u]];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) se = __fadd_rn(se, v[u]);
-    }
-    for (; j < end; ++j) se = __fadd_rn(se, dm[pm[j]]);
-    sse[f] = se;
-    counts[f] = end - beg;
 }
 
 // Bulk copies need 16-byte aligned rows.
@@ -1118,14 +1130,16 @@ cudaError_t launch_key_stats(const StatsArgs &a, cudaStream_t s) {
         m.C = const_cast<float *>(a.C);
         m.cstride = a.cstride;
         m.dmin = a.dmin;
+        m.dsorted = a.dsorted;
         m.kmax = a.kmax;
         m.kmin = a.kmin;
         m.err = a.err;
         e = launch_member_stream_d<MS_STATS>(m, a.d, s);
         if (e != cudaSuccess) return e;
-        const int64_t n = (int64_t)a.BH * a.Ccap;
-        k_cluster_sse<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.perm, a.offs, a.offs_stride, a.dmin, a.n_k,
-                                                                   a.Ccap, a.L, a.BH, a.counts, a.sse);
+        const int64_t n = (int64_t)a.BH * a.Ccap;  // one warp per cluster
+        const unsigned blocks = (unsigned)std::min<int64_t>((n + 7) / 8, 148 * 16);
+        k_cluster_sse<<<blocks, 256, 0, s>>>(a.offs, a.offs_stride, a.dsorted, a.n_k, a.Ccap, a.L, a.BH, a.counts,
+                                             a.sse);
         AC_NOTE_LAUNCH();
         e = cudaGetLastError();
     } else {
