@@ -88,6 +88,8 @@ SIGNATURES = {
     "ac_sparse_attn": (_I, [_P, _P, _P, _P, _P, _P]),
     "ac_layer_forward": (_I, [_P, _P, _P, _P, _P, _I, ctypes.POINTER(ACStageTimes), _P]),
     "ac_layer_forward_host": (_I, [_P, _P, _P, _P, _P, _I, _P]),
+    "ac_layer_forward_host_async": (_I, [_P, _P, _P, _P, _P, _I, _P]),
+    "ac_join": (_I, [_P, _P]),
     "ac_synchronize": (_I, [_P, _P]),
     "ac_get_tensor": (_I, [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int64)]),
     "ac_get_attn_counters": (_I, [_P, ctypes.POINTER(ACAttnCounters)]),

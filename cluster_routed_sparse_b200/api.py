@@ -113,6 +113,19 @@ class SparseLayer:
                                              1 if warm else 0, _stream()), self.ctx)
         return hO
 
+    def forward_host_async(self, hQ, hK, hV, hO, warm: bool = False):
+        """As forward_host, without waiting: hO is written once the current
+        stream has passed join() (or after synchronize()); keep the inputs
+        unchanged until then.  Consecutive calls overlap their copies with the
+        neighbouring calls' layers."""
+        check(self.lib.ac_layer_forward_host_async(self.ctx, _bits(hQ), _bits(hK), _bits(hV), _bits(hO),
+                                                   1 if warm else 0, _stream()), self.ctx)
+        return hO
+
+    def join(self):
+        """Make the current stream wait for the output copies of earlier async calls."""
+        check(self.lib.ac_join(self.ctx, _stream()), self.ctx)
+
     def synchronize(self):
         check(self.lib.ac_synchronize(self.ctx, _stream()), self.ctx)
 

@@ -497,6 +497,15 @@ void free_all(ac_ctx *c) {
         if (p) cudaFreeHost(p);
     for (auto &e : c->ev)
         if (e) cudaEventDestroy(e);
+    for (int b = 0; b < 2; ++b) {
+        for (int i = 0; i < 4; ++i)
+            if (c->abuf[b][i]) cudaFree(c->abuf[b][i]);
+        if (c->ev_in[b]) cudaEventDestroy(c->ev_in[b]);
+        if (c->ev_comp[b]) cudaEventDestroy(c->ev_comp[b]);
+        if (c->ev_out[b]) cudaEventDestroy(c->ev_out[b]);
+    }
+    if (c->s_in) cudaStreamDestroy(c->s_in);
+    if (c->s_out) cudaStreamDestroy(c->s_out);
 }
 
 }  // namespace
@@ -862,7 +871,63 @@ ac_status ac_get_launch_count(int64_t *out) {
 
 ac_status ac_synchronize(ac_ctx *c, void *stream) {
     if (!c) return AC_ERR_INVALID_ARG;
+    ac_status st = ac_join(c, stream);
+    if (st != AC_OK) return st;
     return check_dev_err(c, (cudaStream_t)stream);
+}
+
+ac_status ac_join(ac_ctx *c, void *stream) {
+    if (!c) return AC_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    for (int b = 0; b < 2; ++b)
+        if (c->ev_out[b]) CK(cudaStreamWaitEvent(s, c->ev_out[b], 0), "join");
+    return AC_OK;
+}
+
+// Call n uses staging set n % 2.  Inputs of call n are copied on s_in once
+// call n - 2 (same set) has finished its layer; the layer runs on the caller's
+// stream once those inputs have landed and call n - 2's output copy has left
+// the set; the output is copied on s_out once the layer is done.  So call n's
+// input copy overlaps call n - 1's layer, and its output copy call n + 1's.
+ac_status ac_layer_forward_host_async(ac_ctx *c, const uint16_t *hQ, const uint16_t *hK, const uint16_t *hV,
+                                      uint16_t *hO, int32_t warm, void *stream) {
+    if (!c || !hQ || !hK || !hV || !hO)
+        return fail(c, AC_ERR_INVALID_ARG, "ac_layer_forward_host_async: NULL argument");
+    if (warm && !c->have_state) return fail(c, AC_ERR_STATE, "warm step before any step 0");
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t n = (size_t)c->BH * c->L * c->d;
+    if (!c->s_in) {
+        for (int b = 0; b < 2; ++b)
+            for (int i = 0; i < 4; ++i)
+                if (dalloc(&c->abuf[b][i], n) != cudaSuccess) {
+                    cudaGetLastError();
+                    return fail(c, AC_ERR_WORKSPACE, "host-buffer staging allocation failed");
+                }
+        for (int b = 0; b < 2; ++b) {
+            CK(cudaEventCreateWithFlags(&c->ev_in[b], cudaEventDisableTiming), "event");
+            CK(cudaEventCreateWithFlags(&c->ev_comp[b], cudaEventDisableTiming), "event");
+            CK(cudaEventCreateWithFlags(&c->ev_out[b], cudaEventDisableTiming), "event");
+        }
+        CK(cudaStreamCreateWithFlags(&c->s_in, cudaStreamNonBlocking), "stream");
+        CK(cudaStreamCreateWithFlags(&c->s_out, cudaStreamNonBlocking), "stream");
+    }
+    const int b = (int)(c->async_calls & 1);
+    uint16_t **buf = c->abuf[b];
+    if (c->async_calls >= 2) CK(cudaStreamWaitEvent(c->s_in, c->ev_comp[b], 0), "wait layer");
+    CK(cudaMemcpyAsync(buf[0], hQ, n * 2, cudaMemcpyHostToDevice, c->s_in), "h2d Q");
+    CK(cudaMemcpyAsync(buf[1], hK, n * 2, cudaMemcpyHostToDevice, c->s_in), "h2d K");
+    CK(cudaMemcpyAsync(buf[2], hV, n * 2, cudaMemcpyHostToDevice, c->s_in), "h2d V");
+    CK(cudaEventRecord(c->ev_in[b], c->s_in), "event");
+    CK(cudaStreamWaitEvent(s, c->ev_in[b], 0), "wait inputs");
+    if (c->async_calls >= 2) CK(cudaStreamWaitEvent(s, c->ev_out[b], 0), "wait output copy");
+    ++c->async_calls;
+    ac_status st = ac_layer_forward(c, buf[0], buf[1], buf[2], buf[3], warm, nullptr, stream);
+    if (st != AC_OK) return st;
+    CK(cudaEventRecord(c->ev_comp[b], s), "event");
+    CK(cudaStreamWaitEvent(c->s_out, c->ev_comp[b], 0), "wait layer");
+    CK(cudaMemcpyAsync(hO, buf[3], n * 2, cudaMemcpyDeviceToHost, c->s_out), "d2h O");
+    CK(cudaEventRecord(c->ev_out[b], c->s_out), "event");
+    return AC_OK;
 }
 
 ac_status ac_get_assign_counters(ac_ctx *c, ac_assign_counters *out, int32_t reset) {

@@ -100,6 +100,13 @@ struct ac_ctx {
 
     // ---- host-buffer forward
     uint16_t *hbufQ, *hbufK, *hbufV, *hbufO;  // device staging of the host entry point
+    // asynchronous host entry point: two staging sets (Q, K, V, O each), an
+    // input-copy and an output-copy stream, and per set the events "inputs
+    // landed", "layer done" and "output copied"
+    uint16_t *abuf[2][4];
+    cudaStream_t s_in, s_out;
+    cudaEvent_t ev_in[2], ev_comp[2], ev_out[2];
+    long long async_calls;
 
     uint32_t *err;      // device error word
     int *h_u_cnt;       // pinned host mirrors

@@ -188,7 +188,26 @@ AC_API ac_status ac_layer_forward(ac_ctx *ctx, const uint16_t *Q, const uint16_t
 AC_API ac_status ac_layer_forward_host(ac_ctx *ctx, const uint16_t *hQ, const uint16_t *hK,
                                 const uint16_t *hV, uint16_t *hO, int32_t warm, void *stream);
 
-/* Wait for the work enqueued on `stream` and report any error that a kernel
+/* ac_layer_forward_host without waiting: enqueues the input copies (on a
+ * context-owned copy stream), the layer (on `stream`) and the output copy (on a
+ * second copy stream) and returns.  Consecutive calls pipeline: call n's input
+ * copy overlaps call n - 1's layer and its output copy call n + 1's layer
+ * (two context-owned device staging sets, used alternately).
+ * Ownership: hQ, hK, hV must stay unchanged, and hO must not be read, until
+ * the call is complete: after ac_synchronize(ctx, stream) returns, or once
+ * `stream` has passed an ac_join(ctx, stream).  Host buffers should be pinned
+ * (pageable memory makes the copies synchronous).  Errors: argument and launch
+ * errors are returned; errors that kernels record on the device are reported
+ * by the next ac_synchronize. */
+AC_API ac_status ac_layer_forward_host_async(ac_ctx *ctx, const uint16_t *hQ, const uint16_t *hK,
+                                      const uint16_t *hV, uint16_t *hO, int32_t warm, void *stream);
+
+/* Make `stream` wait (without blocking the host) until the output copies of
+ * every earlier ac_layer_forward_host_async call have finished. */
+AC_API ac_status ac_join(ac_ctx *ctx, void *stream);
+
+/* Wait for the work enqueued on `stream` (and for the output copies of earlier
+ * ac_layer_forward_host_async calls) and report any error that a kernel
  * recorded on the device (AC_ERR_TIMEOUT, AC_ERR_NONFINITE); clears it. */
 AC_API ac_status ac_synchronize(ac_ctx *ctx, void *stream);
 

@@ -137,6 +137,33 @@ def test_host_entry_point_matches_device_forward():
     lay2.close()
 
 
+def test_async_host_entry_point_pipelines_three_steps():
+    """ac_layer_forward_host_async over step 0 and two warm steps (calls queued
+    back to back, copies overlapping the neighbouring layers) gives the same
+    outputs as the device-buffer forward of the same steps."""
+    cfg = synth.CONFIGS[1]
+    p = _params(cfg)
+    steps = [synth.make_layer(cfg, step=s) for s in range(3)]
+    ref = make_layer_ctx(p, *steps[0][0].shape)
+    want = []
+    for s, (Q, K, V) in enumerate(steps):
+        q, k, v = dev(Q), dev(K), dev(V)
+        o = torch.empty_like(q)
+        ref.forward(q, k, v, o, warm=s > 0)
+        ref.synchronize()
+        want.append(o.view(torch.int16).cpu().numpy())
+    lay = make_layer_ctx(p, *steps[0][0].shape)
+    host = [[torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in st] for st in steps]
+    outs = [torch.empty_like(host[0][0]).pin_memory() for _ in steps]
+    for s in range(3):
+        lay.forward_host_async(*host[s], outs[s], warm=s > 0)
+    lay.synchronize()
+    for s in range(3):
+        assert np.array_equal(outs[s].view(torch.int16).numpy(), want[s].reshape(outs[s].shape)), s
+    ref.close()
+    lay.close()
+
+
 def test_state_resume_is_bit_exact():
     """Checkpoint/resume across denoising steps: exporting the warm-start state
     after step 0 and importing it into a fresh context gives the same warm step."""
