@@ -563,7 +563,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
         c->fast_assign = !(ev && ev[0] == '1');
     }
     c->Cpad_q = (c->Cq + 31) & ~31;
-    c->CH_q = std::min(64, c->Cpad_q);  // two-term chunks (c_hi + c_lo) of at most 64 centres
+    c->CH_q = std::min(96, c->Cpad_q);  // two-term chunks (c_hi + c_lo) of at most 96 centres
     c->Cpad_k = (c->Ccap + 31) & ~31;
     c->CH_k = std::min(128, c->Cpad_k);
     const size_t BH = c->BH, Lz = L, dz = d, Cq = c->Cq, Cc = c->Ccap, m0 = cfg->m0;

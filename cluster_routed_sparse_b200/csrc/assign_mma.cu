@@ -34,12 +34,13 @@ constexpr int ACH = 128;      // centres per chunk at most (MMA N)
 constexpr int A_EPI = 256;    // epilogue threads: one per row of the unit
 constexpr int A_THREADS = A_EPI + 64;
 constexpr int A_NC = 2;       // centre chunk stages
+constexpr int QCH = 96;       // query centres per chunk at most (c_hi and c_lo: twice the operand bytes)
 constexpr int A_NCMAX = 3;    // barriers reserved
 
 // Shared memory: [2] row units (two 128-row tiles each) | [NC] centre chunks.
 // A chunk holds the c_hi rows (and the c_lo rows) of up to ACH centres, each
 // operand as [column half][rows][128 B] with the 128-byte swizzle.
-template <int D>
+template <int D, bool FOLD>
 struct ALayout {
     static constexpr int HALVES = D / 64;
     static constexpr uint32_t XT_BYTES = HALVES * AM * 128;  // one 128-row tile
@@ -47,11 +48,12 @@ struct ALayout {
     static constexpr uint32_t OFF_X = 0;
     static constexpr uint32_t OFF_C = OFF_X + 2 * X_BYTES;
     // two stages of ACH key centres (-2 c_hi, then the |c'|^2 slice: two
-    // no-swizzle 16-byte columns of ACH rows), or of up to 64 query centres
+    // no-swizzle 16-byte columns of ACH rows), or of up to QCH query centres
     // (c_hi, c_lo)
-    static constexpr uint32_t C_REGION = A_NC * (HALVES * ACH * 128 + ACH * 32);
-    static constexpr uint32_t OFF_XE = OFF_C + C_REGION;  // the constant [1 1 1 0 ...] K slice, 128 rows
-    static constexpr uint32_t OFF_BAR = OFF_XE + AM * 32;
+    static constexpr uint32_t C_REGION =
+        FOLD ? A_NC * (HALVES * ACH * 128 + ACH * 32) : A_NC * (2 * HALVES * QCH * 128);
+    static constexpr uint32_t OFF_XE = OFF_C + C_REGION;  // keys: the constant [1 1 1 0 ...] K slice, 128 rows
+    static constexpr uint32_t OFF_BAR = OFF_XE + (FOLD ? AM * 32 : 0);
     static constexpr uint32_t BYTES = OFF_BAR + 256;
     static constexpr uint32_t SMEM = BYTES + 1024;
 };
@@ -167,7 +169,7 @@ template <int D, bool FOLD>
 __global__ void __launch_bounds__(A_THREADS, 1)
     k_assign_mma(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_c,
                  const __grid_constant__ CUtensorMap tm_cn, const AsgParams p) {
-    using LY = ALayout<D>;
+    using LY = ALayout<D, FOLD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -715,14 +717,15 @@ __global__ void k_centre_prep(const float *__restrict__ C, int64_t cstride, cons
     }
 }
 
-static_assert(ALayout<128>::SMEM <= 232448, "assignment kernel exceeds the shared memory of a block");
+static_assert(ALayout<128, true>::SMEM <= 232448 && ALayout<128, false>::SMEM <= 232448,
+              "assignment kernel exceeds the shared memory of a block");
 
 template <int D, bool FOLD>
 cudaError_t launch_mma(const FastAssignArgs &a, const AsgParams &p, int grid, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(k_assign_mma<D, FOLD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)ALayout<D>::SMEM);
+                                         (int)ALayout<D, FOLD>::SMEM);
     if (e != cudaSuccess) return e;
-    k_assign_mma<D, FOLD><<<grid, A_THREADS, ALayout<D>::SMEM, s>>>(*a.tm_x, *a.tm_c, FOLD ? *a.tm_cn : *a.tm_c, p);
+    k_assign_mma<D, FOLD><<<grid, A_THREADS, ALayout<D, FOLD>::SMEM, s>>>(*a.tm_x, *a.tm_c, FOLD ? *a.tm_cn : *a.tm_c, p);
     AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
@@ -777,8 +780,10 @@ cudaError_t launch_assign_fast(const FastAssignArgs &a, cudaStream_t s) {
     p.c_stage = (uint32_t)(a.two_term ? 2 * (a.d / 64) * a.CH * 128 : (a.d / 64) * a.CH * 128 + a.CH * 32);
     p.nc = A_NC;
     // the centre stages must fit their region of shared memory
-    if (a.CH < 32 || a.CH > ACH || (a.CH & 31) || (a.two_term && a.CH > 64) || (a.Cpad & 31) ||
-        (uint64_t)p.nc * p.c_stage > (uint64_t)A_NC * ((a.d / 64) * ACH * 128 + ACH * 32))
+    const uint64_t region = a.two_term ? (uint64_t)A_NC * 2 * (a.d / 64) * QCH * 128
+                                       : (uint64_t)A_NC * ((a.d / 64) * ACH * 128 + ACH * 32);
+    if (a.CH < 32 || a.CH > ACH || (a.CH & 31) || (a.two_term && a.CH > QCH) || (a.Cpad & 31) ||
+        (uint64_t)p.nc * p.c_stage > region)
         return cudaErrorInvalidValue;
     const int nunits = BH * p.units_per_head;
     const int grid = nunits < a.num_sms ? nunits : a.num_sms;
