@@ -462,6 +462,8 @@ ac_status score_select_impl(ac_ctx *c, int topk, cudaStream_t s) {
     SelectArgs a{c->cent_q, c->kmax, c->kmin, c->counts_k, c->n_k, c->dense, c->offs_k, c->counts_q,
                  c->Cq, c->Ccap, c->d, c->BH, c->L, topk != 0 ? topk : c->cfg.topk,
                  c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->rbox, c->pgoff, c->nrange};
+    a.score_mode = c->cfg.score_mode;
+    a.cent_k = c->cent_k;
     CK(launch_score_select(a, s), "score select");
     return AC_OK;
 }
@@ -525,7 +527,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     if (d != 64 && d != 128) return AC_ERR_UNSUPPORTED;
     if (cfg->Cq < 1 || cfg->Cq > L || cfg->m0 < 1 || cfg->m0 > L || cfg->n_max < 1 || cfg->iters_q < 0 ||
         cfg->iters_k < 0 || cfg->iters_warm < 0 || cfg->tau_mode < 0 || cfg->tau_mode > 2 || cfg->topk == 0 ||
-        cfg->stage_rule < 0 || cfg->stage_rule > 1 || cfg->reserved1 != 0 || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
+        cfg->stage_rule < 0 || cfg->stage_rule > 1 || (cfg->score_mode != 0 && cfg->score_mode != 1) || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
         return AC_ERR_INVALID_ARG;
     if ((int64_t)B * H * L >= (int64_t)1 << 31) return AC_ERR_INVALID_ARG;
     if (cfg->tau_mode == AC_TAU_PERCENTILE && (cfg->tau_value < 1.f || cfg->tau_value > 1000.f))

@@ -262,6 +262,8 @@ struct SelectArgs {
     int Cq, Ccap, d, BH, L, topk;
     float *score; int *sel; int *ksel; int2 *ranges; int *nboxes; int *tile_prefix;
     int *rbox; int *pgoff; int *nrange;
+    int score_mode = 0;            // 0: Eq. (1) bound; 1: mean-based (q . centre of the key cluster)
+    const float *cent_k = nullptr;  // [BH, Ccap, d] key centres (score_mode 1)
 };
 cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s);
 

@@ -27,7 +27,9 @@ constexpr int QS_PER = 9;                       // query centroids per thread an
 
 // Eq. (1) for every (query cluster, key cluster) of a head:
 //   S[qc, c] = sum_d max(q_d Kmax_d, q_d Kmin_d), summed d = 0, 1, ...; empty
-// clusters -inf.  Block (h, c-chunk): thread (g, ci) takes key cluster
+// clusters -inf.  score_mode 1 (the "w/o Quest" ablation, Sec. 4.4 Table 4)
+// stages the cluster's centre mu as both bounds, so the same loop gives
+// sum_d q_d mu_d.  Block (h, c-chunk): thread (g, ci) takes key cluster
 // c0 + ci against query centroids g, g + QS_G, ...  Bounds stored [d][32]
 // (conflict-free), centroids [Cq][d] (broadcast within a warp).
 __global__ void __launch_bounds__(SEL_THREADS) k_quest_scores(SelectArgs a) {
@@ -39,13 +41,18 @@ __global__ void __launch_bounds__(SEL_THREADS) k_quest_scores(SelectArgs a) {
     const int nk = a.n_k[h];
     if (c0 >= nk) return;
     const int nc = min(QS_C, nk - c0);
+    const bool mean = a.score_mode == 1;
     for (int i = tid; i < a.d * QS_C; i += SEL_THREADS) {
         const int ci = i / a.d, k = i % a.d;  // coalesced over k
         float mx = 0.f, mn = 0.f;
         if (ci < nc) {
             const int64_t o = ((int64_t)h * a.Ccap + c0 + ci) * a.d + k;
-            mx = bf2f(a.kmax[o]);
-            mn = bf2f(a.kmin[o]);
+            if (mean) {
+                mx = mn = a.cent_k[o];  // the mean-based ablation: q_d mu_d
+            } else {
+                mx = bf2f(a.kmax[o]);
+                mn = bf2f(a.kmin[o]);
+            }
         }
         kx[k * QS_C + ci] = mx;
         kn[k * QS_C + ci] = mn;

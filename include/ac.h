@@ -85,7 +85,10 @@ typedef struct ac_config {
                             1: m_t = min(|U|, max(1, ceil(m0 |U| / L)))           */
     uint64_t seed;       /* seeds the initial centres of step 0                   */
     float scale;         /* softmax scale; 0 selects 1/sqrt(d)                    */
-    int32_t reserved1;   /* must be 0                                             */
+    int32_t score_mode;  /* cluster scores before the top-k (Algorithm 3 line 9):
+                            0: the Eq. (1) TensorQuest bound (the method);
+                            1: mean-based, q . mu with mu the key cluster's centre
+                               (the "w/o Quest" ablation of Sec. 4.4, Table 4)    */
 } ac_config;
 
 typedef struct ac_ctx ac_ctx;

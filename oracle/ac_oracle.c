@@ -542,6 +542,27 @@ void or_quest(const float *qc, int nq, int d, const float *kmax, const float *km
     }
 }
 
+/* The mean-based baseline of the TensorQuest ablation (Sec. 4.4, Table 4,
+ * "w/o Quest"): S[qc, kc] = sum_d q_d * mu_d with mu the centre (mean) of the
+ * key cluster, summed over d in order in fp32; empty clusters -inf.  Reading:
+ * "mean-based" scores the cluster by its centre in place of the Eq. (1) bound. */
+void or_mean_scores(const float *qc, int nq, int d, const float *cent, const int32_t *counts, int nk,
+                    float *S)
+{
+    for (int a = 0; a < nq; ++a) {
+        const float *q = qc + (int64_t)a * d;
+        for (int c = 0; c < nk; ++c) {
+            if (counts[c] == 0) {
+                S[(int64_t)a * nk + c] = -INFINITY;
+                continue;
+            }
+            float s = 0.0f;
+            for (int k = 0; k < d; ++k) s = s + q[k] * cent[(int64_t)c * d + k];
+            S[(int64_t)a * nk + c] = s;
+        }
+    }
+}
+
 /* How many key clusters each query cluster keeps.  The pages give "TopK 64"
  * (App. A.5) with no rounding rule.  Reading: topk > 0 is a count; topk < 0
  * is -permille of n_k, k = ceil(permille * n_k / 1000); the result is clamped

@@ -93,6 +93,7 @@ class Params:
     iters_warm: int = 2
     seed: int = 1234
     stage_rule: int = 0
+    score_mode: int = 0   # 0: Eq. (1) bound; 1: mean-based scores (the "w/o Quest" ablation)
 
     @property
     def ccap(self) -> int:
@@ -289,6 +290,18 @@ def quest(qc: np.ndarray, kmax: np.ndarray, kmin: np.ndarray, counts: np.ndarray
     return S
 
 
+def mean_scores(qc: np.ndarray, cent: np.ndarray, counts: np.ndarray) -> np.ndarray:
+    """Mean-based scores of one head (Sec. 4.4 Table 4 "w/o Quest"): qc [nq, d],
+    key-cluster centres cent [nk, d] -> S [nq, nk]."""
+    qc = _c(qc, np.float32)
+    nq, d = qc.shape
+    nk = cent.shape[0]
+    S = np.empty((nq, nk), np.float32)
+    lib().or_mean_scores(_p(qc), ctypes.c_int(nq), ctypes.c_int(d), _p(_c(cent, np.float32)),
+                         _p(_c(counts, np.int32)), ctypes.c_int(nk), _p(S))
+    return S
+
+
 def topk(S: np.ndarray, k: int) -> np.ndarray:
     S = _c(S, np.float32)
     nq, nk = S.shape
@@ -297,14 +310,19 @@ def topk(S: np.ndarray, k: int) -> np.ndarray:
     return sel
 
 
-def score_select(Cq: np.ndarray, st: KStats, n_k: np.ndarray, topk_param: int):
-    """Per head: S = Eq.(1) over the n_k clusters, k = topk_count, Sel [Cq, k].
-    Returns (list of S [Cq, n_k], list of Sel, k per head)."""
+def score_select(Cq: np.ndarray, st: KStats, n_k: np.ndarray, topk_param: int, score_mode: int = 0,
+                 Ck: np.ndarray | None = None):
+    """Per head: S = Eq.(1) (score_mode 0) or the mean-based scores against the
+    key centres Ck [BH, Ccap, d] (score_mode 1) over the n_k clusters,
+    k = topk_count, Sel [Cq, k].  Returns (list of S [Cq, n_k], list of Sel, k per head)."""
     Ss, sels, ks = [], [], []
     for h in range(Cq.shape[0]):
         nk = int(n_k[h])
         cnt = st.counts[h, :nk]
-        S = quest(Cq[h], st.kmax[h, :nk], st.kmin[h, :nk], cnt)
+        if score_mode == 1:
+            S = mean_scores(Cq[h], Ck[h, :nk], cnt)
+        else:
+            S = quest(Cq[h], st.kmax[h, :nk], st.kmin[h, :nk], cnt)
         k = topk_count(topk_param, nk, int((cnt > 0).sum()))
         Ss.append(S)
         sels.append(topk(S, k))
@@ -370,7 +388,7 @@ def layer(Q16, K16, V16, p: Params, warm_from: LayerResult | None = None,
         lq, Cq, cq = cluster_q(Q16, p, init=warm_from.Cq, iters=p.iters_warm)
         kc = cluster_k_warm(K16, p, warm_from.kc)
     st = key_stats(K16, kc)
-    S, sel, k = score_select(Cq, st, kc.n_k, p.topk)
+    S, sel, k = score_select(Cq, st, kc.n_k, p.topk, p.score_mode, kc.C)
     O = None
     if attention:
         r = np.arange(L) if rows is None else np.asarray(rows)

@@ -356,6 +356,43 @@ def test_quest_is_upper_bound_and_tensor_form():
     assert np.allclose(S1[:, 0], q1.astype(np.float64) @ k1[0].astype(np.float64), rtol=1e-5, atol=1e-5)
 
 
+def test_mean_scores_hand_example():
+    """The "w/o Quest" ablation (Sec. 4.4, Table 4): the score of a key cluster
+    is q . mu with mu its centre; worked by hand in binary fractions (exact in
+    fp32): q = [1, -2, 0.5], mu = [0.5, 0.25, -1] -> 0.5 - 0.5 - 0.5 = -0.5;
+    an empty cluster scores -inf."""
+    q = np.array([[1.0, -2.0, 0.5]], np.float32)
+    mu = np.array([[0.5, 0.25, -1.0], [3.0, 3.0, 3.0]], np.float32)
+    S = orc.mean_scores(q, mu, np.array([4, 0], np.int32))
+    assert S[0, 0] == -0.5 and np.isneginf(S[0, 1])
+
+
+def test_mean_scores_below_quest_and_equal_for_single_members():
+    """mu_d lies between the members' min and max in every dimension, so
+    q_d mu_d <= max(q_d Kmax_d, q_d Kmin_d) and the mean score never exceeds
+    Eq. (1) (up to the rounding of the fp32 mean); a single-member cluster has
+    mu = Kmax = Kmin, where the two scores are the same fp32 sum."""
+    cfg = synth.CONFIGS[1]
+    Q, K, _ = synth.make_layer(cfg, heads=[0])
+    p = orc.Params.from_layer_config(cfg)
+    kc = orc.cluster_k_multistage(K[0], p)
+    st = orc.key_stats(K[0], kc)
+    nk = int(kc.n_k[0])
+    _, qh = orc.qnorm(Q[0, 0][:300])
+    cnt = st.counts[0, :nk]
+    Sq = orc.quest(qh, st.kmax[0, :nk], st.kmin[0, :nk], cnt)
+    Sm = orc.mean_scores(qh, kc.C[0, :nk], cnt)
+    ne = cnt > 0
+    assert np.isneginf(Sm[:, ~ne]).all() and np.isfinite(Sm[:, ne]).all()
+    scale = np.abs(qh).astype(np.float64) @ np.maximum(np.abs(st.kmax[0, :nk]), np.abs(st.kmin[0, :nk])).T
+    assert (Sm[:, ne] <= Sq[:, ne] + 1e-6 * scale[:, ne]).all()
+    # scores differ where clusters have several members
+    assert (Sm[:, cnt > 1] < Sq[:, cnt > 1]).mean() > 0.9
+    X = synth.bf16_bits_to_f32(K[0, 0][:40])
+    one = np.ones(40, np.int32)
+    assert np.array_equal(orc.mean_scores(qh, X, one), orc.quest(qh, X, X, one))
+
+
 def test_topk_bruteforce_with_ties_and_empties():
     rng = np.random.default_rng(9)
     S = rng.integers(0, 6, size=(20, 30)).astype(np.float32)

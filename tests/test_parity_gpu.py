@@ -38,6 +38,21 @@ def test_tiny_layer_step0_end_to_end():
     lay.close()
 
 
+def test_mean_score_ablation_end_to_end():
+    """score_mode 1 (the "w/o Quest" ablation, Sec. 4.4 Table 4): key clusters
+    scored by q . centre; scores, selections and outputs against the oracle."""
+    cfg = synth.CONFIGS[1]
+    Q, K, V = synth.make_layer(cfg)
+    p = _params(cfg, score_mode=1)
+    r = orc.layer(_flat(Q), _flat(K), _flat(V), p)
+    lay, O, gs = run_gpu_layer(Q, K, V, p)
+    compare_layer(gs, r, p, O)
+    # the ablation changes what is kept
+    r0 = orc.layer(_flat(Q), _flat(K), _flat(V), _params(cfg), attention=False)
+    assert any(not np.array_equal(a, b) for a, b in zip(r.sel, r0.sel))
+    lay.close()
+
+
 def test_tiny_layer_warm_chain():
     """Step 0 then two warm-started steps on perturbed tokens (Sec. 3.2.2)."""
     cfg = synth.CONFIGS[1]
