@@ -503,6 +503,8 @@ void free_all(ac_ctx *c) {
         for (int i = 0; i < 4; ++i)
             if (c->abuf[b][i]) cudaFree(c->abuf[b][i]);
         if (c->ev_in[b]) cudaEventDestroy(c->ev_in[b]);
+        if (c->ev_inq[b]) cudaEventDestroy(c->ev_inq[b]);
+        if (c->ev_ink[b]) cudaEventDestroy(c->ev_ink[b]);
         if (c->ev_comp[b]) cudaEventDestroy(c->ev_comp[b]);
         if (c->ev_out[b]) cudaEventDestroy(c->ev_out[b]);
     }
@@ -763,19 +765,21 @@ ac_status ac_sparse_attn(ac_ctx *c, const uint16_t *Q, const uint16_t *K, const 
                             reinterpret_cast<const bf16 *>(V), reinterpret_cast<bf16 *>(O), (cudaStream_t)stream);
 }
 
-ac_status ac_layer_forward(ac_ctx *c, const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O,
-                           int32_t warm, ac_stage_times *times, void *stream) {
-    if (!c || !Q || !K || !V || !O) return fail(c, AC_ERR_INVALID_ARG, "ac_layer_forward: NULL argument");
-    if (warm && !c->have_state) return fail(c, AC_ERR_STATE, "warm step before any step 0");
-    cudaStream_t s = (cudaStream_t)stream;
+namespace {
+// The layer's steps on stream s; each of wq, wk, wv (nullable) is an event the
+// stream waits for before the first step that reads Q, K or V respectively.
+ac_status layer_steps(ac_ctx *c, const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O, int32_t warm,
+                      ac_stage_times *times, cudaStream_t s, cudaEvent_t wq, cudaEvent_t wk, cudaEvent_t wv) {
     const bf16 *Qb = reinterpret_cast<const bf16 *>(Q), *Kb = reinterpret_cast<const bf16 *>(K),
                *Vb = reinterpret_cast<const bf16 *>(V);
     ac_status st;
     c->timing = times != nullptr;
     if (times) CK(cudaEventRecord(c->ev[0], s), "event");
+    if (wq) CK(cudaStreamWaitEvent(s, wq, 0), "wait Q");
     st = cluster_q_impl(c, Qb, warm ? c->cent_q : nullptr, warm ? c->cfg.iters_warm : c->cfg.iters_q, s);
     if (st != AC_OK) return st;
     if (times) CK(cudaEventRecord(c->ev[1], s), "event");
+    if (wk) CK(cudaStreamWaitEvent(s, wk, 0), "wait K");
     st = warm ? cluster_k_warm(c, Kb, s) : cluster_k_step0(c, Kb, s);
     if (st != AC_OK) return st;
     if (times) CK(cudaEventRecord(c->ev[2], s), "event");
@@ -783,7 +787,19 @@ ac_status ac_layer_forward(ac_ctx *c, const uint16_t *Q, const uint16_t *K, cons
     if (times) CK(cudaEventRecord(c->ev[3], s), "event");
     if ((st = score_select_impl(c, 0, s)) != AC_OK) return st;
     if (times) CK(cudaEventRecord(c->ev[4], s), "event");
+    if (wv) CK(cudaStreamWaitEvent(s, wv, 0), "wait V");
     if ((st = sparse_attn_impl(c, Qb, Kb, Vb, reinterpret_cast<bf16 *>(O), s)) != AC_OK) return st;
+    return AC_OK;
+}
+}  // namespace
+
+ac_status ac_layer_forward(ac_ctx *c, const uint16_t *Q, const uint16_t *K, const uint16_t *V, uint16_t *O,
+                           int32_t warm, ac_stage_times *times, void *stream) {
+    if (!c || !Q || !K || !V || !O) return fail(c, AC_ERR_INVALID_ARG, "ac_layer_forward: NULL argument");
+    if (warm && !c->have_state) return fail(c, AC_ERR_STATE, "warm step before any step 0");
+    cudaStream_t s = (cudaStream_t)stream;
+    ac_status st = layer_steps(c, Q, K, V, O, warm, times, s, nullptr, nullptr, nullptr);
+    if (st != AC_OK) return st;
     if (times) CK(cudaEventRecord(c->ev[5], s), "event");
     c->have_state = true;
     if (times) {
@@ -907,6 +923,8 @@ ac_status ac_layer_forward_host_async(ac_ctx *c, const uint16_t *hQ, const uint1
                 }
         for (int b = 0; b < 2; ++b) {
             CK(cudaEventCreateWithFlags(&c->ev_in[b], cudaEventDisableTiming), "event");
+            CK(cudaEventCreateWithFlags(&c->ev_inq[b], cudaEventDisableTiming), "event");
+            CK(cudaEventCreateWithFlags(&c->ev_ink[b], cudaEventDisableTiming), "event");
             CK(cudaEventCreateWithFlags(&c->ev_comp[b], cudaEventDisableTiming), "event");
             CK(cudaEventCreateWithFlags(&c->ev_out[b], cudaEventDisableTiming), "event");
         }
@@ -916,15 +934,20 @@ ac_status ac_layer_forward_host_async(ac_ctx *c, const uint16_t *hQ, const uint1
     const int b = (int)(c->async_calls & 1);
     uint16_t **buf = c->abuf[b];
     if (c->async_calls >= 2) CK(cudaStreamWaitEvent(c->s_in, c->ev_comp[b], 0), "wait layer");
+    // Q, K and V land one after the other; the layer starts on Q as soon as it
+    // has landed (the query clustering overlaps the copies of K and V)
     CK(cudaMemcpyAsync(buf[0], hQ, n * 2, cudaMemcpyHostToDevice, c->s_in), "h2d Q");
+    CK(cudaEventRecord(c->ev_inq[b], c->s_in), "event");
     CK(cudaMemcpyAsync(buf[1], hK, n * 2, cudaMemcpyHostToDevice, c->s_in), "h2d K");
+    CK(cudaEventRecord(c->ev_ink[b], c->s_in), "event");
     CK(cudaMemcpyAsync(buf[2], hV, n * 2, cudaMemcpyHostToDevice, c->s_in), "h2d V");
     CK(cudaEventRecord(c->ev_in[b], c->s_in), "event");
-    CK(cudaStreamWaitEvent(s, c->ev_in[b], 0), "wait inputs");
     if (c->async_calls >= 2) CK(cudaStreamWaitEvent(s, c->ev_out[b], 0), "wait output copy");
     ++c->async_calls;
-    ac_status st = ac_layer_forward(c, buf[0], buf[1], buf[2], buf[3], warm, nullptr, stream);
+    ac_status st = layer_steps(c, buf[0], buf[1], buf[2], buf[3], warm, nullptr, s, c->ev_inq[b], c->ev_ink[b],
+                               c->ev_in[b]);
     if (st != AC_OK) return st;
+    c->have_state = true;
     CK(cudaEventRecord(c->ev_comp[b], s), "event");
     CK(cudaStreamWaitEvent(c->s_out, c->ev_comp[b], 0), "wait layer");
     CK(cudaMemcpyAsync(hO, buf[3], n * 2, cudaMemcpyDeviceToHost, c->s_out), "d2h O");

@@ -106,6 +106,7 @@ struct ac_ctx {
     uint16_t *abuf[2][4];
     cudaStream_t s_in, s_out;
     cudaEvent_t ev_in[2], ev_comp[2], ev_out[2];
+    cudaEvent_t ev_inq[2], ev_ink[2];  // Q landed, K landed (ev_in: V, the last)
     long long async_calls;
 
     uint32_t *err;      // device error word

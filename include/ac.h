@@ -195,7 +195,8 @@ AC_API ac_status ac_layer_forward_host(ac_ctx *ctx, const uint16_t *hQ, const ui
  * context-owned copy stream), the layer (on `stream`) and the output copy (on a
  * second copy stream) and returns.  Consecutive calls pipeline: call n's input
  * copy overlaps call n - 1's layer and its output copy call n + 1's layer
- * (two context-owned device staging sets, used alternately).
+ * (two context-owned device staging sets, used alternately); within a call
+ * the query clustering starts once Q has landed, while K and V still copy.
  * Ownership: hQ, hK, hV must stay unchanged, and hO must not be read, until
  * the call is complete: after ac_synchronize(ctx, stream) returns, or once
  * `stream` has passed an ac_join(ctx, stream).  Host buffers should be pinned
