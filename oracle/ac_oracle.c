@@ -662,6 +662,93 @@ void or_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V, 
     }
 }
 
+/* Per key cluster c < nk: count and mean of the member rows (bf16 -> fp32),
+ * members summed in ascending token order in fp32 and divided by the count,
+ * as the Lloyd update does; empty clusters get count 0 and mean 0. */
+void or_cluster_means(const uint16_t *X, int L, int d, const int32_t *labels, int nk, float *mean,
+                      int32_t *count)
+{
+    for (int c = 0; c < nk; ++c) count[c] = 0;
+    for (int64_t i = 0; i < (int64_t)nk * d; ++i) mean[i] = 0.0f;
+    for (int64_t j = 0; j < L; ++j) {
+        const int c = labels[j];
+        if (c < 0 || c >= nk) continue;
+        count[c] += 1;
+        for (int t = 0; t < d; ++t) mean[(int64_t)c * d + t] = mean[(int64_t)c * d + t] + bf2f(X[j * d + t]);
+    }
+    for (int c = 0; c < nk; ++c)
+        if (count[c] > 0)
+            for (int t = 0; t < d; ++t) mean[(int64_t)c * d + t] = mean[(int64_t)c * d + t] / (float)count[c];
+}
+
+/* Centroid ("stripe-mean") compensation of the clusters a query cluster does
+ * not select (ClusterAttention Sec. 1.2, Eq. (5)-(6)): for query row i of
+ * query cluster qc, the keys of the selected clusters enter the softmax as in
+ * or_attention_rows, and every other non-empty key cluster c < nk enters as
+ * one pseudo-token with key kbar_c, value vbar_c and multiplicity |c|, i.e.
+ * with weight |c| exp(scale q . kbar_c).  Dense units: every key, nothing to
+ * compensate.  fp64. */
+void or_attention_rows_comp(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int L, int d,
+                            const int32_t *labels_q, const int32_t *labels_k, const int32_t *sel,
+                            int32_t k, int dense, double scale, const int64_t *rows, int64_t nrows,
+                            int nk, const int32_t *counts, const double *kbar, const double *vbar,
+                            double *out)
+{
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t i = rows[r];
+        double *s = (double *)malloc((size_t)L * sizeof(double));
+        double *sc = (double *)malloc((size_t)(nk > 0 ? nk : 1) * sizeof(double));
+        char *chosen = (char *)calloc((size_t)(nk > 0 ? nk : 1), 1);
+        double *q = (double *)malloc((size_t)d * sizeof(double));
+        for (int t = 0; t < d; ++t) q[t] = (double)bf2f(Q[i * d + t]);
+        if (dense) {
+            for (int c = 0; c < nk; ++c) chosen[c] = 1;
+        } else {
+            const int32_t *my = sel + (int64_t)labels_q[i] * k;
+            for (int a = 0; a < k; ++a)
+                if (my[a] >= 0 && my[a] < nk) chosen[my[a]] = 1;
+        }
+        double mx = -INFINITY;
+        for (int64_t j = 0; j < L; ++j) {
+            const int c = labels_k[j];
+            if (!(dense || (c >= 0 && c < nk && chosen[c]))) continue;
+            double acc = 0.0;
+            for (int t = 0; t < d; ++t) acc += q[t] * (double)bf2f(K[j * d + t]);
+            s[j] = acc * scale;
+            if (s[j] > mx) mx = s[j];
+        }
+        for (int c = 0; c < nk; ++c) {
+            if (chosen[c] || counts[c] == 0) continue;
+            double acc = 0.0;
+            for (int t = 0; t < d; ++t) acc += q[t] * kbar[(int64_t)c * d + t];
+            sc[c] = acc * scale + log((double)counts[c]);
+            if (sc[c] > mx) mx = sc[c];
+        }
+        double l = 0.0;
+        double *o = out + r * d;
+        for (int t = 0; t < d; ++t) o[t] = 0.0;
+        for (int64_t j = 0; j < L; ++j) {
+            const int c = labels_k[j];
+            if (!(dense || (c >= 0 && c < nk && chosen[c]))) continue;
+            double p = exp(s[j] - mx);
+            l += p;
+            for (int t = 0; t < d; ++t) o[t] += p * (double)bf2f(V[j * d + t]);
+        }
+        for (int c = 0; c < nk; ++c) {
+            if (chosen[c] || counts[c] == 0) continue;
+            double p = exp(sc[c] - mx);
+            l += p;
+            for (int t = 0; t < d; ++t) o[t] += p * vbar[(int64_t)c * d + t];
+        }
+        for (int t = 0; t < d; ++t) o[t] /= l;
+        free(s);
+        free(sc);
+        free(chosen);
+        free(q);
+    }
+}
+
 /* Dense softmax weights of one query row over all L keys, fp64 (used by the
  * error-split self-check, ClusterAttention Sec. 1.2 Eq. (1)-(4)). */
 void or_dense_weights(const uint16_t *q16, const uint16_t *K, int L, int d, double scale, double *w)

@@ -351,6 +351,41 @@ def attention_rows(Q16h, K16h, V16h, labels_q, labels_k, sel, dense: bool, rows,
     return out
 
 
+def cluster_means(X16h: np.ndarray, labels: np.ndarray, nk: int):
+    """Member means of the clusters c < nk of one head (fp32, ascending token
+    order, as the Lloyd update) and their counts."""
+    X16h = _c(X16h, np.uint16)
+    L, d = X16h.shape
+    mean = np.empty((max(nk, 1), d), np.float32)
+    cnt = np.empty(max(nk, 1), np.int32)
+    lib().or_cluster_means(_p(X16h), ctypes.c_int(L), ctypes.c_int(d), _p(_c(labels, np.int32)),
+                           ctypes.c_int(nk), _p(mean), _p(cnt))
+    return mean[:nk], cnt[:nk]
+
+
+def attention_rows_comp(Q16h, K16h, V16h, labels_q, labels_k, sel, dense: bool, rows, nk: int,
+                        counts, kbar, vbar, scale: float | None = None) -> np.ndarray:
+    """attention_rows with the unselected clusters compensated by their centroids
+    (ClusterAttention Sec. 1.2 Eq. (5)-(6)): kbar / vbar [nk, d] (fp64), counts [nk]."""
+    Q16h = _c(Q16h, np.uint16)
+    K16h = _c(K16h, np.uint16)
+    L, d = K16h.shape
+    rows = _c(rows, np.int64)
+    out = np.empty((rows.size, d), np.float64)
+    sc = 1.0 / np.sqrt(d) if scale is None else scale
+    if sel is None:
+        sel = np.zeros((1, 1), np.int32)
+        dense = True
+    sel = _c(sel, np.int32)
+    lib().or_attention_rows_comp(_p(Q16h), _p(K16h), _p(_c(V16h, np.uint16)), ctypes.c_int(L), ctypes.c_int(d),
+                                 _p(_c(labels_q, np.int32)), _p(_c(labels_k, np.int32)), _p(sel),
+                                 ctypes.c_int32(sel.shape[1]), ctypes.c_int(1 if dense else 0),
+                                 ctypes.c_double(sc), _p(rows), ctypes.c_int64(rows.size), ctypes.c_int(nk),
+                                 _p(_c(counts, np.int32)), _p(_c(kbar, np.float64)), _p(_c(vbar, np.float64)),
+                                 _p(out))
+    return out
+
+
 def dense_weights(q16: np.ndarray, K16h: np.ndarray, scale: float | None = None) -> np.ndarray:
     K16h = _c(K16h, np.uint16)
     L, d = K16h.shape

@@ -393,6 +393,108 @@ def test_mean_scores_below_quest_and_equal_for_single_members():
     assert np.array_equal(orc.mean_scores(qh, X, one), orc.quest(qh, X, X, one))
 
 
+def _comp_case(seed, L=240, d=8, nk=12, dup=False):
+    """A small head with random bf16 Q, K, V, random key clusters (or clusters
+    of identical members when dup), one query cluster selecting 3 of them."""
+    rng = np.random.default_rng(seed)
+    labels_k = rng.integers(0, nk, L).astype(np.int32)
+    labels_k[:nk] = np.arange(nk)  # every cluster non-empty
+    if dup:
+        proto_k = rng.normal(size=(nk, d)) * 0.8
+        proto_v = rng.normal(size=(nk, d))
+        Kf, Vf = proto_k[labels_k], proto_v[labels_k]
+    else:
+        Kf, Vf = rng.normal(size=(L, d)) * 0.8, rng.normal(size=(L, d))
+    Qf = rng.normal(size=(L, d))
+    Q16, K16, V16 = (synth.f32_to_bf16_bits(x.astype(np.float32)) for x in (Qf, Kf, Vf))
+    sel = np.array([[1, 4, 7]], np.int32)
+    return Q16, K16, V16, labels_k, sel
+
+
+def test_compensation_error_identity():
+    """ClusterAttention Sec. 1.2 Eq. (5): with w the dense softmax weights,
+    w_bar_c the mean weight of cluster c, w_hat_c = exp(s(k_bar_c)) / Z the
+    centroid's weight, delta_c = w_bar_c - w_hat_c, Cov_c the weight-value
+    covariance of c and d_hat the compensated partition sum (relative to Z),
+    o - o_hat = (1 / d_hat) sum_c |c| (delta_c (v_bar_c - o) + Cov_c) over
+    the unselected clusters, exactly (here to fp64 rounding).  k_bar may be
+    any point; v_bar must be the member mean."""
+    Q16, K16, V16, labels_k, sel = _comp_case(3)
+    L, d = K16.shape
+    nk = 12
+    Kf, Vf, Qf = (synth.bf16_bits_to_f32(x).astype(np.float64) for x in (K16, V16, Q16))
+    cnt = np.bincount(labels_k, minlength=nk).astype(np.int32)
+    vbar = np.stack([Vf[labels_k == c].mean(0) for c in range(nk)])
+    kbar = np.stack([Kf[labels_k == c].mean(0) for c in range(nk)]) + 0.05  # any point will do
+    rows = np.arange(0, L, 17)
+    lq = np.zeros(L, np.int32)
+    o = orc.attention_rows(Q16, K16, V16, lq, labels_k, None, True, rows)
+    oh = orc.attention_rows_comp(Q16, K16, V16, lq, labels_k, sel, False, rows, nk, cnt, kbar, vbar)
+    sc = 1.0 / np.sqrt(d)
+    excl = [c for c in range(nk) if c not in sel[0]]
+    for r, i in enumerate(rows):
+        s = Kf @ Qf[i] * sc
+        Z = np.exp(s).sum()
+        w = np.exp(s) / Z
+        dhat = w[np.isin(labels_k, sel[0])].sum()
+        rhs = np.zeros(d)
+        for c in excl:
+            m = labels_k == c
+            wb = w[m].mean()
+            wh = np.exp(kbar[c] @ Qf[i] * sc) / Z
+            dhat += cnt[c] * wh
+            cov = ((w[m] - wb)[:, None] * (Vf[m] - vbar[c])).mean(0)
+            rhs += cnt[c] * ((wb - wh) * (vbar[c] - o[r]) + cov)
+        rhs /= dhat
+        assert np.allclose(o[r] - oh[r], rhs, rtol=0, atol=1e-12), (i, np.abs(o[r] - oh[r] - rhs).max())
+    # the unselected mass is not negligible here: compensation changes the output
+    osel = orc.attention_rows(Q16, K16, V16, lq, labels_k, sel, False, rows)
+    assert np.abs(osel - oh).max() > 1e-3
+
+
+def test_compensation_exact_for_identical_members_and_all_selected():
+    """Clusters of identical members: delta_c = 0 and Cov_c = 0, so the
+    compensated output equals dense attention; with every cluster selected
+    there is nothing to compensate."""
+    Q16, K16, V16, labels_k, sel = _comp_case(5, dup=True)
+    L, d = K16.shape
+    nk = 12
+    km, cnt = orc.cluster_means(K16, labels_k, nk)
+    vm, _ = orc.cluster_means(V16, labels_k, nk)
+    rows = np.arange(0, L, 11)
+    lq = np.zeros(L, np.int32)
+    o = orc.attention_rows(Q16, K16, V16, lq, labels_k, None, True, rows)
+    oh = orc.attention_rows_comp(Q16, K16, V16, lq, labels_k, sel, False, rows, nk, cnt, km, vm)
+    assert np.allclose(oh, o, rtol=0, atol=1e-12)
+    Q16, K16, V16, labels_k, _ = _comp_case(6)
+    km, cnt = orc.cluster_means(K16, labels_k, nk)
+    vm, _ = orc.cluster_means(V16, labels_k, nk)
+    every = np.arange(nk, dtype=np.int32)[None]
+    o = orc.attention_rows(Q16, K16, V16, lq, labels_k, every, False, rows)
+    oh = orc.attention_rows_comp(Q16, K16, V16, lq, labels_k, every, False, rows, nk, cnt, km, vm)
+    assert np.array_equal(o, oh)
+
+
+def test_cluster_means_are_member_order_fp32_sums():
+    """or_cluster_means follows the Lloyd update's rule (fp32 sums in ascending
+    token order, then one division); a consistency check of that rule, not a
+    pin: counts, the order-defined fp32 values, empty clusters 0."""
+    rng = np.random.default_rng(2)
+    X16 = synth.f32_to_bf16_bits(rng.normal(size=(500, 16)).astype(np.float32))
+    lab = rng.integers(0, 9, 500).astype(np.int32)
+    lab[lab == 4] = 5  # cluster 4 empty
+    mean, cnt = orc.cluster_means(X16, lab, 9)
+    Xf = synth.bf16_bits_to_f32(X16)
+    for c in range(9):
+        acc = np.zeros(16, np.float32)
+        for j in np.nonzero(lab == c)[0]:
+            acc = (acc + Xf[j]).astype(np.float32)
+        n = int((lab == c).sum())
+        assert cnt[c] == n
+        want = (acc / np.float32(n)).astype(np.float32) if n else np.zeros(16, np.float32)
+        assert np.array_equal(mean[c], want)
+
+
 def test_topk_bruteforce_with_ties_and_empties():
     rng = np.random.default_rng(9)
     S = rng.integers(0, 6, size=(20, 30)).astype(np.float32)
