@@ -386,6 +386,73 @@ def attention_rows_comp(Q16h, K16h, V16h, labels_q, labels_k, sel, dense: bool, 
     return out
 
 
+def tail_merge(labels_q: np.ndarray, masks: np.ndarray, b: int = 128):
+    """Two-stage tail merging of one head's query clusters (iCATS, "tail merging
+    strategy" and its worked example), for a kernel that runs query clusters in
+    b-row tiles.  labels_q [L]: query cluster of each token; masks [Cq, nk] bool:
+    the key clusters each query cluster attends to.
+
+    Stage 1 (lossless): query clusters with identical masks form one group,
+    owned by its lowest-index member; a group's tokens are its members' tokens,
+    member by member in cluster order, each in ascending token order.
+    Stage 2 (tail remap): among the groups whose size has a tail
+    t = size mod b > 0, each finds its nearest neighbour by the Hamming
+    distance of the masks (ties to the lower index); two groups that are each
+    other's nearest neighbour and whose tails fit one tile (t_i + t_j <= b)
+    pair up: the higher-index group j hands its last t_j tokens to the
+    lower-index group i, and i's mask becomes the union of both.
+    Readings: the pages do not say which cluster of a pair absorbs the other's
+    tail (their example is consistent with either); here the lower index does.
+
+    Returns (owner [L] int32: the group whose mask each token attends with,
+    new_masks [Cq, nk] bool, groups {owner: token list in group order},
+    pairs [(i, j, moved)])."""
+    labels_q = np.asarray(labels_q)
+    masks = np.asarray(masks, bool)
+    Cq = masks.shape[0]
+    members = [np.nonzero(labels_q == c)[0] for c in range(Cq)]
+    # stage 1: identical masks
+    rep = list(range(Cq))
+    for c in range(Cq):
+        if members[c].size == 0:
+            continue
+        for r in range(c):
+            if members[r].size and rep[r] == r and np.array_equal(masks[r], masks[c]):
+                rep[c] = r
+                break
+    groups = {}
+    for c in range(Cq):
+        if members[c].size:
+            groups.setdefault(rep[c], []).extend(members[c].tolist())
+    new_masks = masks.copy()
+    # stage 2: mutual nearest neighbours among the groups with a tail
+    tails = {g: len(t) % b for g, t in groups.items() if len(t) % b > 0}
+    keys = sorted(tails)
+    nn = {}
+    for g in keys:
+        best, bd = None, None
+        for h in keys:
+            if h == g:
+                continue
+            dist = int(np.count_nonzero(masks[g] != masks[h]))
+            if bd is None or dist < bd:
+                best, bd = h, dist
+        nn[g] = best
+    pairs = []
+    for g in keys:
+        h = nn[g]
+        if h is not None and g < h and nn.get(h) == g and tails[g] + tails[h] <= b:
+            moved = groups[h][len(groups[h]) - tails[h]:]
+            groups[h] = groups[h][:len(groups[h]) - tails[h]]
+            groups[g] = groups[g] + moved
+            new_masks[g] = masks[g] | masks[h]
+            pairs.append((g, h, len(moved)))
+    owner = np.full(labels_q.shape[0], -1, np.int32)
+    for g, toks in groups.items():
+        owner[np.asarray(toks, np.int64)] = g
+    return owner, new_masks, groups, pairs
+
+
 def dense_weights(q16: np.ndarray, K16h: np.ndarray, scale: float | None = None) -> np.ndarray:
     K16h = _c(K16h, np.uint16)
     L, d = K16h.shape

@@ -495,6 +495,67 @@ def test_cluster_means_are_member_order_fp32_sums():
         assert np.array_equal(mean[c], want)
 
 
+def test_tail_merge_worked_example():
+    """The worked example of iCATS's tail merging (tests/golden/tail_merge_example.json):
+    query clusters #12 and #45 (210 and 180 tokens) attend to the same key
+    clusters and merge into #12 (390); #3 (300 tokens, tail 44) and #18 (170,
+    tail 42) are each other's nearest masks and 44 + 42 <= 128, so #18's last
+    42 tokens move to #3, whose mask becomes the union."""
+    g = _golden("tail_merge_example.json")
+    b = g["b"]
+    sizes = {3: 300, 12: 210, 18: 170, 45: 180}
+    nk = 8
+    masks = np.zeros((46, nk), bool)
+    masks[12, [0, 1]] = masks[45, [0, 1]] = True
+    masks[3, [2, 3, 4]] = True
+    masks[18, [2, 3, 5]] = True
+    rng = np.random.default_rng(4)
+    labels = np.concatenate([np.full(n, c, np.int32) for c, n in sizes.items()])
+    rng.shuffle(labels)
+    owner, new_masks, groups, pairs = orc.tail_merge(labels, masks, b)
+    s1 = g["stage1"]
+    assert len(groups[s1["merged_into"]]) == s1["merged_size"] == sum(s1["sizes"])
+    s2 = g["stage2"]
+    assert [sizes[c] % b for c in s2["clusters"]] == s2["tails"] and sum(s2["tails"]) == s2["tail_sum"] <= b
+    assert pairs == [(s2["tokens_moved_to"], s2["tokens_moved_from"], s2["moved"])]
+    last = np.nonzero(labels == s2["tokens_moved_from"])[0][-s2["moved"]:]
+    assert (owner[last] == s2["tokens_moved_to"]).all()
+    assert len(groups[3]) == 300 + 42 and len(groups[18]) == 128
+    assert np.array_equal(new_masks[3], masks[3] | masks[18])
+    # the 390-token group keeps its tail: its nearest mask (#3) pairs with #18
+    assert np.array_equal(new_masks[12], masks[12])
+
+
+def test_tail_merge_invariants():
+    """Every token keeps exactly one owner; tiles never increase; a token's key
+    set after merging contains its own cluster's; stage 1 changes no token's
+    key set; paired tails fit one tile and leave the donor aligned."""
+    rng = np.random.default_rng(12)
+    b, Cq, nk = 128, 24, 40
+    base = rng.random((8, nk)) < 0.2
+    masks = base[rng.integers(0, 8, Cq)] | (rng.random((Cq, nk)) < 0.03)
+    masks[5] = masks[2]
+    masks[9] = masks[2]
+    labels = rng.integers(0, Cq, 4000).astype(np.int32)
+    owner, new_masks, groups, pairs = orc.tail_merge(labels, masks, b)
+    assert (owner >= 0).all() and sorted(np.concatenate([np.asarray(t) for t in groups.values()])) == list(range(4000))
+    sizes = np.bincount(labels, minlength=Cq)
+    before = int(np.sum((sizes + b - 1) // b))
+    after = int(sum((len(t) + b - 1) // b for t in groups.values()))
+    assert after <= before
+    moved = set()
+    for i, j, n in pairs:
+        assert 0 < n < b and (len(groups[j]) % b) == 0
+        moved.update(np.nonzero(owner == i)[0].tolist())
+    for t in range(4000):
+        mine = masks[labels[t]]
+        assert (new_masks[owner[t]] >= mine).all()
+        if owner[t] not in [i for i, _, _ in pairs]:
+            assert np.array_equal(new_masks[owner[t]], mine)
+    # clusters 5 and 9 share cluster 2's mask: stage 1 folds them into 2
+    assert 2 in groups and 5 not in groups and 9 not in groups
+
+
 def test_topk_bruteforce_with_ties_and_empties():
     rng = np.random.default_rng(9)
     S = rng.integers(0, 6, size=(20, 30)).astype(np.float32)
