@@ -50,7 +50,7 @@ class ACConfig(ctypes.Structure):
                 ("tau_mode", ctypes.c_int32), ("tau_value", ctypes.c_float), ("topk", ctypes.c_int32),
                 ("iters_q", ctypes.c_int32), ("iters_k", ctypes.c_int32), ("iters_warm", ctypes.c_int32),
                 ("stage_rule", ctypes.c_int32), ("seed", ctypes.c_uint64), ("scale", ctypes.c_float),
-                ("score_mode", ctypes.c_int32)]
+                ("score_mode", ctypes.c_int32), ("tail_merge", ctypes.c_int32), ("reserved2", ctypes.c_int32)]
 
 
 class ACStageTimes(ctypes.Structure):

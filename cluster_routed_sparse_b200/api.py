@@ -59,11 +59,12 @@ class SparseLayer:
     def __init__(self, B: int, H: int, L: int, d: int, *, Cq: int, m0: int, n_max: int,
                  tau_mode: int, tau_value: float, topk: int, iters_q: int = 10,
                  iters_k: int = 10, iters_warm: int = 2, seed: int = 1234, scale: float = 0.0,
-                 stage_rule: int = 0, score_mode: int = 0):
+                 stage_rule: int = 0, score_mode: int = 0, tail_merge: int = 0):
         self.lib = _lib.load()
         self.B, self.H, self.L, self.d = B, H, L, d
         self.cfg = ACConfig(Cq, m0, n_max, tau_mode, float(tau_value), topk, iters_q, iters_k,
-                            iters_warm, stage_rule, seed & (2**64 - 1), float(scale), score_mode)
+                            iters_warm, stage_rule, seed & (2**64 - 1), float(scale), score_mode,
+                            tail_merge, 0)
         self.Cq, self.Ccap = Cq, n_max + m0
         h = ctypes.c_void_p()
         check(self.lib.ac_create(ctypes.byref(self.cfg), B, H, L, d, ctypes.byref(h)))

@@ -465,16 +465,26 @@ ac_status score_select_impl(ac_ctx *c, int topk, cudaStream_t s) {
     a.score_mode = c->cfg.score_mode;
     a.cent_k = c->cent_k;
     CK(launch_score_select(a, s), "score select");
+    if (c->cfg.tail_merge) {
+        TailMergeArgs t{c->sel, c->ksel, c->dense, c->labels_q, c->perm_q, c->offs_q, c->counts_q, c->counts_k,
+                        c->pgoff, c->ranges, c->rbox, c->nrange, c->nboxes, c->perm_qm, c->offs_qm, c->counts_qm,
+                        c->tm_scratch, c->tile_prefix, c->Cq, c->Ccap, c->BH, c->cfg.tail_merge, c->L};
+        CK(launch_tail_merge(t, s), "tail merge");
+    }
     return AC_OK;
 }
 
 ac_status sparse_attn_impl(ac_ctx *c, const bf16 *Q, const bf16 *K, const bf16 *V, bf16 *O, cudaStream_t s) {
-    CK(launch_permute_rows(Q, c->perm_q, c->Qp, c->L, c->d, c->BH, s), "permute q");
+    // with tail merging the query rows are laid out by group
+    const bool tm = c->cfg.tail_merge != 0;
+    const int *pq = tm ? c->perm_qm : c->perm_q, *oq = tm ? c->offs_qm : c->offs_q;
+    const int *cq = tm ? c->counts_qm : c->counts_q;
+    CK(launch_permute_rows(Q, pq, c->Qp, c->L, c->d, c->BH, s), "permute q");
     CK(launch_permute_kv_padded(K, V, c->perm_k, c->labels_k, c->offs_k, c->Ccap + 1, c->pgoff, c->Ccap, c->Kp, c->Vp,
                                 c->L, c->Lpad, c->d, c->BH, s),
        "permute k, v");
     CK(cudaMemsetAsync(c->counters, 0, 8 * sizeof(unsigned long long), s), "counters");
-    AttnArgs a{&c->tm_q, c->tm_kg, c->tm_vg, O, c->perm_q, c->offs_q, c->counts_q, c->tile_prefix, c->ranges,
+    AttnArgs a{&c->tm_q, c->tm_kg, c->tm_vg, O, pq, oq, cq, c->tile_prefix, c->ranges,
                c->nboxes, c->nrange, c->rbox, c->L, c->Lpad, c->Cq, c->Ccap, c->BH, c->d,
                (float)(c->scale * 1.4426950408889634), c->err, c->counters};
     if (c->timing) CK(cudaEventRecord(c->ev[6], s), "event");
@@ -491,7 +501,8 @@ void free_all(ac_ctx *c) {
                    c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->Qp, c->Kp, c->Vp,
                    c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err, c->chi_q, c->chi_k, c->cn,
                    c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats, c->rbox, c->pgoff, c->nrange,
-                   c->sort_scratch, c->cnp_k, c->rowsq_u, c->cent_st};
+                   c->sort_scratch, c->cnp_k, c->rowsq_u, c->cent_st, c->perm_qm, c->offs_qm, c->counts_qm,
+                   c->tm_scratch};
     for (void *p : dev)
         if (p) cudaFree(p);
     void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err};
@@ -529,7 +540,8 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     if (d != 64 && d != 128) return AC_ERR_UNSUPPORTED;
     if (cfg->Cq < 1 || cfg->Cq > L || cfg->m0 < 1 || cfg->m0 > L || cfg->n_max < 1 || cfg->iters_q < 0 ||
         cfg->iters_k < 0 || cfg->iters_warm < 0 || cfg->tau_mode < 0 || cfg->tau_mode > 2 || cfg->topk == 0 ||
-        cfg->stage_rule < 0 || cfg->stage_rule > 1 || (cfg->score_mode != 0 && cfg->score_mode != 1) || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
+        cfg->stage_rule < 0 || cfg->stage_rule > 1 || (cfg->score_mode != 0 && cfg->score_mode != 1) ||
+        cfg->tail_merge < 0 || cfg->tail_merge > 2 || cfg->reserved2 != 0 || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
         return AC_ERR_INVALID_ARG;
     if ((int64_t)B * H * L >= (int64_t)1 << 31) return AC_ERR_INVALID_ARG;
     if (cfg->tau_mode == AC_TAU_PERCENTILE && (cfg->tau_value < 1.f || cfg->tau_value > 1000.f))
@@ -621,6 +633,12 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->hstat, 2 * BH));
     A(dalloc(&c->rowsq_k, BH * Lz));
     A(dalloc(&c->rowsq_u, BH * Lz));
+    if (cfg->tail_merge) {
+        A(dalloc(&c->perm_qm, BH * Lz));
+        A(dalloc(&c->offs_qm, BH * (Cq + 1)));
+        A(dalloc(&c->counts_qm, BH * Cq));
+        A(dalloc(&c->tm_scratch, 4 * BH * Cq));
+    }
     A(dalloc(&c->cent_st, BH * (size_t)m0 * dz));
     A(dalloc(&c->cand, BH * Lz));
     A(dalloc(&c->amb_list, BH * Lz));

@@ -65,6 +65,11 @@ struct ac_ctx {
     int *nboxes;       // [BH*Cq]         8-row key boxes per query cluster
     int *rbox;         // [BH*Cq, Ccap+1] first box of each selected range (exclusive prefix)
     int *tile_prefix;  // [BH*Cq+1]       attention items (pairs of 128-query tiles), exclusive prefix
+    // tail merging (cfg.tail_merge != 0): the attention's query layout by group
+    int *perm_qm;      // [BH, L]   token of each row of Qp
+    int *offs_qm;      // [BH, Cq+1] first row of each group (owner cluster id)
+    int *counts_qm;    // [BH, Cq]  rows of each group (0: merged into another)
+    int *tm_scratch;   // [4, BH, Cq] owner, position in group, rows kept, base of handed rows
 
     // ---- tensor-core assignment (centres split into bf16 + remainder)
     int Cpad_q, CH_q, Cpad_k, CH_k;  // padded centre rows per unit, centres per chunk
@@ -267,6 +272,20 @@ struct SelectArgs {
     const float *cent_k = nullptr;  // [BH, Ccap, d] key centres (score_mode 1)
 };
 cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s);
+
+// Tail merging of the query tiles after the selection (see ac_config.tail_merge):
+// regroups the rows of Qp (perm_qm, offs_qm, counts_qm), rewrites the key
+// ranges of the clusters that take another's tail, and the attention items.
+struct TailMergeArgs {
+    const int *sel; const int *ksel; const uint8_t *dense;
+    const int *labels_q; const int *perm_q; const int *offs_q; const int *counts_q;
+    const int *counts_k; const int *pgoff;
+    int2 *ranges; int *rbox; int *nrange; int *nboxes;
+    int *perm_qm; int *offs_qm; int *counts_qm; int *scratch; int *tile_prefix;
+    int Cq, Ccap, BH, mode;
+    int64_t L;
+};
+cudaError_t launch_tail_merge(const TailMergeArgs &a, cudaStream_t s);
 
 struct AttnArgs {
     const CUtensorMap *tm_q, *tm_kg, *tm_vg;  // tm_kg / tm_vg: [4] box sizes

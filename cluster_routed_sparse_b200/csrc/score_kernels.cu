@@ -266,6 +266,194 @@ __global__ void __launch_bounds__(1024) k_tile_prefix(const int *counts_q, int n
     if (threadIdx.x == 0) prefix[n] = base_s;
 }
 
+// ------------------------------------------------------------------ tail merging
+// Query-tile tail merging (iCATS, "tail merging strategy"), one block per unit.
+// Stage 1: a query cluster joins the lowest-index non-empty cluster whose
+// selection equals its own (the same key clusters; in a dense unit every
+// cluster walks every key, so all join the first); a group's rows are its
+// members' rows, member by member in cluster order.  Stage 2 (mode 2, sparse
+// units): among the groups with a tail t = rows mod 128 > 0, each finds the
+// group whose selection differs from its own in the fewest key clusters
+// (ties to the lower index); two groups that are each other's choice and
+// whose tails fit one tile pair up: the higher index hands its last t rows to
+// the lower, whose key ranges become the union of both selections.
+constexpr int TM_TILE = 128;
+
+__device__ __forceinline__ bool tm_same(const int *a, const int *b, int k) {
+    for (int i = 0; i < k; ++i)
+        if (a[i] != b[i]) return false;
+    return true;
+}
+// |A \ B| + |B \ A| of two ascending lists of k entries
+__device__ __forceinline__ int tm_hamming(const int *a, const int *b, int k) {
+    int i = 0, j = 0, common = 0;
+    while (i < k && j < k) {
+        if (a[i] == b[j]) {
+            ++common;
+            ++i;
+            ++j;
+        } else if (a[i] < b[j]) {
+            ++i;
+        } else {
+            ++j;
+        }
+    }
+    return 2 * (k - common);
+}
+
+__global__ void __launch_bounds__(SEL_THREADS) k_tail_merge_plan(TailMergeArgs a) {
+    extern __shared__ int tm_sm[];
+    const int Cq = a.Cq, h = blockIdx.x, tid = threadIdx.x;
+    int *cnt = tm_sm, *own = cnt + Cq, *S = own + Cq, *tail = S + Cq, *nn = tail + Cq;
+    int *partner = nn + Cq, *mv_in = partner + Cq, *mv_out = mv_in + Cq, *offs = mv_out + Cq;  // offs: Cq + 1
+    int *pre = offs + Cq + 1;
+    const int k = a.ksel[h];
+    const bool dense = a.dense[h] != 0;
+    const int *sel = a.sel + (int64_t)h * Cq * a.Ccap;
+    for (int q = tid; q < Cq; q += SEL_THREADS) {
+        cnt[q] = a.counts_q[(int64_t)h * Cq + q];
+        S[q] = 0;
+        partner[q] = -1;
+        mv_in[q] = mv_out[q] = 0;
+    }
+    __syncthreads();
+    // stage 1
+    for (int q = tid; q < Cq; q += SEL_THREADS) {
+        int o = q;
+        if (cnt[q] > 0)
+            for (int r = 0; r < q; ++r)
+                if (cnt[r] > 0 && (dense || tm_same(sel + (int64_t)r * a.Ccap, sel + (int64_t)q * a.Ccap, k))) {
+                    o = r;
+                    break;
+                }
+        own[q] = o;
+    }
+    __syncthreads();
+    for (int q = tid; q < Cq; q += SEL_THREADS)
+        if (cnt[q] > 0) atomicAdd(&S[own[q]], cnt[q]);
+    __syncthreads();
+    // stage 2
+    for (int g = tid; g < Cq; g += SEL_THREADS)
+        tail[g] = (a.mode >= 2 && !dense && own[g] == g && S[g] > 0) ? S[g] % TM_TILE : 0;
+    __syncthreads();
+    for (int g = tid; g < Cq; g += SEL_THREADS) {
+        int best = -1, bd = 0x7FFFFFFF;
+        if (tail[g] > 0)
+            for (int o = 0; o < Cq; ++o) {
+                if (o == g || tail[o] == 0) continue;
+                const int dist = tm_hamming(sel + (int64_t)g * a.Ccap, sel + (int64_t)o * a.Ccap, k);
+                if (dist < bd) {
+                    bd = dist;
+                    best = o;
+                }
+            }
+        nn[g] = best;
+    }
+    __syncthreads();
+    for (int g = tid; g < Cq; g += SEL_THREADS) {
+        const int o = nn[g];
+        if (tail[g] > 0 && o > g && nn[o] == g && tail[g] + tail[o] <= TM_TILE) {
+            partner[g] = o;  // g takes o's tail
+            partner[o] = g;
+            mv_in[g] = tail[o];
+            mv_out[o] = tail[o];
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // group offsets (owners only) and every cluster's first position in its group
+        int run = 0;
+        for (int g = 0; g < Cq; ++g) {
+            offs[g] = run;
+            run += own[g] == g ? S[g] + mv_in[g] - mv_out[g] : 0;
+        }
+        offs[Cq] = run;
+        for (int g = 0; g < Cq; ++g) nn[g] = 0;  // reused: rows placed so far per group
+        for (int q = 0; q < Cq; ++q) {
+            pre[q] = nn[own[q]];
+            nn[own[q]] += cnt[q];
+        }
+    }
+    __syncthreads();
+    int *sc = a.scratch + (int64_t)h * Cq;
+    const int64_t plane = (int64_t)a.BH * Cq;
+    for (int q = tid; q < Cq; q += SEL_THREADS) {
+        const int g = own[q];
+        a.counts_qm[(int64_t)h * Cq + q] = own[q] == q ? S[q] + mv_in[q] - mv_out[q] : 0;
+        a.offs_qm[(int64_t)h * (Cq + 1) + q] = offs[q];
+        sc[q] = g;                                  // owner
+        sc[plane + q] = pre[q];                     // first position within the group
+        sc[2 * plane + q] = S[q] - mv_out[q];       // rows the group keeps (owners)
+        sc[3 * plane + q] = mv_out[q] > 0 ? offs[partner[q]] + S[partner[q]] : 0;  // where handed rows go
+    }
+    if (tid == 0) a.offs_qm[(int64_t)h * (Cq + 1) + Cq] = offs[Cq];
+    // key ranges of the groups that take a tail: the union of both selections, in cluster order
+    for (int g = tid; g < Cq; g += SEL_THREADS) {
+        if (mv_in[g] == 0) continue;
+        const int *A = sel + (int64_t)g * a.Ccap, *B = sel + (int64_t)partner[g] * a.Ccap;
+        const int64_t hq = (int64_t)h * Cq + g;
+        const int *cntk = a.counts_k + (int64_t)h * a.Ccap;
+        const int *pg = a.pgoff + (int64_t)h * a.Ccap;
+        int2 *rg = a.ranges + hq * a.Ccap;
+        int *rb = a.rbox + hq * (a.Ccap + 1);
+        int i = 0, j = 0, nr = 0, box = 0;
+        while (i < k || j < k) {
+            int c;
+            if (j >= k || (i < k && A[i] < B[j])) {
+                c = A[i++];
+            } else if (i >= k || B[j] < A[i]) {
+                c = B[j++];
+            } else {
+                c = A[i++];
+                ++j;
+            }
+            rg[nr] = make_int2(pg[c], cntk[c]);
+            rb[nr] = box;
+            box += (cntk[c] + 7) / 8;
+            ++nr;
+        }
+        rb[nr] = box;
+        a.nrange[hq] = nr;
+        a.nboxes[hq] = box;
+    }
+}
+
+// Rows of Qp in group order: the row at cluster-order position p (cluster q,
+// i-th member) goes to its group's position pre[q] + i, or, past the rows the
+// group keeps, to the group that takes its tail.
+__global__ void k_tail_merge_perm(TailMergeArgs a) {
+    const int h = blockIdx.y;
+    const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (p >= a.L) return;
+    const int64_t plane = (int64_t)a.BH * a.Cq;
+    const int tok = a.perm_q[(int64_t)h * a.L + p];
+    const int q = a.labels_q[(int64_t)h * a.L + tok];
+    const int *sc = a.scratch + (int64_t)h * a.Cq;
+    const int g = sc[q];
+    const int gp = sc[plane + q] + (int)(p - a.offs_q[(int64_t)h * (a.Cq + 1) + q]);
+    const int keep = sc[2 * plane + g];
+    const int dest = gp < keep ? a.offs_qm[(int64_t)h * (a.Cq + 1) + g] + gp : sc[3 * plane + g] + (gp - keep);
+    a.perm_qm[(int64_t)h * a.L + dest] = tok;
+}
+
+cudaError_t launch_tail_merge(const TailMergeArgs &a, cudaStream_t s) {
+    const size_t smem = (size_t)(10 * a.Cq + 1) * sizeof(int);
+    cudaError_t e;
+    if (smem > 48 * 1024) {
+        e = cudaFuncSetAttribute(k_tail_merge_plan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    k_tail_merge_plan<<<a.BH, SEL_THREADS, smem, s>>>(a);
+    AC_NOTE_LAUNCH();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_tail_merge_perm<<<dim3((unsigned)((a.L + 255) / 256), a.BH), 256, 0, s>>>(a);
+    AC_NOTE_LAUNCH();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_tile_prefix<<<1, 1024, 0, s>>>(a.counts_qm, a.BH * a.Cq, a.tile_prefix);
+    AC_NOTE_LAUNCH();
+    return cudaGetLastError();
+}
+
 cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s) {
     const size_t qsm = (size_t)(2 * a.d * QS_C + a.Cq * a.d) * 4;
     if (qsm > 200 * 1024) return cudaErrorInvalidValue;  // ac_create keeps Cq within this

@@ -89,6 +89,14 @@ typedef struct ac_config {
                             0: the Eq. (1) TensorQuest bound (the method);
                             1: mean-based, q . mu with mu the key cluster's centre
                                (the "w/o Quest" ablation of Sec. 4.4, Table 4)    */
+    int32_t tail_merge;  /* query-tile tail merging before the attention (iCATS,
+                            "tail merging strategy"): 0: off; 1: query clusters
+                            that select the same key clusters share tiles
+                            (lossless); 2: also, two clusters whose tails are
+                            each other's nearest selection (Hamming) and fit one
+                            128-row tile pool them: the higher index hands its
+                            tail to the lower, which attends to the union      */
+    int32_t reserved2;   /* must be 0                                             */
 } ac_config;
 
 typedef struct ac_ctx ac_ctx;

@@ -94,6 +94,7 @@ class Params:
     seed: int = 1234
     stage_rule: int = 0
     score_mode: int = 0   # 0: Eq. (1) bound; 1: mean-based scores (the "w/o Quest" ablation)
+    tail_merge: int = 0   # 0: off; 1: stage 1 of tail_merge (lossless); 2: both stages
 
     @property
     def ccap(self) -> int:
@@ -386,7 +387,7 @@ def attention_rows_comp(Q16h, K16h, V16h, labels_q, labels_k, sel, dense: bool, 
     return out
 
 
-def tail_merge(labels_q: np.ndarray, masks: np.ndarray, b: int = 128):
+def tail_merge(labels_q: np.ndarray, masks: np.ndarray, b: int = 128, stages: int = 2):
     """Two-stage tail merging of one head's query clusters (iCATS, "tail merging
     strategy" and its worked example), for a kernel that runs query clusters in
     b-row tiles.  labels_q [L]: query cluster of each token; masks [Cq, nk] bool:
@@ -404,6 +405,7 @@ def tail_merge(labels_q: np.ndarray, masks: np.ndarray, b: int = 128):
     Readings: the pages do not say which cluster of a pair absorbs the other's
     tail (their example is consistent with either); here the lower index does.
 
+    stages = 1 skips stage 2.
     Returns (owner [L] int32: the group whose mask each token attends with,
     new_masks [Cq, nk] bool, groups {owner: token list in group order},
     pairs [(i, j, moved)])."""
@@ -426,7 +428,7 @@ def tail_merge(labels_q: np.ndarray, masks: np.ndarray, b: int = 128):
             groups.setdefault(rep[c], []).extend(members[c].tolist())
     new_masks = masks.copy()
     # stage 2: mutual nearest neighbours among the groups with a tail
-    tails = {g: len(t) % b for g, t in groups.items() if len(t) % b > 0}
+    tails = {g: len(t) % b for g, t in groups.items() if len(t) % b > 0} if stages >= 2 else {}
     keys = sorted(tails)
     nn = {}
     for g in keys:
@@ -496,6 +498,25 @@ def layer(Q16, K16, V16, p: Params, warm_from: LayerResult | None = None,
         r = np.arange(L) if rows is None else np.asarray(rows)
         O = np.empty((BH, r.size, d), np.float64)
         for h in range(BH):
-            O[h] = attention_rows(Q16[h], K16[h], V16[h], lq[h], kc.labels[h], sel[h],
-                                  bool(kc.F[h]), r)
+            lab, sl = lq[h], sel[h]
+            if p.tail_merge and not kc.F[h]:
+                lab, sl = merged_selection(lq[h], sel[h], int(kc.n_k[h]), p.tail_merge)
+            O[h] = attention_rows(Q16[h], K16[h], V16[h], lab, kc.labels[h], sl, bool(kc.F[h]), r)
     return LayerResult(lq, Cq, cq, kc, st, S, sel, k, O)
+
+
+def merged_selection(labels_q, sel, nk: int, mode: int, b: int = 128):
+    """The per-token attention sets after tail merging (mode 1: stage 1 only, 2:
+    both stages) of one head: (owner per token, each owner's key clusters as
+    rows padded with -1)."""
+    Cq = sel.shape[0]
+    masks = np.zeros((Cq, nk), bool)
+    for q in range(Cq):
+        masks[q, sel[q]] = True
+    owner, new_masks, _, _ = tail_merge(labels_q, masks, b, stages=2 if mode >= 2 else 1)
+    width = int(new_masks.sum(1).max())
+    out = np.full((Cq, max(width, 1)), -1, np.int32)
+    for q in range(Cq):
+        c = np.nonzero(new_masks[q])[0]
+        out[q, :c.size] = c
+    return owner, out

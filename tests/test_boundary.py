@@ -48,7 +48,8 @@ def test_config_struct_layout_matches_header(tmp_path):
 def _create(**kw):
     lib = _lib.load()
     base = dict(Cq=16, m0=32, n_max=128, tau_mode=1, tau_value=0.5, topk=8, iters_q=10, iters_k=10,
-                iters_warm=2, stage_rule=0, seed=1, scale=0.0, score_mode=0)
+                iters_warm=2, stage_rule=0, seed=1, scale=0.0, score_mode=0, tail_merge=0,
+                reserved2=0)
     dims = kw.pop("dims", (1, 2, 4096, 64))
     base.update(kw)
     cfg = _lib.ACConfig(**base)

@@ -53,6 +53,36 @@ def test_mean_score_ablation_end_to_end():
     lay.close()
 
 
+@pytest.mark.parametrize("mode", [1, 2])
+def test_tail_merge_end_to_end(mode):
+    """ac_config.tail_merge (iCATS tail merging of the query tiles): query
+    clusters with the same selection share tiles (mode 1; four of the sixteen
+    clusters fold in here), and mutually nearest clusters with small tails pool
+    them (mode 2; three pairs here); outputs against the oracle's per-token key
+    sets after the same merge."""
+    cfg = synth.CONFIGS[1]
+    Q, K, V = synth.make_layer(cfg)
+    p = _params(cfg, tail_merge=mode)
+    r = orc.layer(_flat(Q), _flat(K), _flat(V), p)
+    lay, O, gs = run_gpu_layer(Q, K, V, p)
+    compare_layer(gs, r, p, O)
+    lay.close()
+
+
+def test_tail_merge_dense_units():
+    """Every unit dense: every query cluster walks every key, so stage 1 folds
+    all of them into one group; the output stays dense attention."""
+    cfg = synth.LayerConfig("dense", 1, 2, 1200, 64, Cq=5, m0=8, n_max=20, tau_mode=0, tau_value=0.0,
+                            topk=2, key_components=20, iters_q=3, iters_k=2)
+    Q, K, V = synth.make_layer(cfg)
+    p = _params(cfg, tail_merge=2)
+    r = orc.layer(_flat(Q), _flat(K), _flat(V), p)
+    assert r.kc.F.all()
+    lay, O, gs = run_gpu_layer(Q, K, V, p)
+    compare_layer(gs, r, p, O)
+    lay.close()
+
+
 def test_tiny_layer_warm_chain():
     """Step 0 then two warm-started steps on perturbed tokens (Sec. 3.2.2)."""
     cfg = synth.CONFIGS[1]
