@@ -23,10 +23,6 @@ __device__ __forceinline__ void set_err(uint32_t *err, uint32_t bit) {
 // ------------------------------------------------------------------ numbers
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-__device__ __forceinline__ float bfbits2f(uint16_t b) {
-    return __uint_as_float(((uint32_t)b) << 16);
-}
-
 // SplitMix64 output function (Steele, Lea, Flood, OOPSLA 2014).
 __device__ __forceinline__ uint64_t mix64(uint64_t z) {
     z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
@@ -140,25 +136,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int3
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar)
         : "memory");
-}
-
-// 3-D tiled bulk tensor load (coordinates x innermost).  No cluster multicast.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int32_t x, int32_t y, int32_t z,
-                                            uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
-        : "memory");
-}
-
-// Plain bulk copy of `bytes` contiguous bytes from global memory into this
-// CTA's shared memory (no tensor map, no cluster multicast), completion counted
-// on `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
 }
 
 // 4-D tiled bulk tensor load (coordinates x innermost).  No cluster multicast.
