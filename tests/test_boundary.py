@@ -67,6 +67,9 @@ def _create(**kw):
     (dict(tau_mode=2, tau_value=0.0), _lib.AC_ERR_INVALID_ARG),
     (dict(iters_k=-1), _lib.AC_ERR_INVALID_ARG),
     (dict(stage_rule=3), _lib.AC_ERR_INVALID_ARG),
+    (dict(score_mode=2), _lib.AC_ERR_INVALID_ARG),
+    (dict(tail_merge=3), _lib.AC_ERR_INVALID_ARG),
+    (dict(reserved2=1), _lib.AC_ERR_INVALID_ARG),
     (dict(dims=(1, 2, 0, 64)), _lib.AC_ERR_INVALID_ARG),
     (dict(dims=(1, 2, 4096, 96)), _lib.AC_ERR_UNSUPPORTED),
 ])
@@ -80,6 +83,8 @@ def test_null_arguments_rejected():
     assert lib.ac_create(None, 1, 1, 1, 64, None) == _lib.AC_ERR_INVALID_ARG
     assert lib.ac_destroy(None) == _lib.AC_ERR_INVALID_ARG
     assert lib.ac_synchronize(None, None) == _lib.AC_ERR_INVALID_ARG
+    assert lib.ac_join(None, None) == _lib.AC_ERR_INVALID_ARG
+    assert lib.ac_layer_forward_host_async(None, None, None, None, None, 0, None) == _lib.AC_ERR_INVALID_ARG
     assert lib.ac_last_error_string(None) == b""
 
 
