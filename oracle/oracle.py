@@ -95,6 +95,7 @@ class Params:
     stage_rule: int = 0
     score_mode: int = 0   # 0: Eq. (1) bound; 1: mean-based scores (the "w/o Quest" ablation)
     tail_merge: int = 0   # 0: off; 1: stage 1 of tail_merge (lossless); 2: both stages
+    compensate: int = 0   # 1: unselected clusters enter as centroid pseudo-tokens (attention_rows_comp)
 
     @property
     def ccap(self) -> int:
@@ -501,7 +502,14 @@ def layer(Q16, K16, V16, p: Params, warm_from: LayerResult | None = None,
             lab, sl = lq[h], sel[h]
             if p.tail_merge and not kc.F[h]:
                 lab, sl = merged_selection(lq[h], sel[h], int(kc.n_k[h]), p.tail_merge)
-            O[h] = attention_rows(Q16[h], K16[h], V16[h], lab, kc.labels[h], sl, bool(kc.F[h]), r)
+            if p.compensate and not kc.F[h]:
+                nk = int(kc.n_k[h])
+                km, cnt = cluster_means(K16[h], kc.labels[h], nk)
+                vm, _ = cluster_means(V16[h], kc.labels[h], nk)
+                O[h] = attention_rows_comp(Q16[h], K16[h], V16[h], lab, kc.labels[h], sl, False, r, nk, cnt,
+                                           km.astype(np.float64), vm.astype(np.float64))
+            else:
+                O[h] = attention_rows(Q16[h], K16[h], V16[h], lab, kc.labels[h], sl, bool(kc.F[h]), r)
     return LayerResult(lq, Cq, cq, kc, st, S, sel, k, O)
 
 

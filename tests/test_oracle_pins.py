@@ -475,6 +475,27 @@ def test_compensation_exact_for_identical_members_and_all_selected():
     assert np.array_equal(o, oh)
 
 
+def test_compensated_layer_is_closer_to_dense():
+    """Layer level (Params.compensate): the unselected key clusters enter as
+    member-mean pseudo-tokens.  On the tiny layer, whose key clusters are tight
+    mixture components, the compensated output lies closer to dense attention
+    than the plain sparse one for most rows, and far closer on average."""
+    cfg = synth.CONFIGS[1]
+    Q, K, V = synth.make_layer(cfg, heads=[0])
+    B, H, L, d = Q.shape
+    f = lambda x: x.reshape(B * H, L, d)  # noqa: E731
+    p = orc.Params.from_layer_config(cfg)
+    rows = np.arange(0, L, 29)
+    plain = orc.layer(f(Q), f(K), f(V), p, rows=rows)
+    p.compensate = 1
+    comp = orc.layer(f(Q), f(K), f(V), p, rows=rows)
+    assert not plain.kc.F[0]
+    dense = orc.attention_rows(f(Q)[0], f(K)[0], f(V)[0], plain.labels_q[0], plain.kc.labels[0], None, True, rows)
+    e_plain = np.linalg.norm(plain.O[0] - dense, axis=1)
+    e_comp = np.linalg.norm(comp.O[0] - dense, axis=1)
+    assert (e_comp < e_plain).mean() > 0.8 and e_comp.mean() < 0.5 * e_plain.mean()
+
+
 def test_cluster_means_are_member_order_fp32_sums():
     """or_cluster_means follows the Lloyd update's rule (fp32 sums in ascending
     token order, then one division); a consistency check of that rule, not a
