@@ -149,7 +149,8 @@ def oracle_sample(cfg_id: int, rows_attn: int = 256, heads=(0,)):
     """The oracle on a bounded sample of the workload: full step-0 clustering of
     the sampled heads (tau pooled over them), Quest + top-k, and attention for
     `rows_attn` query rows per head, extrapolated linearly to all L rows.
-    Returns (effective TFLOP/s, seconds, description, threads)."""
+    Returns (effective TFLOP/s, extrapolated seconds of the sampled heads' layer,
+    description, threads, wall seconds the sample itself took)."""
     from oracle import oracle as orc
     from cluster_routed_sparse_b200 import synth
     cfg = synth.CONFIGS[cfg_id]
@@ -164,11 +165,12 @@ def oracle_sample(cfg_id: int, rows_attn: int = 256, heads=(0,)):
         orc.attention_rows(Qf[h], Kf[h], Vf[h], r.labels_q[h], r.kc.labels[h], r.sel[h], bool(r.kc.F[h]), rows)
     t2 = time.perf_counter()
     t_total = (t1 - t0) + (t2 - t1) * cfg.L / rows_attn
+    t_wall = t2 - t0
     flops = 4.0 * len(heads) * cfg.L * cfg.L * cfg.d
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     desc = (f"{len(heads)} of {cfg.H} heads, step 0: full clustering + Quest/top-k; attention on "
             f"{rows_attn} of {cfg.L} query rows, extrapolated linearly")
-    return flops / t_total / 1e12, t_total, desc, threads
+    return flops / t_total / 1e12, t_total, desc, threads, t_wall
 
 
 def run_reference(args):
@@ -178,7 +180,7 @@ def run_reference(args):
     vals = []
     desc, threads = "", 1
     for i in range(args.warmup + args.steps):
-        v, t, desc, threads = oracle_sample(CONFIG_ID, rows_attn=128)
+        v, t, desc, threads, _ = oracle_sample(CONFIG_ID, rows_attn=128)
         if i >= args.warmup:
             vals.append((v, t))
     value = float(np.mean([v for v, _ in vals]))
@@ -372,9 +374,9 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, tsec, desc, threads = oracle_sample(CONFIG_ID)
+        v, tsec, desc, threads, twall = oracle_sample(CONFIG_ID)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
-               "seconds": tsec}
+               "extrapolated_seconds": tsec, "sample_wall_seconds": twall}
 
     if rank == 0:
         out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
