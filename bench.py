@@ -344,8 +344,8 @@ def main():
     hbm = peaks.get("hbm_gbs") or 6650.0
     tensor_bytes = 2.0 * cfg.B * cfg.H * cfg.L * cfg.d
     passes = {"q_cluster_ms": 1 + 3 + 2,   # norms, 3 assignment passes, 2 centre updates
-              "k_cluster_ms": 1 + 3 + 2 + 1,  # norms, 3 passes, 2 updates, exact distances
-              "stats_sort_ms": 1}          # per-cluster max / min / SSE
+              "k_cluster_ms": 1 + 3 + 2,   # norms, 3 passes, 2 updates
+              "stats_sort_ms": 1}          # per-cluster max / min, exact distances, SSE (one pass)
     red = {}
     for k, n in passes.items():
         gbs = n * tensor_bytes / (splitw[k] * 1e-3) / 1e9
@@ -359,6 +359,16 @@ def main():
              "assign_counters_since_create": lay.assign_counters(),
              "kept_pair_frac": cnt["kept_pairs"] / float(cfg.H * cfg.L * cfg.L),
              "tile_efficiency": cnt["kept_pairs"] / max(1, cnt["computed_pairs"])}
+    # per-head state after the last call: key clusters, dense fallback, compactness, step-0 stages
+    try:
+        from cluster_routed_sparse_b200 import _lib as L
+        extra["per_head"] = {
+            "n_k": lay.tensor(L.AC_T_N_K).cpu().tolist(),
+            "dense": lay.tensor(L.AC_T_DENSE).cpu().tolist(),
+            "comp": [round(float(x), 5) for x in lay.tensor(L.AC_T_COMP).cpu().tolist()],
+            "stages": lay.tensor(L.AC_T_STAGES).cpu().tolist()}
+    except Exception as exc:  # reporting only: never fail the bench line on it
+        extra["per_head"] = {"unavailable": str(exc)[:200]}
     # dense SDPA on the same tensors (one warm step's inputs)
     if not args.no_sdpa and rank == 0:
         extra["dense_sdpa"] = time_sdpa(*steps_in[1])
