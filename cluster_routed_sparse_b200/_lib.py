@@ -95,7 +95,7 @@ SIGNATURES = {
     "ac_get_attn_counters": (_I, [_P, ctypes.POINTER(ACAttnCounters)]),
     "ac_get_launch_count": (_I, [ctypes.POINTER(ctypes.c_int64)]),
     "ac_get_assign_counters": (_I, [_P, ctypes.POINTER(ACAssignCounters), _I]),
-    "ac_cluster_q_noalloc": (_I, [_P, _I, _I, _I, _I, _I, ctypes.c_uint64, _P, _P, _P, _P]),
+    "ac_cluster_q_noalloc": (_I, [_P, _I, _I, _I, _I, _I, ctypes.c_uint64, _P, _P, _P, _P, _P]),
     "ac_state_export": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int64)]),
     "ac_state_import": (_I, [_P, _P, ctypes.c_int64]),
 }

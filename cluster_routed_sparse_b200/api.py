@@ -40,14 +40,16 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def cluster_q_noalloc(Q, Cq: int, labels, centroids, iters: int = 10, seed: int = 1234, init=None):
+def cluster_q_noalloc(Q, Cq: int, labels, centroids, iters: int = 10, seed: int = 1234, init=None, err=None):
     """ac_cluster_q_noalloc: angular k-means of Q [B, H, L, d] (bf16, CUDA) into
     caller-provided labels [B, H, L] int32 and centroids [B, H, Cq, d] fp32,
-    with no device allocation inside the library (see include/ac.h)."""
+    with no device allocation inside the library (see include/ac.h).  err: an
+    optional one-element int32 CUDA tensor that receives the kernels' error
+    bits (1: a bounded wait expired, 4: non-finite input)."""
     lib = _lib.load()
     B, H, L, d = Q.shape
     check(lib.ac_cluster_q_noalloc(_bits(Q), B * H, L, d, Cq, iters, seed & (2**64 - 1), _ptr(init),
-                                   _ptr(labels), _ptr(centroids), _stream()))
+                                   _ptr(labels), _ptr(centroids), _ptr(err), _stream()))
 
 
 class SparseLayer:

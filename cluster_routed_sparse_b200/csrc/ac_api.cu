@@ -964,7 +964,14 @@ ac_status ac_layer_forward_host_async(ac_ctx *c, const uint16_t *hQ, const uint1
     ++c->async_calls;
     ac_status st = layer_steps(c, buf[0], buf[1], buf[2], buf[3], warm, nullptr, s, c->ev_inq[b], c->ev_ink[b],
                                c->ev_in[b]);
-    if (st != AC_OK) return st;
+    if (st != AC_OK) {
+        // Kernels of this call may already be enqueued and read set b: the
+        // set's events must order its next use after them, as on success.
+        if (cudaEventRecord(c->ev_comp[b], s) == cudaSuccess &&
+            cudaStreamWaitEvent(c->s_out, c->ev_comp[b], 0) == cudaSuccess)
+            cudaEventRecord(c->ev_out[b], c->s_out);
+        return st;
+    }
     c->have_state = true;
     CK(cudaEventRecord(c->ev_comp[b], s), "event");
     CK(cudaStreamWaitEvent(c->s_out, c->ev_comp[b], 0), "wait layer");

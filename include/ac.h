@@ -279,8 +279,9 @@ AC_API ac_status ac_get_attn_counters(ac_ctx *ctx, ac_attn_counters *out);
  * tensor cores: centres split into bf16 + remainder, x . c_hi per pair, then
  * a rigorous error bound decides each row; rows the bound cannot settle are
  * rescored with the exact fp32 arithmetic, so labels equal the exact
- * definition's.  Stages t >= 1 of Algorithm 1 (gathered rows) and inputs not
- * 16-byte aligned take the exact CUDA-core kernel.  The environment variable
+ * definition's.  Stages t >= 1 of Algorithm 1 run on a gathered copy of the
+ * unabsorbed keys, on the tensor cores too; only inputs that are not 16-byte
+ * aligned take the exact CUDA-core kernel.  The environment variable
  * AC_EXACT_ASSIGN=1 at ac_create forces the exact kernel everywhere.
  * Synchronises `ctx`'s device; reset != 0 zeroes the counters afterwards. */
 typedef struct ac_assign_counters {
@@ -304,18 +305,27 @@ AC_API ac_status ac_get_assign_counters(ac_ctx *ctx, ac_assign_counters *out, in
  *    ac_cluster_q does).  iters >= 0 Lloyd iterations, then a final assignment.
  *  - Outputs (device, required): labels_out [BH, L] int32; centroids_out
  *    [BH, Cq, d] fp32, also used as the working centres (updated in place).
- *  - Limits: BH*L <= 1048576 and BH*(Cq+1) <= 65536, else AC_ERR_INVALID_ARG
- *    before any work.  The scratch (norms, permutation, offsets, counts) is one
- *    8.5 MiB __device__ array that every GPU which loads libac holds until the
- *    process exits; nothing is allocated per call.
- *  - The first call on a device looks the array's address up
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - err_out: nullable device uint32.  The call sets it to 0 on `stream`, and
+ *    its kernels OR in their error bits: 1 = a bounded in-kernel wait expired
+ *    (the outputs are not valid), 4 = NaN or Inf in Q.  Read it once `stream`
+ *    has passed the call.  With NULL, errors are recorded in the scratch array
+ *    and cannot be read.
+ *  - Limits: BH*L <= 1048576, BH*(Cq+1) <= 65536 and Cq <= 4096 (the sort's
+ *    shared-memory histograms), else AC_ERR_INVALID_ARG before any work.  The
+ *    scratch (error word, norms, permutation, offsets, counts) is one 8.5 MiB
+ *    __device__ array that every GPU which loads libac holds until the process
+ *    exits; nothing is allocated per call.
+ *  - The first call in a CUDA context looks the array's address up
+ *    (cudaGetSymbolAddress) and keeps it per context, so a context that was
+ *    reset and created again looks it up anew; make the first call in a
+ *    context before any stream capture.
  *  - Every call shares the one array: calls that overlap on the GPU (two
  *    streams, two threads) race and corrupt each other's results.  Serialise
- *    them.  Asynchronous on `stream`; no NaN check (no error word to read). */
+ *    them.  Asynchronous on `stream`. */
 AC_API ac_status ac_cluster_q_noalloc(const uint16_t *Q, int32_t BH, int32_t L, int32_t d, int32_t Cq,
                                       int32_t iters, uint64_t seed, const float *init_centroids,
-                                      int32_t *labels_out, float *centroids_out, void *stream);
+                                      int32_t *labels_out, float *centroids_out, uint32_t *err_out,
+                                      void *stream);
 
 /* Number of kernels libac has launched in this process so far (all contexts). */
 AC_API ac_status ac_get_launch_count(int64_t *out);

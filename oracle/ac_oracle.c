@@ -51,6 +51,9 @@ typedef struct or_cfg {
     int iters_warm;  /* Lloyd iterations in a warm-started step */
     int stage_rule;  /* cluster count of stages t > 0, see or_stage_clusters */
     uint64_t seed;
+    int64_t unit0;   /* (batch, head) index of the first unit of the call: unit h of
+                        the call draws its initial centres as unit unit0 + h, so a
+                        head can be run on its own with the seeds of the whole layer */
 } or_cfg;
 
 /* ------------------------------------------------------------------ */
@@ -243,7 +246,7 @@ void or_cluster_q(const uint16_t *Q, int BH, int L, int d, const or_cfg *cfg,
             memcpy(Ch, init + (int64_t)h * m * d, (size_t)m * d * sizeof(float));
         } else {
             int64_t *pos = (int64_t *)malloc((size_t)m * sizeof(int64_t));
-            or_seed_pick(cfg->seed, h, 0, L, m, pos);
+            or_seed_pick(cfg->seed, cfg->unit0 + h, 0, L, m, pos);
             for (int j = 0; j < m; ++j) memcpy(Ch + (int64_t)j * d, X + pos[j] * d, (size_t)d * sizeof(float));
             free(pos);
         }
@@ -372,7 +375,7 @@ int or_cluster_k_multistage(const uint16_t *K, int BH, int L, int d, const or_cf
         int64_t *uidx = (int64_t *)malloc((size_t)L * sizeof(int64_t));
         for (int64_t i = 0; i < L; ++i) uidx[i] = i;
         int32_t m = or_stage_clusters(cfg->m0, L, L, 0, cfg->stage_rule);
-        ms_stage(Kf, d, uidx, L, m, cfg, h, 0, C + (int64_t)h * Ccap * d, dist0 + (int64_t)h * L);
+        ms_stage(Kf, d, uidx, L, m, cfg, cfg->unit0 + h, 0, C + (int64_t)h * Ccap * d, dist0 + (int64_t)h * L);
         n_k[h] = m;
         free(Kf);
         free(uidx);
@@ -413,7 +416,7 @@ int or_cluster_k_multistage(const uint16_t *K, int BH, int L, int d, const or_cf
                 break;
             }
             int32_t m = or_stage_clusters(cfg->m0, nU, L, t, cfg->stage_rule); /* line 11 */
-            ms_stage(Kf, d, uidx, nU, m, cfg, h, t, Ch + (int64_t)nc * d, dist); /* line 12, 14 */
+            ms_stage(Kf, d, uidx, nU, m, cfg, cfg->unit0 + h, t, Ch + (int64_t)nc * d, dist); /* line 12, 14 */
             int64_t keep = 0;
             for (int64_t j = 0; j < nU; ++j) {                     /* lines 13-18 */
                 if (dist[j] < tau) {

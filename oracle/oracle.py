@@ -47,7 +47,7 @@ class _Cfg(ctypes.Structure):
                 ("tau_mode", ctypes.c_int), ("tau_value", ctypes.c_float),
                 ("topk", ctypes.c_int), ("iters_q", ctypes.c_int), ("iters_k", ctypes.c_int),
                 ("iters_warm", ctypes.c_int), ("stage_rule", ctypes.c_int),
-                ("seed", ctypes.c_uint64)]
+                ("seed", ctypes.c_uint64), ("unit0", ctypes.c_int64)]
 
 
 _lib = None
@@ -96,6 +96,7 @@ class Params:
     score_mode: int = 0   # 0: Eq. (1) bound; 1: mean-based scores (the "w/o Quest" ablation)
     tail_merge: int = 0   # 0: off; 1: stage 1 of tail_merge (lossless); 2: both stages
     compensate: int = 0   # 1: unselected clusters enter as centroid pseudo-tokens (attention_rows_comp)
+    unit0: int = 0        # (batch, head) index of the first unit of a call (the seeds of a head subset)
 
     @property
     def ccap(self) -> int:
@@ -104,7 +105,7 @@ class Params:
     def c(self) -> _Cfg:
         return _Cfg(self.Cq, self.m0, self.n_max, self.tau_mode, float(self.tau_value),
                     self.topk, self.iters_q, self.iters_k, self.iters_warm, self.stage_rule,
-                    ctypes.c_uint64(self.seed & (2**64 - 1)))
+                    ctypes.c_uint64(self.seed & (2**64 - 1)), ctypes.c_int64(self.unit0))
 
     @staticmethod
     def from_layer_config(cfg, seed: int = 1234) -> "Params":

@@ -18,13 +18,13 @@ from cluster_routed_sparse_b200 import _lib, synth
 pytestmark = pytest.mark.gpu
 
 
-def _noalloc(lib, Q, Cq, iters, seed, labels, cent, init=None):
+def _noalloc(lib, Q, Cq, iters, seed, labels, cent, init=None, err=None):
     B, H, L, d = Q.shape
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     return lib.ac_cluster_q_noalloc(ctypes.c_void_p(Q.data_ptr()), B * H, L, d, Cq, iters, seed,
                                     ctypes.c_void_p(init.data_ptr()) if init is not None else None,
                                     ctypes.c_void_p(labels.data_ptr()), ctypes.c_void_p(cent.data_ptr()),
-                                    stream)
+                                    ctypes.c_void_p(err.data_ptr()) if err is not None else None, stream)
 
 
 @pytest.mark.parametrize("cfg", [synth.CONFIGS[1],
@@ -44,9 +44,11 @@ def test_noalloc_matches_cluster_q_on_two_calls(cfg):
     for call in range(2):
         lab = torch.full((BH, cfg.L), -7, dtype=torch.int32, device="cuda")
         cent = torch.full((BH, cfg.Cq, cfg.d), float("nan"), dtype=torch.float32, device="cuda")
-        st = _noalloc(lib, Q, cfg.Cq, cfg.iters_q, p.seed, lab, cent)
+        err = torch.full((1,), 99, dtype=torch.int32, device="cuda")  # the call clears it
+        st = _noalloc(lib, Q, cfg.Cq, cfg.iters_q, p.seed, lab, cent, err=err)
         assert st == _lib.AC_OK, lib.ac_last_error_string(None)
         torch.cuda.synchronize()
+        assert int(err.item()) == 0, f"kernel error bits {int(err.item())} on call {call}"
         assert torch.equal(lab, ref_lab), f"labels differ on call {call}"
         err = (cent.double() - ref_cent.double()).abs()
         tol = CENT_RTOL * ref_cent.double().abs().clamp_min(1e-3)
@@ -76,7 +78,12 @@ def test_noalloc_warm_start_and_limits():
     # beyond the stated maximum: rejected before any work, with a message
     big = torch.empty((1, 1, 1, 64), dtype=torch.bfloat16, device="cuda")
     st = lib.ac_cluster_q_noalloc(ctypes.c_void_p(big.data_ptr()), 1 << 11, 1 << 10, 64, 4, 1, 0, None,
-                                  ctypes.c_void_p(lab.data_ptr()), ctypes.c_void_p(cent.data_ptr()), None)
+                                  ctypes.c_void_p(lab.data_ptr()), ctypes.c_void_p(cent.data_ptr()), None, None)
     assert st == _lib.AC_ERR_INVALID_ARG
     assert b"1048576" in lib.ac_last_error_string(None)
+    # more centres than the sort's shared-memory histograms hold: rejected up front too
+    st = lib.ac_cluster_q_noalloc(ctypes.c_void_p(big.data_ptr()), 1, 8192, 64, 4097, 1, 0, None,
+                                  ctypes.c_void_p(lab.data_ptr()), ctypes.c_void_p(cent.data_ptr()), None, None)
+    assert st == _lib.AC_ERR_INVALID_ARG
+    assert b"4096" in lib.ac_last_error_string(None)
     lay.close()
