@@ -1,18 +1,21 @@
 """Benchmark of the cluster-routed sparse attention layer on B200.
 
-Workload: the Wan-2.1-14B-class layer (B=1, H=40, L=75,600, d=128, bf16) with
-ten simulated denoising steps: step 0 runs the full multi-stage clustering,
-steps 1-9 warm-start from the previous step's centres (2 Lloyd iterations).
-One bench "step" is that whole ten-step sequence over one layer: every row of
-the hot path (query clustering, multi-stage / warm key clustering, stats and
-permutations, Quest scores + top-k, sparse attention) runs inside the timed
-region on inputs already resident in HBM (3 x 774 MB per denoising step, far
-larger than L2).
+Default workload: the Wan-2.1-14B-class layer (B=1, H=40, L=75,600, d=128,
+bf16) with ten simulated denoising steps: step 0 runs the full multi-stage
+clustering, steps 1-9 warm-start from the previous step's centres (2 Lloyd
+iterations).  One bench "step" is that whole ten-step sequence over one layer:
+every row of the hot path (query clustering, multi-stage / warm key
+clustering, stats and permutations, Quest scores + top-k, sparse attention)
+runs inside the timed region on inputs already resident in HBM (3 x 774 MB per
+denoising step, far larger than L2).  --config N selects another workload of
+synth.CONFIGS (one step-0 layer call per bench step; L2 flushed between bench
+steps, outside the timed events).
 
-metric: effective TFLOP/s = 10 x 4*B*H*L^2*d / t (dense-equivalent FLOPs of
-the ten layer calls over their device time); higher is better.
+metric: effective TFLOP/s = calls x 4*B*H*L^2*d / t (dense-equivalent FLOPs of
+the layer calls over their device time); higher is better.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config N] [--topk -PERMILLE] [--stage-rule R] [--tail-merge M]
 
 Under torchrun every rank runs its own layer (independent problems, weak
 scaling, no collective on the data path); time is the max over ranks.
@@ -21,7 +24,6 @@ from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import subprocess
 import sys
@@ -33,9 +35,44 @@ sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
 
-CONFIG_ID = 4
-N_DENOISE = 10
+DEFAULT_CONFIG = 4
+CONFIG_ID = DEFAULT_CONFIG
 NOISE_STD = 0.02
+METRIC = "sparse-attn layer ms & effective TFLOP/s (L=75,600 H=40 d=128) vs dense SDPA"
+
+
+def workload(args):
+    """The synth.LayerConfig the run measures (with any overrides)."""
+    import dataclasses
+    from cluster_routed_sparse_b200 import synth
+    cfg = synth.CONFIGS[args.config]
+    over = {}
+    if args.topk:
+        over["topk"] = args.topk
+    if args.stage_rule is not None:
+        over["stage_rule"] = args.stage_rule
+    if args.heads:
+        over["H"] = args.heads
+    return dataclasses.replace(cfg, **over) if over else cfg
+
+
+def tau_text(cfg):
+    return {0: f"tau={cfg.tau_value:g}", 1: f"tau={cfg.tau_value:g}x mean",
+            2: f"tau=p{cfg.tau_value / 10:g} of the stage-0 distances"}[cfg.tau_mode]
+
+
+def workload_config(cfg, args):
+    steps = cfg.steps
+    seq = (f"{steps} denoising steps (step 0 multi-stage, {steps - 1} warm)" if steps > 1
+           else "one step-0 layer call (multi-stage key clustering)")
+    topk = f"top-k {-cfg.topk / 10:g}% of key clusters" if cfg.topk < 0 else f"top-k {cfg.topk}"
+    return {"workload": f"{cfg.name}: B={cfg.B} H={cfg.H} L={cfg.L} d={cfg.d} bf16, {seq}, Cq={cfg.Cq}, "
+                        f"m0={cfg.m0}, N_max={cfg.n_max}, {tau_text(cfg)}, {topk}, stage rule {cfg.stage_rule}"
+                        + (f", tail merging {args.tail_merge}" if args.tail_merge else ""),
+            "global_batch": cfg.B, "seq_len": cfg.L, "heads": cfg.H, "head_dim": cfg.d,
+            "l2": ("inputs larger than L2 (3 x 774 MB per denoising step, 10 distinct steps)" if steps > 1
+                   else "L2 flushed (512 MB write) before every timed bench step, outside its events"),
+            "parallelism": "one layer per rank"}
 
 
 # ---------------------------------------------------------------- inputs
@@ -48,27 +85,27 @@ def max_over_ranks(ms_local, world, device, dist=None):
     return float(t.item())
 
 
+def dense_flops(cfg):
+    return 4.0 * cfg.B * cfg.H * cfg.L * cfg.L * cfg.d
+
+
 def job_tflops(ms, world, cfg):
-    """Whole-job dense-equivalent rate: every rank runs one layer of cfg (weak scaling)."""
-    return world * N_DENOISE * 4.0 * cfg.B * cfg.H * cfg.L * cfg.L * cfg.d / (ms * 1e-3) / 1e12
+    """Whole-job dense-equivalent rate: every rank runs one layer of cfg, cfg.steps
+    calls per bench step (weak scaling)."""
+    return world * cfg.steps * dense_flops(cfg) / (ms * 1e-3) / 1e12
 
 
 def _gen_head(args):
     cfg, head = args
     from cluster_routed_sparse_b200 import synth
-    g = synth
-    q = g._head_queries_f32(cfg, head)
-    k = g._head_keys_f32(cfg, head)
-    v = g._head_values_f32(cfg, head)
-    return head, q, k, v
+    return head, synth._head_queries_f32(cfg, head), synth._head_keys_f32(cfg, head), synth._head_values_f32(cfg, head)
 
 
 def generate_step0_f32(cfg, heads, procs: int):
     """fp32 step-0 tokens of the listed heads, generated in a spawn pool."""
     import multiprocessing as mp
     out = np.empty((3, len(heads), cfg.L, cfg.d), np.float32)
-    ctx = mp.get_context("spawn")
-    with ctx.Pool(procs) as pool:
+    with mp.get_context("spawn").Pool(procs) as pool:
         for h, q, k, v in pool.imap_unordered(_gen_head, [(cfg, h) for h in heads]):
             i = heads.index(h)
             out[0, i], out[1, i], out[2, i] = q, k, v
@@ -144,87 +181,119 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-# ---------------------------------------------------------------- CPU oracle leg
-def oracle_sample(cfg_id: int, rows_attn: int = 256, heads=(0,)):
-    """The oracle on a bounded sample of the workload: full step-0 clustering of
-    the sampled heads (tau pooled over them), Quest + top-k, and attention for
-    `rows_attn` query rows per head, extrapolated linearly to all L rows.
-    Returns (effective TFLOP/s, extrapolated seconds of the sampled heads' layer,
-    description, threads, wall seconds the sample itself took)."""
-    from oracle import oracle as orc
-    from cluster_routed_sparse_b200 import synth
-    cfg = synth.CONFIGS[cfg_id]
-    Q, K, V = synth.make_layer(cfg, heads=list(heads))
-    Qf, Kf, Vf = (x.reshape(-1, cfg.L, cfg.d) for x in (Q, K, V))
-    p = orc.Params.from_layer_config(cfg)
-    t0 = time.perf_counter()
-    r = orc.layer(Qf, Kf, Vf, p, attention=False)
-    t1 = time.perf_counter()
-    rows = np.linspace(0, cfg.L - 1, rows_attn).astype(np.int64)
-    for h in range(len(heads)):
-        orc.attention_rows(Qf[h], Kf[h], Vf[h], r.labels_q[h], r.kc.labels[h], r.sel[h], bool(r.kc.F[h]), rows)
-    t2 = time.perf_counter()
-    t_total = (t1 - t0) + (t2 - t1) * cfg.L / rows_attn
-    t_wall = t2 - t0
-    flops = 4.0 * len(heads) * cfg.L * cfg.L * cfg.d
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    desc = (f"{len(heads)} of {cfg.H} heads, step 0: full clustering + Quest/top-k; attention on "
-            f"{rows_attn} of {cfg.L} query rows, extrapolated linearly")
-    return flops / t_total / 1e12, t_total, desc, threads, t_wall
+# ---------------------------------------------------------------- CPU oracle legs
+class OracleSample:
+    """The oracle, as it stands, on a bounded sample of one head of the workload:
+    step-0 clustering (tau from that head's own distances), Quest + top-k and
+    attention for `rows` query rows; with warm steps in the workload, also one
+    warm-started step of the same head.  Attention is extrapolated linearly to
+    all L rows; the head's sequence time is t0 + (steps - 1) * t_warm."""
+
+    def __init__(self, cfg, rows: int = 128, head: int = 0):
+        from oracle import oracle as orc
+        from cluster_routed_sparse_b200 import synth
+        self.orc, self.cfg, self.rows = orc, cfg, rows
+        Q, K, V = synth.make_layer(cfg, heads=[head])
+        self.Q, self.K, self.V = (x.reshape(-1, cfg.L, cfg.d) for x in (Q, K, V))
+        self.p = orc.Params.from_layer_config(cfg)
+        self.rowsel = np.linspace(0, cfg.L - 1, rows).astype(np.int64)
+        self.r0 = None
+        self.t0 = self.tw = None
+
+    def _attn(self, r):
+        self.orc.attention_rows(self.Q[0], self.K[0], self.V[0], r.labels_q[0], r.kc.labels[0], r.sel[0],
+                                bool(r.kc.F[0]), self.rowsel)
+
+    def step0(self):
+        a = time.perf_counter()
+        self.r0 = self.orc.layer(self.Q, self.K, self.V, self.p, attention=False)
+        b = time.perf_counter()
+        self._attn(self.r0)
+        c = time.perf_counter()
+        self.t0 = (b - a) + (c - b) * self.cfg.L / self.rows
+        return c - a
+
+    def warm(self):
+        if self.r0 is None:
+            self.step0()
+        a = time.perf_counter()
+        r = self.orc.layer(self.Q, self.K, self.V, self.p, warm_from=self.r0, attention=False)
+        b = time.perf_counter()
+        self._attn(r)
+        c = time.perf_counter()
+        self.tw = (b - a) + (c - b) * self.cfg.L / self.rows
+        return c - a
+
+    def sequence_seconds(self):
+        steps = self.cfg.steps
+        return self.t0 + (steps - 1) * (self.tw if steps > 1 else 0.0)
+
+    def tflops(self):
+        return self.cfg.steps * 4.0 * self.cfg.L * self.cfg.L * self.cfg.d / self.sequence_seconds() / 1e12
+
+    def describe(self):
+        w = (f" + one warm step ({self.cfg.iters_warm} Lloyd iterations), sequence time t0 + "
+             f"{self.cfg.steps - 1} x t_warm" if self.cfg.steps > 1 else "")
+        return (f"1 of {self.cfg.H} heads: step-0 clustering (tau from that head's distances) + Quest/top-k"
+                f"{w}; attention on {self.rows} of {self.cfg.L} query rows per step, extrapolated linearly")
+
+
+def threads_used():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
 
 def run_reference(args):
+    """The reference arm: the oracle timed on the host cores (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    vals = []
-    desc, threads = "", 1
-    for i in range(args.warmup + args.steps):
-        v, t, desc, threads, _ = oracle_sample(CONFIG_ID, rows_attn=128)
-        if i >= args.warmup:
-            vals.append((v, t))
-    value = float(np.mean([v for v, _ in vals]))
-    ms = float(np.mean([t for _, t in vals])) * 1e3
+    cfg = workload(args)
+    smp = OracleSample(cfg, rows=128)
+    # each step: the step-0 sample, or (workloads with warm steps) alternately the
+    # step-0 and the warm-step sample; warm-up steps run the attention rows only
+    for _ in range(args.warmup):
+        if smp.r0 is None:
+            smp.step0()
+        else:
+            smp._attn(smp.r0)
+    walls = []
+    for i in range(args.steps):
+        walls.append(smp.warm() if (cfg.steps > 1 and i % 2 == 1) else smp.step0())
+    if cfg.steps > 1 and smp.tw is None:
+        smp.warm()
+    value = smp.tflops()
+    ms = float(np.mean(walls)) * 1e3
     out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference",
            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+           "ms_per_step_note": "wall time of each step's oracle sample (one head); value is that head's "
+                               "extrapolated sequence rate",
+           "extrapolated_head_sequence_ms": smp.sequence_seconds() * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-           "data": "synthetic", "config": workload_config(),
-           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                            "sample": desc},
+           "data": "synthetic", "config": workload_config(cfg, args),
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads_used(), "kind": "oracle",
+                            "sample": smp.describe()},
            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
     return 0
 
 
-METRIC = "sparse-attn layer ms & effective TFLOP/s (L=75,600 H=40 d=128) vs dense SDPA"
-
-
-def workload_config():
-    from cluster_routed_sparse_b200 import synth
-    c = synth.CONFIGS[CONFIG_ID]
-    return {"workload": f"{c.name}: B={c.B} H={c.H} L={c.L} d={c.d} bf16, {N_DENOISE} denoising steps "
-                        f"(step 0 multi-stage, 9 warm), Cq={c.Cq}, m0={c.m0}, N_max={c.n_max}, "
-                        f"tau=1.5x mean, top-k 10% of key clusters",
-            "global_batch": c.B, "seq_len": c.L, "heads": c.H, "head_dim": c.d,
-            "l2": "inputs larger than L2 (3 x 774 MB per denoising step, 10 distinct steps)",
-            "parallelism": "one layer per rank"}
-
-
 # ---------------------------------------------------------------- main
-# DRAM bytes (read + write) of one k_sparse_attn launch per head, from the ncu capture summarised
-# in profiles/k_sparse_attn_wan14b_h8.md (8 heads, scaled by heads), valid only for the kernel
-# source it was taken on: any change to attn_kernel.cu turns the figure into null.
+# DRAM bytes (read + write) of one k_sparse_attn launch per head of the bench
+# workload, from an ncu capture of its 8-head reduction, valid only for the
+# kernel source it was taken on: any change to attn_kernel.cu turns it into null.
 ATTN_TRAFFIC = {"sha256_prefix": "f0e4b1ad3dc6ebe4", "bytes_per_head": (313.705472e6 + 132.507648e6) / 8}
 
 
-def attn_traffic_bytes(heads):
+def attn_traffic_bytes(cfg):
     import hashlib
+    if cfg.name != "wan14b-L75600-H40-d128":
+        return None
     src = os.path.join(ROOT, "cluster_routed_sparse_b200", "csrc", "attn_kernel.cu")
     with open(src, "rb") as f:
         digest = hashlib.sha256(f.read()).hexdigest()
     if not digest.startswith(ATTN_TRAFFIC["sha256_prefix"]):
         return None
-    return round(ATTN_TRAFFIC["bytes_per_head"] * heads)
+    return round(ATTN_TRAFFIC["bytes_per_head"] * cfg.H)
 
 
 def main():
@@ -233,6 +302,11 @@ def main():
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, help="workload id in synth.CONFIGS")
+    ap.add_argument("--topk", type=int, default=0, help="override the top-k (negative: -permille of n_k)")
+    ap.add_argument("--stage-rule", type=int, default=None, help="override the m_t rule of stages t > 0")
+    ap.add_argument("--tail-merge", type=int, default=0, help="query-tile tail merging mode (0, 1, 2)")
+    ap.add_argument("--e2e-reps", type=int, default=3, help="repetitions of the end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sdpa", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -246,11 +320,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    from cluster_routed_sparse_b200 import synth
-    import dataclasses
-    cfg = synth.CONFIGS[CONFIG_ID]
-    if args.heads:
-        cfg = dataclasses.replace(cfg, H=args.heads)
+    cfg = workload(args)
+    n_calls = cfg.steps  # layer calls per bench step
 
     # inputs first (spawn pool, before any CUDA call); each rank its own layer
     x0 = generate_step0_f32(cfg, list(range(cfg.H)), max(1, args.procs // max(1, world)))
@@ -264,12 +335,14 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     from cluster_routed_sparse_b200.api import SparseLayer
 
-    steps_in = denoise_inputs(x0, N_DENOISE, seed=100 + rank, device=dev)
-    lay = SparseLayer.from_config(cfg, seed=1234 + rank)
+    steps_in = denoise_inputs(x0, n_calls, seed=100 + rank, device=dev)
+    del x0
+    lay = SparseLayer.from_config(cfg, seed=1234 + rank, tail_merge=args.tail_merge)
     O = torch.empty_like(steps_in[0][0])
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
 
     def one_step(collect=None):
-        for s in range(N_DENOISE):
+        for s in range(n_calls):
             Q, K, V = steps_in[s]
             if collect is None:
                 lay.forward(Q, K, V, O, warm=s > 0)
@@ -282,41 +355,42 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    launches0 = lay.launch_count()
     for _ in range(args.warmup):
         one_step()
     lay.synchronize()
 
-    # ---- timed region
+    # ---- timed region: K bench steps, each between its own events on the
+    # launching stream; the L2 flush before each step lies outside them
+    stream = torch.cuda.current_stream()
     clocks = ClockSampler(local)
     barrier()
     clocks.start()
-    stream = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches1 = lay.launch_count()
-    e0.record(stream)
-    per_call = []
+    per_call, ev = [], []
     for _ in range(args.steps):
+        flush_buf.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
         one_step(per_call)
-    e1.record(stream)
+        e1.record(stream)
+        ev.append((e0, e1))
     barrier()
     clk = clocks.stop()
     launches = lay.launch_count() - launches1
     lay.synchronize()
-    ms_local = e0.elapsed_time(e1) / args.steps
+    ms_local = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     ms = max_over_ranks(ms_local, world, dev, dist if world > 1 else None)
-
-    dense_flops_layer = 4.0 * cfg.B * cfg.H * cfg.L * cfg.L * cfg.d
     value = job_tflops(ms, world, cfg)
 
-    # stage split (from the same timed calls)
-    step0 = [c for i, c in enumerate(per_call) if i % N_DENOISE == 0]
-    warm = [c for i, c in enumerate(per_call) if i % N_DENOISE != 0]
-    avg = lambda rows, k: float(np.mean([r[k] for r in rows]))  # noqa: E731
+    # stage split (from the same timed calls): step 0 and the warm steps
+    step0 = [c for i, c in enumerate(per_call) if i % n_calls == 0]
+    warm = [c for i, c in enumerate(per_call) if i % n_calls != 0]
     keys = ["q_cluster_ms", "k_cluster_ms", "stats_sort_ms", "score_select_ms", "attention_ms",
             "attn_kernel_ms", "total_ms"]
+    avg = lambda rows, k: float(np.mean([r[k] for r in rows]))  # noqa: E731
     split0 = {k: avg(step0, k) for k in keys}
-    splitw = {k: avg(warm, k) for k in keys}
+    splitw = {k: avg(warm, k) for k in keys} if warm else None
+    steady = splitw or split0  # the call the roofline and the SDPA comparison use
     cnt = lay.counters()
 
     # roofline of the dominant kernel (sparse attention, tensor-bound)
@@ -329,72 +403,84 @@ def main():
     peak_tf = peaks.get("bf16_tflops_sustained")
     peak_src = "of measured (bf16_tflops_sustained)" if peak_tf else "of fallback"
     peak_tf = peak_tf or 1400.0
-    attn_flops = 4.0 * cfg.d * cnt["kept_pairs"]  # last call (a warm step)
-    traffic = attn_traffic_bytes(cfg.H)
-    achieved = attn_flops / (splitw["attn_kernel_ms"] * 1e-3) / 1e12
+    attn_flops = 4.0 * cfg.d * cnt["kept_pairs"]  # last call (a warm step when there are warm steps)
+    achieved = attn_flops / (steady["attn_kernel_ms"] * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": round(achieved / peak_tf, 4), "traffic": traffic, "peak_source": peak_src,
-                "kernel": "k_sparse_attn (warm-step launch)",
+                "frac": round(achieved / peak_tf, 4), "traffic": attn_traffic_bytes(cfg), "peak_source": peak_src,
+                "kernel": "k_sparse_attn (" + ("warm-step launch" if warm else "step-0 launch") + ")",
                 "algorithmic_flops_per_launch": attn_flops,
                 "computed_tile_flops_per_launch": 4.0 * cfg.d * cnt["computed_pairs"],
-                "computed_frac": round(4.0 * cfg.d * cnt["computed_pairs"] / (splitw["attn_kernel_ms"] * 1e-3) / 1e12
-                                       / peak_tf, 4)}
-    # achieved HBM fraction of the reduction stages of a warm call: the bytes they must read
+                "computed_frac": round(4.0 * cfg.d * cnt["computed_pairs"] / (steady["attn_kernel_ms"] * 1e-3)
+                                       / 1e12 / peak_tf, 4)}
+    # achieved HBM fraction of the reduction stages: the bytes they must read
     # (a tensor of B*H*L*d bf16 per pass) over their measured time
     hbm = peaks.get("hbm_gbs") or 6650.0
     tensor_bytes = 2.0 * cfg.B * cfg.H * cfg.L * cfg.d
-    passes = {"q_cluster_ms": 1 + 3 + 2,   # norms, 3 assignment passes, 2 centre updates
-              "k_cluster_ms": 1 + 3 + 2,   # norms, 3 passes, 2 updates
-              "stats_sort_ms": 1}          # per-cluster max / min, exact distances, SSE (one pass)
+    passes = ({"q_cluster_ms": 1 + (cfg.iters_warm + 1) + cfg.iters_warm,   # norms, assignment passes, updates
+               "k_cluster_ms": 1 + (cfg.iters_warm + 1) + cfg.iters_warm,
+               "stats_sort_ms": 1} if warm else
+              {"q_cluster_ms": 1 + (cfg.iters_q + 1) + cfg.iters_q, "stats_sort_ms": 1})
     red = {}
     for k, n in passes.items():
-        gbs = n * tensor_bytes / (splitw[k] * 1e-3) / 1e9
-        red[k.replace("_ms", "")] = {"algorithmic_bytes": n * tensor_bytes, "ms": round(splitw[k], 3),
+        gbs = n * tensor_bytes / (steady[k] * 1e-3) / 1e9
+        red[k.replace("_ms", "")] = {"algorithmic_bytes": n * tensor_bytes, "ms": round(steady[k], 3),
                                      "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / hbm, 4)}
 
+    clustering_ms = steady["total_ms"] - steady["attention_ms"]
     extra = {"step0": split0, "warm": splitw, "counters_last_call": cnt,
              "reduction_stages_hbm": red,
-             "clustering_share_warm": round((splitw["q_cluster_ms"] + splitw["k_cluster_ms"] + splitw["stats_sort_ms"]
-                                             + splitw["score_select_ms"]) / splitw["total_ms"], 4),
+             "clustering_share": round(clustering_ms / steady["total_ms"], 4),
              "assign_counters_since_create": lay.assign_counters(),
-             "kept_pair_frac": cnt["kept_pairs"] / float(cfg.H * cfg.L * cfg.L),
+             "kept_pair_frac": cnt["kept_pairs"] / float(cfg.B * cfg.H * cfg.L * cfg.L),
              "tile_efficiency": cnt["kept_pairs"] / max(1, cnt["computed_pairs"])}
-    # per-head state after the last call: key clusters, dense fallback, compactness, step-0 stages
     try:
         from cluster_routed_sparse_b200 import _lib as L
-        extra["per_head"] = {
-            "n_k": lay.tensor(L.AC_T_N_K).cpu().tolist(),
-            "dense": lay.tensor(L.AC_T_DENSE).cpu().tolist(),
-            "comp": [round(float(x), 5) for x in lay.tensor(L.AC_T_COMP).cpu().tolist()],
-            "stages": lay.tensor(L.AC_T_STAGES).cpu().tolist()}
+        n_k = lay.tensor(L.AC_T_N_K).cpu().numpy()
+        ksel = lay.tensor(L.AC_T_KSEL).cpu().numpy()
+        dense = lay.tensor(L.AC_T_DENSE).cpu().numpy()
+        sparse = dense == 0
+        extra["kept_cluster_frac"] = float(np.mean(ksel[sparse] / n_k[sparse])) if sparse.any() else 1.0
+        extra["per_head"] = {"n_k": n_k.tolist(), "dense": dense.tolist(),
+                             "comp": [round(float(x), 5) for x in lay.tensor(L.AC_T_COMP).cpu().tolist()],
+                             "stages": lay.tensor(L.AC_T_STAGES).cpu().tolist()}
     except Exception as exc:  # reporting only: never fail the bench line on it
         extra["per_head"] = {"unavailable": str(exc)[:200]}
-    # dense SDPA on the same tensors (one warm step's inputs)
+    # dense SDPA on the same tensors (a warm step's inputs when there are warm steps)
     if not args.no_sdpa and rank == 0:
-        extra["dense_sdpa"] = time_sdpa(*steps_in[1])
-        if extra["dense_sdpa"].get("ms"):
-            sd = extra["dense_sdpa"]["ms"]
-            extra["speedup_warm_layer_vs_sdpa"] = sd / splitw["total_ms"]
-            extra["speedup_sequence_vs_sdpa"] = sd * N_DENOISE / ms
+        sd = time_sdpa(*steps_in[1 if n_calls > 1 else 0])
+        extra["dense_sdpa"] = sd
+        if sd.get("ms"):
+            extra["speedup_layer_vs_sdpa"] = sd["ms"] / steady["total_ms"]
+            extra["speedup_sequence_vs_sdpa"] = sd["ms"] * n_calls / ms
+            # What the kept pairs allow: the layer cannot beat SDPA by more than
+            # t_sdpa / (t_clustering + kept FLOPs at the peak rate), nor, with free
+            # clustering, by more than t_sdpa / (kept FLOPs at the peak rate).
+            t_attn_peak = attn_flops / (peak_tf * 1e12) * 1e3
+            extra["speedup_bound_at_peak"] = sd["ms"] / (clustering_ms + t_attn_peak)
+            extra["speedup_bound_free_clustering"] = sd["ms"] / t_attn_peak
+            extra["speedup_bound_note"] = ("t_sdpa / (measured clustering + selection ms + kept-pair FLOPs at "
+                                           f"{peak_tf} TFLOP/s); the second bound drops the clustering")
 
-    # e2e through the host-buffer entry point
+    # e2e through the asynchronous host-buffer entry point
     e2e = None
     if not args.no_e2e:
-        e2e = time_e2e(lay, steps_in, cfg, dense_flops_layer, world, dist if world > 1 else None)
+        e2e = time_e2e(lay, steps_in, cfg, args, world, dist if world > 1 else None)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, tsec, desc, threads, twall = oracle_sample(CONFIG_ID)
-        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
-               "extrapolated_seconds": tsec, "sample_wall_seconds": twall}
+        smp = OracleSample(cfg, rows=256)
+        wall = smp.step0() + (smp.warm() if cfg.steps > 1 else 0.0)
+        cpu = {"value": smp.tflops(), "unit": "TFLOP/s", "cores": threads_used(), "kind": "oracle",
+               "sample": smp.describe(), "extrapolated_head_sequence_seconds": smp.sequence_seconds(),
+               "sample_wall_seconds": wall}
 
     if rank == 0:
         out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-               "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(),
+               "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(cfg, args),
                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-               "clocks": clk, "layer_ms_warm": splitw["total_ms"], "layer_ms_step0": split0["total_ms"],
-               "extra": extra}
+               "clocks": clk, "layer_ms_step0": split0["total_ms"],
+               "layer_ms_warm": splitw["total_ms"] if splitw else None, "extra": extra}
         print(json.dumps(out), flush=True)
     lay.close()
     if world > 1:
@@ -407,6 +493,7 @@ def time_sdpa(Q, K, V, reps: int = 3):
     import torch
     from torch.nn.attention import SDPBackend, sdpa_kernel
     F = torch.nn.functional
+    last = None
     for be, name in ((SDPBackend.CUDNN_ATTENTION, "cudnn"), (SDPBackend.FLASH_ATTENTION, "flash"),
                      (SDPBackend.EFFICIENT_ATTENTION, "efficient")):
         try:
@@ -429,39 +516,45 @@ def time_sdpa(Q, K, V, reps: int = 3):
     return {"backend": None, "ms": None, "error": last}
 
 
-def time_e2e(lay, steps_in, cfg, dense_flops_layer, world, dist):
-    """One ten-step sequence through the asynchronous host-buffer entry point
+def time_e2e(lay, steps_in, cfg, args, world, dist):
+    """The bench steps through the asynchronous host-buffer entry point
     (ac_layer_forward_host_async): every call copies that step's Q, K, V from
     pinned host memory and O back; a call's copies overlap its neighbours'
-    layers.  Timed from before the first call's input copy to the end of the
-    last call's output copy (ac_join on the timing stream)."""
+    layers.  Each repetition times args.steps bench steps back to back, from
+    before the first call's input copy to the end of the last call's output copy
+    (ac_join on the timing stream); the value is the median repetition."""
     import torch
-    host = []
-    for s in range(N_DENOISE):
-        host.append([x.cpu().pin_memory() for x in steps_in[s]])
+    n_calls = cfg.steps
+    host = [[x.cpu().pin_memory() for x in steps_in[s]] for s in range(n_calls)]
     hO = torch.empty_like(host[0][0]).pin_memory()
     torch.cuda.synchronize()
     lay.forward_host_async(*host[0], hO, warm=False)  # warm-up of the staging buffers and streams
     lay.synchronize()
     stream = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for s in range(N_DENOISE):
-        lay.forward_host_async(*host[s], hO, warm=s > 0)
-    lay.join()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    lay.synchronize()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    reps = []
+    for _ in range(max(1, args.e2e_reps)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            for s in range(n_calls):
+                lay.forward_host_async(*host[s], hO, warm=s > 0)
+        lay.join()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        lay.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        if dist is not None:
+            t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        reps.append(ms)
+    ms = float(np.median(reps))
     nbytes = cfg.B * cfg.H * cfg.L * cfg.d * 2
-    return {"value": world * N_DENOISE * dense_flops_layer / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-            "h2d_bytes_per_step": 3 * nbytes * N_DENOISE, "d2h_bytes_per_step": nbytes * N_DENOISE,
-            "ms_per_step": ms, "api": "ac_layer_forward_host_async x 10, ac_join",
-            "clock": "CUDA events around the ten host-buffer calls"}
+    return {"value": world * n_calls * dense_flops(cfg) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": 3 * nbytes * n_calls, "d2h_bytes_per_step": nbytes * n_calls,
+            "ms_per_step": ms, "ms_per_step_reps": [round(x, 2) for x in reps],
+            "api": f"ac_layer_forward_host_async x {n_calls} per step, ac_join",
+            "clock": "CUDA events around each repetition's host-buffer calls"}
 
 
 if __name__ == "__main__":

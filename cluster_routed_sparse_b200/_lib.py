@@ -50,7 +50,7 @@ class ACConfig(ctypes.Structure):
                 ("tau_mode", ctypes.c_int32), ("tau_value", ctypes.c_float), ("topk", ctypes.c_int32),
                 ("iters_q", ctypes.c_int32), ("iters_k", ctypes.c_int32), ("iters_warm", ctypes.c_int32),
                 ("stage_rule", ctypes.c_int32), ("seed", ctypes.c_uint64), ("scale", ctypes.c_float),
-                ("score_mode", ctypes.c_int32), ("tail_merge", ctypes.c_int32), ("reserved2", ctypes.c_int32)]
+                ("score_mode", ctypes.c_int32), ("tail_merge", ctypes.c_int32), ("unit0", ctypes.c_int32)]
 
 
 class ACStageTimes(ctypes.Structure):
@@ -78,6 +78,8 @@ class ACAssignCounters(ctypes.Structure):
 # every function that include/ac.h declares, with its ctypes signature
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
+# int32_t (*ac_sum_u64_fn)(void *user, uint64_t *data, int32_t count)
+SUM_U64_FN = ctypes.CFUNCTYPE(ctypes.c_int32, ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint64), ctypes.c_int32)
 SIGNATURES = {
     "ac_create": (_I, [ctypes.POINTER(ACConfig), _I, _I, _I, _I, ctypes.POINTER(_P)]),
     "ac_destroy": (_I, [_P]),
@@ -97,6 +99,9 @@ SIGNATURES = {
     "ac_get_assign_counters": (_I, [_P, ctypes.POINTER(ACAssignCounters), _I]),
     "ac_cluster_q_noalloc": (_I, [_P, _I, _I, _I, _I, _I, ctypes.c_uint64, _P, _P, _P, _P, _P]),
     "ac_state_export": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int64)]),
+    "ac_set_tau_exchange": (_I, [_P, SUM_U64_FN, _P]),
+    "ac_tau_mean_from_sums": (_I, [ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64, ctypes.POINTER(ctypes.c_float)]),
+    "ac_tau_radix_pick": (_I, [ctypes.POINTER(ctypes.c_uint64), _I, ctypes.POINTER(ctypes.c_uint32)]),
     "ac_state_import": (_I, [_P, _P, ctypes.c_int64]),
 }
 

@@ -52,6 +52,36 @@ def cluster_q_noalloc(Q, Cq: int, labels, centroids, iters: int = 10, seed: int 
                                    _ptr(labels), _ptr(centroids), _ptr(err), _stream()))
 
 
+def tau_exchange_allreduce(group=None, device=None):
+    """An exchange function for SparseLayer.set_tau_exchange that sums the
+    partial results over the ranks of a torch.distributed process group
+    (all-reduce; NCCL over NVLink when device is a CUDA device, gloo on CPU)."""
+    import torch.distributed as dist
+
+    def fn(vals):
+        t = torch.as_tensor(vals.astype("int64"), device=device or "cpu")
+        dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+        vals[:] = t.cpu().numpy().astype(vals.dtype)
+    return fn
+
+
+def tau_mean_from_sums(factor: float, fixed_sum: int, n: int) -> float:
+    """ac_tau_mean_from_sums: tau = factor x the mean of the pooled distances,
+    from the sum of floor(d_i 2^24) and their number."""
+    out = ctypes.c_float(0.0)
+    check(_lib.load().ac_tau_mean_from_sums(float(factor), int(fixed_sum), int(n), ctypes.byref(out)))
+    return float(out.value)
+
+
+def tau_radix_pick(hist, shift: int, state):
+    """ac_tau_radix_pick on a 256-bin summed histogram (sequence of ints) and the
+    selection state [prefix, mask, rank] (updated and returned)."""
+    h = (ctypes.c_uint64 * 256)(*[int(x) for x in hist])
+    st = (ctypes.c_uint32 * 3)(*[int(x) for x in state])
+    check(_lib.load().ac_tau_radix_pick(h, int(shift), st))
+    return [int(st[0]), int(st[1]), int(st[2])]
+
+
 class SparseLayer:
     """One cluster-routed sparse attention layer context for [B, H, L, d] inputs.
 
@@ -61,24 +91,46 @@ class SparseLayer:
     def __init__(self, B: int, H: int, L: int, d: int, *, Cq: int, m0: int, n_max: int,
                  tau_mode: int, tau_value: float, topk: int, iters_q: int = 10,
                  iters_k: int = 10, iters_warm: int = 2, seed: int = 1234, scale: float = 0.0,
-                 stage_rule: int = 0, score_mode: int = 0, tail_merge: int = 0):
+                 stage_rule: int = 0, score_mode: int = 0, tail_merge: int = 0, unit0: int = 0):
         self.lib = _lib.load()
         self.B, self.H, self.L, self.d = B, H, L, d
         self.cfg = ACConfig(Cq, m0, n_max, tau_mode, float(tau_value), topk, iters_q, iters_k,
                             iters_warm, stage_rule, seed & (2**64 - 1), float(scale), score_mode,
-                            tail_merge, 0)
+                            tail_merge, unit0)
         self.Cq, self.Ccap = Cq, n_max + m0
         h = ctypes.c_void_p()
         check(self.lib.ac_create(ctypes.byref(self.cfg), B, H, L, d, ctypes.byref(h)))
         self.ctx = h
 
     @classmethod
-    def from_config(cls, cfg, seed: int = 1234, B=None, H=None, L=None):
-        """Build from a synth.LayerConfig (shape overrides allowed)."""
+    def from_config(cls, cfg, seed: int = 1234, B=None, H=None, L=None, **kw):
+        """Build from a synth.LayerConfig (shape overrides allowed; keyword
+        arguments such as score_mode or tail_merge are passed on)."""
         return cls(B or cfg.B, H or cfg.H, L or cfg.L, cfg.d, Cq=cfg.Cq, m0=cfg.m0, n_max=cfg.n_max,
                    tau_mode=cfg.tau_mode, tau_value=cfg.tau_value, topk=cfg.topk,
                    iters_q=cfg.iters_q, iters_k=cfg.iters_k, iters_warm=cfg.iters_warm, seed=seed,
-                   stage_rule=cfg.stage_rule)
+                   stage_rule=cfg.stage_rule, **kw)
+
+    def set_tau_exchange(self, fn):
+        """Pool tau with other contexts that hold the other heads of the layer:
+        fn(vals) receives a numpy uint64 array of partial sums and must replace
+        it, in place, by the sums over all contexts (see ac_set_tau_exchange);
+        None: tau from this context's heads."""
+        import numpy as np
+        if fn is None:
+            self._xchg = None
+            check(self.lib.ac_set_tau_exchange(self.ctx, _lib.SUM_U64_FN(), None), self.ctx)
+            return
+
+        def cb(_user, data, count):
+            try:
+                vals = np.ctypeslib.as_array(data, shape=(count,))
+                fn(vals)
+                return 0
+            except Exception:  # reported to the library as a failed exchange
+                return 1
+        self._xchg = _lib.SUM_U64_FN(cb)  # kept alive with the context
+        check(self.lib.ac_set_tau_exchange(self.ctx, self._xchg, None), self.ctx)
 
     # ------------------------------------------------------------------ calls
     def cluster_q(self, Q, init=None, iters: int = -1, labels=None, centroids=None):

@@ -13,7 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libac.so")
-SOURCES = ["ac_api.cu", "cluster_kernels.cu", "assign_mma.cu", "score_kernels.cu", "attn_kernel.cu", "noalloc.cu"]
+SOURCES = ["ac_api.cu", "cluster_kernels.cu", "assign_mma.cu", "score_kernels.cu", "quest_mma.cu", "attn_kernel.cu",
+           "noalloc.cu"]
 HEADERS = ["ac_device.cuh", "ac_internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -285,6 +285,7 @@ ac_status cluster_q_impl(ac_ctx *c, const bf16 *Q, const float *init, int iters,
     } else {
         SeedArgs sa{Q, c->inv_q, L, nullptr, nullptr, c->L, c->cent_q, (int64_t)c->Cq * c->d, nullptr,
                     nullptr, c->Cq, c->Cq, c->cfg.seed, 0, c->BH, c->d};
+        sa.unit0 = c->cfg.unit0;
         CK(launch_seed(sa, s), "seed q");
     }
     Lloyd k;
@@ -297,6 +298,57 @@ ac_status cluster_q_impl(ac_ctx *c, const bf16 *Q, const float *init, int iters,
     make_fast(c, k, Q, true, c->cent_q, (int64_t)c->Cq * c->d, nullptr, c->Cq, c->labels_q, nullptr);
     CK(run_lloyd(c, k, iters, true, s), "q lloyd");
     c->have_q = true;
+    return AC_OK;
+}
+
+// The pooled tau when the heads of one layer are split over several contexts
+// (ranks): each context reduces its own stage-0 distances and the caller's
+// exchange function sums the partial results over the contexts, so tau is the
+// one a single context over all heads computes, bit for bit (the fixed-point
+// sum and the radix-select histograms are order-independent integers).
+//  mean rule:       {sum floor(d_i 2^24), n}, then tau on the host as k_tau_mean forms it;
+//  percentile rule: {n}, then per 8-bit digit the 256-bin histogram of the
+//                   distances that match the digits chosen so far.
+ac_status exchange_tau(ac_ctx *c, cudaStream_t s) {
+    const int BH = c->BH, L = c->L;
+    uint64_t *hx = c->h_xchg;
+    float tau = 0.f;
+    if (c->cfg.tau_mode == AC_TAU_MEAN_FACTOR) {
+        CK(cudaMemcpyAsync(hx, c->tau_acc, sizeof(uint64_t), cudaMemcpyDeviceToHost, s), "tau partial");
+        CK(cudaStreamSynchronize(s), "tau partial");
+        hx[1] = (uint64_t)BH * (uint64_t)L;
+        if (c->xchg(c->xchg_user, hx, 2) != 0) return fail(c, AC_ERR_STATE, "tau exchange function failed");
+        ac_status st = ac_tau_mean_from_sums(c->cfg.tau_value, hx[0], hx[1], &tau);
+        if (st != AC_OK) return fail(c, st, "tau exchange: no distances");
+    } else {
+        hx[0] = (uint64_t)BH * (uint64_t)L;
+        if (c->xchg(c->xchg_user, hx, 1) != 0) return fail(c, AC_ERR_STATE, "tau exchange function failed");
+        const uint64_t n_total = hx[0];
+        if (n_total == 0 || n_total > 0xFFFFFFFFull) return fail(c, AC_ERR_INVALID_ARG, "tau exchange: bad key count");
+        int64_t idx = ((int64_t)c->cfg.tau_value * (int64_t)n_total + 999) / 1000 - 1;
+        idx = std::max<int64_t>(0, std::min<int64_t>(idx, (int64_t)n_total - 1));
+        uint32_t state[3] = {0u, 0u, (uint32_t)idx};  // prefix, mask, rank within the prefix
+        uint32_t *hh = reinterpret_cast<uint32_t *>(hx + 256);
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
+            uint32_t init[259];
+            for (int i = 0; i < 256; ++i) init[i] = 0u;
+            init[256] = state[0];
+            init[257] = state[1];
+            init[258] = state[2];
+            CK(cudaMemcpyAsync(c->radix, init, sizeof(init), cudaMemcpyHostToDevice, s), "radix state");
+            CK(launch_radix_hist(c->st_dist, c->st_m, L, BH, c->radix, shift, s), "radix histogram");
+            CK(cudaMemcpyAsync(hh, c->radix, 256 * sizeof(uint32_t), cudaMemcpyDeviceToHost, s), "histogram");
+            CK(cudaStreamSynchronize(s), "histogram");
+            for (int i = 0; i < 256; ++i) hx[i] = hh[i];
+            if (c->xchg(c->xchg_user, hx, 256) != 0) return fail(c, AC_ERR_STATE, "tau exchange function failed");
+            ac_status st = ac_tau_radix_pick(hx, shift, state);
+            if (st != AC_OK) return fail(c, st, "tau exchange: inconsistent histograms");
+        }
+        std::memcpy(&tau, &state[0], sizeof(float));
+    }
+    CK(cudaMemcpyAsync(c->tau, &tau, sizeof(float), cudaMemcpyHostToDevice, s), "tau");
+    CK(cudaStreamSynchronize(s), "tau");  // `init` and the pinned buffer are reused
     return AC_OK;
 }
 
@@ -351,6 +403,7 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
         // line 12: KMeans(U, m_t), stage centres appended after the n_k existing ones
         SeedArgs sa{K, nullptr, L, c->u_idx, c->u_cnt, 0, c->cent_k, cstride, c->n_k, c->st_m, 0, max_m,
                     c->cfg.seed, 1 + t, BH, d};
+        sa.unit0 = c->cfg.unit0;
         CK(launch_seed(sa, s), "seed k");
         Lloyd k;
         k.as = AssignArgs{K, nullptr, L, c->u_idx, c->u_cnt, 0, c->cent_k, cstride, c->n_k, c->st_m, 0,
@@ -385,7 +438,10 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
            "stage dist");
         if (t == 0) {
             const int64_t n_total = (int64_t)BH * L;
-            if (c->cfg.tau_mode == AC_TAU_MEAN_FACTOR) {
+            if (c->xchg && c->cfg.tau_mode != AC_TAU_ABSOLUTE) {
+                ac_status st = exchange_tau(c, s);
+                if (st != AC_OK) return st;
+            } else if (c->cfg.tau_mode == AC_TAU_MEAN_FACTOR) {
                 CK(launch_tau_mean(c->tau_acc, nullptr, n_total, c->cfg.tau_value, c->tau, s), "tau mean");
             } else if (c->cfg.tau_mode == AC_TAU_PERCENTILE) {
                 CK(launch_tau_percentile(c->st_dist, c->st_m, L, BH, n_total, (int)c->cfg.tau_value, c->radix,
@@ -464,6 +520,12 @@ ac_status score_select_impl(ac_ctx *c, int topk, cudaStream_t s) {
                  c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->rbox, c->pgoff, c->nrange};
     a.score_mode = c->cfg.score_mode;
     a.cent_k = c->cent_k;
+    a.tm_kmax = &c->tm_kmax;
+    a.tm_kmin = &c->tm_kmin;
+    a.kabs = c->kabs;
+    a.err = c->err;
+    a.exact_cuda_cores = c->exact_scores;
+    a.bound_scale = c->quest_bound_scale;
     CK(launch_score_select(a, s), "score select");
     if (c->cfg.tail_merge) {
         TailMergeArgs t{c->sel, c->ksel, c->dense, c->labels_q, c->perm_q, c->offs_q, c->counts_q, c->counts_k,
@@ -502,10 +564,10 @@ void free_all(ac_ctx *c) {
                    c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err, c->chi_q, c->chi_k, c->cn,
                    c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats, c->rbox, c->pgoff, c->nrange,
                    c->sort_scratch, c->cnp_k, c->rowsq_u, c->cent_st, c->perm_qm, c->offs_qm, c->counts_qm,
-                   c->tm_scratch};
+                   c->tm_scratch, c->kabs};
     for (void *p : dev)
         if (p) cudaFree(p);
-    void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err};
+    void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err, c->h_xchg};
     for (void *p : host)
         if (p) cudaFreeHost(p);
     for (auto &e : c->ev)
@@ -541,7 +603,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     if (cfg->Cq < 1 || cfg->Cq > L || cfg->m0 < 1 || cfg->m0 > L || cfg->n_max < 1 || cfg->iters_q < 0 ||
         cfg->iters_k < 0 || cfg->iters_warm < 0 || cfg->tau_mode < 0 || cfg->tau_mode > 2 || cfg->topk == 0 ||
         cfg->stage_rule < 0 || cfg->stage_rule > 1 || (cfg->score_mode != 0 && cfg->score_mode != 1) ||
-        cfg->tail_merge < 0 || cfg->tail_merge > 2 || cfg->reserved2 != 0 || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
+        cfg->tail_merge < 0 || cfg->tail_merge > 2 || cfg->unit0 < 0 || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
         return AC_ERR_INVALID_ARG;
     if ((int64_t)B * H * L >= (int64_t)1 << 31) return AC_ERR_INVALID_ARG;
     if (cfg->tau_mode == AC_TAU_PERCENTILE && (cfg->tau_value < 1.f || cfg->tau_value > 1000.f))
@@ -577,6 +639,10 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     {
         const char *ev = std::getenv("AC_EXACT_ASSIGN");
         c->fast_assign = !(ev && ev[0] == '1');
+        const char *es = std::getenv("AC_EXACT_SCORES");
+        c->exact_scores = es && es[0] == '1';
+        const char *bs = std::getenv("AC_QUEST_BOUND_SCALE");
+        c->quest_bound_scale = bs ? std::max(1.0f, (float)std::atof(bs)) : 1.0f;
     }
     c->Cpad_q = (c->Cq + 31) & ~31;
     c->CH_q = std::min(96, c->Cpad_q);  // two-term chunks (c_hi + c_lo) of at most 96 centres
@@ -620,6 +686,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->radix, 260));
     A(dalloc(&c->sort_scratch, BH * 128 * std::max(Cc, Cq)));
     A(dalloc(&c->score, BH * Cq * Cc));
+    A(dalloc(&c->kabs, BH * Cc));
     A(dalloc(&c->sel, BH * Cq * Cc));
     A(dalloc(&c->ksel, BH));
     A(dalloc(&c->ranges, BH * Cq * Cc));
@@ -656,6 +723,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(cudaMallocHost(&c->h_n_k, BH * sizeof(int)));
     A(cudaMallocHost(&c->h_dense, BH));
     A(cudaMallocHost(&c->h_err, sizeof(uint32_t)));
+    A(cudaMallocHost(&c->h_xchg, 256 * sizeof(uint64_t) + 256 * sizeof(uint32_t)));
     for (auto &e : c->ev) A(cudaEventCreate(&e));
     if (!okm) {
         free_all(c);
@@ -681,7 +749,9 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     if (!maps_ok ||
         make_tmap(c, &c->tm_chi_q, c->chi_q, (int64_t)2 * BH * c->Cpad_q, d, c->CH_q) != AC_OK ||
         make_tmap(c, &c->tm_chi_k, c->chi_k, (int64_t)BH * c->Cpad_k, d, c->CH_k) != AC_OK ||
-        make_tmap_plain16(c, &c->tm_cnp_k, c->cnp_k, (int64_t)BH * c->Cpad_k, c->CH_k) != AC_OK) {
+        make_tmap_plain16(c, &c->tm_cnp_k, c->cnp_k, (int64_t)BH * c->Cpad_k, c->CH_k) != AC_OK ||
+        make_tmap(c, &c->tm_kmax, c->kmax, (int64_t)BH * c->Ccap, d, 64) != AC_OK ||
+        make_tmap(c, &c->tm_kmin, c->kmin, (int64_t)BH * c->Ccap, d, 64) != AC_OK) {
         free_all(c);
         delete c;
         return AC_ERR_CUDA;
@@ -902,6 +972,41 @@ ac_status ac_get_tensor(ac_ctx *c, int32_t which, void **ptr, int64_t shape[4]) 
 ac_status ac_get_launch_count(int64_t *out) {
     if (!out) return AC_ERR_INVALID_ARG;
     *out = (int64_t)g_launches.load(std::memory_order_relaxed);
+    return AC_OK;
+}
+
+ac_status ac_set_tau_exchange(ac_ctx *c, ac_sum_u64_fn fn, void *user) {
+    if (!c) return AC_ERR_INVALID_ARG;
+    c->xchg = fn;
+    c->xchg_user = user;
+    return AC_OK;
+}
+
+ac_status ac_tau_mean_from_sums(float factor, uint64_t fixed_sum, uint64_t n, float *tau) {
+    if (!tau || n == 0) return AC_ERR_INVALID_ARG;
+    // the operations of k_tau_mean: fp64, round to nearest, then fp32
+    const double mean = ((double)fixed_sum / 16777216.0) / (double)n;
+    *tau = (float)((double)factor * mean);
+    return AC_OK;
+}
+
+ac_status ac_tau_radix_pick(const uint64_t *hist, int32_t shift, uint32_t *state) {
+    if (!hist || !state || shift < 0 || shift > 24 || (shift & 7)) return AC_ERR_INVALID_ARG;
+    // the digit of the rank-th smallest (0-based) among the matching distances
+    const uint64_t rank = state[2];
+    uint64_t cum = 0;
+    int dg = -1;
+    for (int i = 0; i < 256; ++i) {
+        if (cum + hist[i] > rank) {
+            dg = i;
+            break;
+        }
+        cum += hist[i];
+    }
+    if (dg < 0) return AC_ERR_INVALID_ARG;
+    state[2] = (uint32_t)(rank - cum);
+    state[0] |= (uint32_t)dg << shift;
+    state[1] |= 255u << shift;
     return AC_OK;
 }
 

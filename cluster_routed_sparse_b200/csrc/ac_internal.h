@@ -59,6 +59,8 @@ struct ac_ctx {
 
     // ---- selection (Algorithm 3 line 9)
     float *score;      // [BH, Cq, Ccap]
+    float *kabs;       // [BH, Ccap]      max_d max(|Kmax_d|, |Kmin_d|) per key cluster
+    CUtensorMap tm_kmax, tm_kmin;  // Kmax / Kmin rows in 64-row boxes (tensor-core Eq. (1))
     int *sel;          // [BH, Cq, Ccap]
     int *ksel;         // [BH]
     int2 *ranges;      // [BH, Cq, Ccap]  (start row in cluster order, count)
@@ -90,6 +92,8 @@ struct ac_ctx {
     float *cent_st;            // [BH, m0, d] the stage's centres, copied out of cent_k for the GEMM
     int num_sms;
     bool fast_assign;
+    bool exact_scores;  // Eq. (1) on CUDA cores instead of the tensor cores
+    float quest_bound_scale;  // >= 1: the tensor-core Eq. (1) path rescores a wider band
     long long n_fast, n_exact, n_fast_rows;
 
     // ---- attention
@@ -120,6 +124,9 @@ struct ac_ctx {
     int *h_n_k;
     uint8_t *h_dense;
     uint32_t *h_err;
+    uint64_t *h_xchg;   // [256] u64 + [256] u32: the tau exchange's partial sums
+    ac_sum_u64_fn xchg = nullptr;  // sums partial results over the contexts of one layer
+    void *xchg_user = nullptr;
 
     bool have_q, have_k, have_state;
     bool timing;        // record events around the attention kernel
@@ -228,6 +235,7 @@ struct SeedArgs {
     float *C; int64_t cstride; const int *coff;
     const int *m; int m_const; int max_m;
     uint64_t seed; int tag; int BH, d;
+    int unit0 = 0;  // unit index of the first unit (a head subset of a larger layer)
 };
 cudaError_t launch_seed(const SeedArgs &a, cudaStream_t s);
 
@@ -237,6 +245,8 @@ cudaError_t launch_stage_dist(const float *dmin, float *dist, const int *u_cnt, 
                               int64_t L, int BH, unsigned long long *tau_acc, cudaStream_t s);
 cudaError_t launch_tau_mean(const unsigned long long *tau_acc, const int *u_cnt0_total_unused,
                             int64_t n_total, float factor, float *tau, cudaStream_t s);
+cudaError_t launch_radix_hist(const float *dist, const int *st_m, int64_t L, int BH, uint32_t *radix, int shift,
+                              cudaStream_t s);
 cudaError_t launch_tau_percentile(const float *dist, const int *st_m, int64_t L, int BH,
                                   int64_t n_total, int permille, uint32_t *radix, float *tau,
                                   cudaStream_t s);
@@ -270,8 +280,17 @@ struct SelectArgs {
     int *rbox; int *pgoff; int *nrange;
     int score_mode = 0;            // 0: Eq. (1) bound; 1: mean-based (q . centre of the key cluster)
     const float *cent_k = nullptr;  // [BH, Ccap, d] key centres (score_mode 1)
+    // tensor-core path of Eq. (1) (quest_mma.cu): Kmax / Kmin rows [BH * Ccap, d]
+    // in 64-row boxes, the per-cluster column bounds, the error word
+    const CUtensorMap *tm_kmax = nullptr, *tm_kmin = nullptr;
+    float *kabs = nullptr;         // [BH, Ccap]
+    uint32_t *err = nullptr;
+    bool exact_cuda_cores = false;  // force the CUDA-core kernels (k_quest_scores + k_score_select)
+    float bound_scale = 1.f;        // widens the tensor-core path's error bound (tests of the rescoring)
 };
 cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s);
+bool quest_mma_supported(const SelectArgs &a);
+cudaError_t launch_quest_select_mma(const SelectArgs &a, cudaStream_t s);
 
 // Tail merging of the query tiles after the selection (see ac_config.tail_merge):
 // regroups the rows of Qp (perm_qm, offs_qm, counts_qm), rewrites the key

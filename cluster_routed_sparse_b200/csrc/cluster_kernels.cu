@@ -878,7 +878,7 @@ __global__ void k_seed(SeedArgs a) {
     const int m = a.m ? a.m[h] : a.m_const;
     if (j >= m) return;
     const int64_t n = a.nrows ? a.nrows[h] : a.nrows_const;
-    const int64_t pos = stratum_pick(a.seed, h, a.tag, n, m, j);
+    const int64_t pos = stratum_pick(a.seed, (int64_t)a.unit0 + h, a.tag, n, m, j);
     const int64_t tok = a.rows ? a.rows[(int64_t)h * a.L + pos] : pos;
     const float sc = a.inv ? a.inv[(int64_t)h * a.L + tok] : 1.f;
     const int off = a.coff ? a.coff[h] : 0;
@@ -997,6 +997,13 @@ __global__ void k_radix_pick(uint32_t *radix, int shift, float *tau, int last) {
 
 __global__ void k_radix_init(uint32_t *radix, uint32_t rank) {
     for (int i = threadIdx.x; i < 259; i += blockDim.x) radix[i] = (i == 258) ? rank : 0u;
+}
+
+cudaError_t launch_radix_hist(const float *dist, const int *st_m, int64_t L, int BH, uint32_t *radix, int shift,
+                              cudaStream_t s) {
+    k_radix_hist<<<dim3(64, BH), 256, 0, s>>>(dist, st_m, L, radix, shift);
+    AC_NOTE_LAUNCH();
+    return cudaGetLastError();
 }
 
 cudaError_t launch_tau_percentile(const float *dist, const int *st_m, int64_t L, int BH, int64_t n_total,

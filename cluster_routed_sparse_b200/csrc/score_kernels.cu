@@ -1,10 +1,12 @@
 // score_kernels.cu -- critical-cluster selection (AdaCluster, arXiv
 // 2604.18348, Sec. 3.2.3 Eq. (1) / Algorithm 2, and Algorithm 3 line 9).
 //
-// At cluster granularity the score matrix of one head is Cq x n_k (65 x ~1000)
-// over d = 128: about 17 MFLOP per head, far too small to fill the tensor
-// cores, so it runs on CUDA cores in fp32, each score summed in dimension
-// order.  k_quest_scores: one block per (head, 32 key clusters) stages the
+// The method's path runs Eq. (1) on the tensor cores, fused with the top-k
+// (quest_mma.cu).  The kernels here serve the mean-based ablation
+// (score_mode 1) and, on request (AC_EXACT_SCORES=1 at ac_create), Eq. (1) on
+// CUDA cores in fp32, each score summed in dimension order, the reference
+// arithmetic the tensor-core path reproduces.
+// k_quest_scores: one block per (head, 32 key clusters) stages the
 // clusters' bounds and all query centroids in shared memory, each thread
 // accumulating the scores of one key cluster against 9 query centroids per
 // pass.
@@ -455,10 +457,22 @@ cudaError_t launch_tail_merge(const TailMergeArgs &a, cudaStream_t s) {
 }
 
 cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s) {
+    cudaError_t e;
+    if (!a.exact_cuda_cores && quest_mma_supported(a)) {
+        // Eq. (1) on the tensor cores fused with the top-k and the key ranges
+        // (quest_mma.cu); it needs each cluster's first 8-row group first
+        k_group_offsets<<<a.BH, SEL_THREADS, 0, s>>>(a.counts_k, a.n_k, a.Ccap, a.pgoff);
+        AC_NOTE_LAUNCH();
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_quest_select_mma(a, s)) != cudaSuccess) return e;
+        k_tile_prefix<<<1, 1024, 0, s>>>(a.counts_q, a.BH * a.Cq, a.tile_prefix);
+        AC_NOTE_LAUNCH();
+        return cudaGetLastError();
+    }
     const size_t qsm = (size_t)(2 * a.d * QS_C + a.Cq * a.d) * 4;
     if (qsm > 200 * 1024) return cudaErrorInvalidValue;  // ac_create keeps Cq within this
-    cudaError_t e = cudaFuncSetAttribute(k_quest_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(qsm < 48 * 1024 ? 48 * 1024 : qsm));
+    e = cudaFuncSetAttribute(k_quest_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(qsm < 48 * 1024 ? 48 * 1024 : qsm));
     if (e != cudaSuccess) return e;
     k_quest_scores<<<dim3((a.Ccap + QS_C - 1) / QS_C, a.BH), SEL_THREADS, qsm, s>>>(a);
     AC_NOTE_LAUNCH();

@@ -96,7 +96,12 @@ typedef struct ac_config {
                             each other's nearest selection (Hamming) and fit one
                             128-row tile pool them: the higher index hands its
                             tail to the lower, which attends to the union      */
-    int32_t reserved2;   /* must be 0                                             */
+    int32_t unit0;       /* (batch, head) index of this context's first unit in
+                            the layer, >= 0: unit u of the context seeds its
+                            initial centres as unit unit0 + u, so a layer split
+                            over contexts (ac_set_tau_exchange) clusters each
+                            head as a single context over all heads would; 0
+                            for a whole layer                                */
 } ac_config;
 
 typedef struct ac_ctx ac_ctx;
@@ -326,6 +331,41 @@ AC_API ac_status ac_cluster_q_noalloc(const uint16_t *Q, int32_t BH, int32_t L, 
                                       int32_t iters, uint64_t seed, const float *init_centroids,
                                       int32_t *labels_out, float *centroids_out, uint32_t *err_out,
                                       void *stream);
+
+/* Splitting the heads of one layer over several contexts (one per GPU or
+ * rank; Algorithm 1 works per (batch, head), the only coupling of the heads is
+ * tau, pooled over the stage-0 distances of every head of the layer, Sec. 4.1).
+ * With an exchange function set, the step-0 key clustering of the context
+ * reduces its own heads' stage-0 distances and calls fn(user, data, count) on
+ * the calling thread: data (host memory) holds `count` partial sums that fn
+ * must replace, in place, by their sums over all contexts of the layer (for
+ * example an all-reduce over the ranks), returning 0 on success.  The calls
+ * are, in order, for the mean rule: count 2, {sum over the distances d_i of
+ * floor(d_i 2^24), number of distances}; for the percentile rule: count 1, the
+ * number of distances, then four times count 256, the histogram of the next
+ * 8-bit digit of the distances' bit patterns among those that match the digits
+ * chosen so far (radix select, most significant digit first).  Every context
+ * of the layer must take part in the same step-0 calls.  The absolute rule
+ * exchanges nothing.  The pooled tau equals the one a single context over all
+ * heads computes, bit for bit.  fn = NULL: tau from this context's heads.
+ * Errors: INVALID_ARG; the step-0 call returns AC_ERR_STATE if fn fails. */
+typedef int32_t (*ac_sum_u64_fn)(void *user, uint64_t *data, int32_t count);
+AC_API ac_status ac_set_tau_exchange(ac_ctx *ctx, ac_sum_u64_fn fn, void *user);
+
+/* Host-side steps of the pooled tau (no device work; used by the step-0
+ * clustering when an exchange function is set, and callable on their own).
+ * ac_tau_mean_from_sums: tau = factor * ((fixed_sum / 2^24) / n), in fp64
+ * rounded to nearest, then to fp32 (Sec. 4.1, 1.5x the mean stage-0
+ * distance).  ac_tau_radix_pick: one digit of a nearest-rank selection:
+ * state = {prefix, mask, rank}; given the summed 256-bin histogram of the
+ * digit at `shift` (24, 16, 8, 0) among the distances whose bits match
+ * prefix under mask, it appends the digit that holds the rank-th smallest
+ * (0-based) distance and leaves the rank within that digit; after the pass
+ * with shift 0, prefix is the bit pattern of the selected distance.
+ * Errors: INVALID_ARG (n = 0, bad shift, or a histogram with fewer entries than
+ * rank + 1). */
+AC_API ac_status ac_tau_mean_from_sums(float factor, uint64_t fixed_sum, uint64_t n, float *tau);
+AC_API ac_status ac_tau_radix_pick(const uint64_t *hist, int32_t shift, uint32_t *state);
 
 /* Number of kernels libac has launched in this process so far (all contexts). */
 AC_API ac_status ac_get_launch_count(int64_t *out);
