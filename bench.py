@@ -15,7 +15,7 @@ metric: effective TFLOP/s = calls x 4*B*H*L^2*d / t (dense-equivalent FLOPs of
 the layer calls over their device time); higher is better.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config N] [--topk -PERMILLE] [--stage-rule R] [--tail-merge M]
+                    [--config N] [--topk -PERMILLE] [--stage-rule R] [--tail-merge M] [--compensate]
 
 Under torchrun every rank runs its own layer (independent problems, weak
 scaling, no collective on the data path); time is the max over ranks.
@@ -68,11 +68,13 @@ def workload_config(cfg, args):
     topk = f"top-k {-cfg.topk / 10:g}% of key clusters" if cfg.topk < 0 else f"top-k {cfg.topk}"
     return {"workload": f"{cfg.name}: B={cfg.B} H={cfg.H} L={cfg.L} d={cfg.d} bf16, {seq}, Cq={cfg.Cq}, "
                         f"m0={cfg.m0}, N_max={cfg.n_max}, {tau_text(cfg)}, {topk}, stage rule {cfg.stage_rule}"
-                        + (f", tail merging {args.tail_merge}" if args.tail_merge else ""),
+                        + (f", tail merging {args.tail_merge}" if args.tail_merge else "")
+                        + (", centroid compensation" if args.compensate else ""),
             "global_batch": cfg.B, "seq_len": cfg.L, "heads": cfg.H, "head_dim": cfg.d,
             "l2": ("inputs larger than L2 (3 x 774 MB per denoising step, 10 distinct steps)" if steps > 1
                    else "L2 flushed (512 MB write) before every timed bench step, outside its events"),
-            "parallelism": "one layer per rank"}
+            "parallelism": ("the layer's heads split over the ranks, tau pooled by an NCCL all-reduce"
+                            if getattr(args, "split_heads", False) else "one layer per rank")}
 
 
 # ---------------------------------------------------------------- inputs
@@ -306,7 +308,12 @@ def main():
     ap.add_argument("--topk", type=int, default=0, help="override the top-k (negative: -permille of n_k)")
     ap.add_argument("--stage-rule", type=int, default=None, help="override the m_t rule of stages t > 0")
     ap.add_argument("--tail-merge", type=int, default=0, help="query-tile tail merging mode (0, 1, 2)")
+    ap.add_argument("--compensate", action="store_true",
+                    help="centroid compensation of the unselected key clusters")
     ap.add_argument("--e2e-reps", type=int, default=3, help="repetitions of the end-to-end measurement")
+    ap.add_argument("--split-heads", action="store_true",
+                    help="under torchrun: one layer, its heads split over the ranks (strong scaling), the "
+                         "step-0 tau pooled by an all-reduce")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sdpa", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -324,7 +331,12 @@ def main():
     n_calls = cfg.steps  # layer calls per bench step
 
     # inputs first (spawn pool, before any CUDA call); each rank its own layer
-    x0 = generate_step0_f32(cfg, list(range(cfg.H)), max(1, args.procs // max(1, world)))
+    split = args.split_heads and world > 1
+    h_lo, h_hi = (rank * cfg.H // world, (rank + 1) * cfg.H // world) if split else (0, cfg.H)
+    heads = list(range(h_lo, h_hi))
+    import dataclasses
+    lcfg = dataclasses.replace(cfg, H=len(heads)) if split else cfg  # this rank's share
+    x0 = generate_step0_f32(cfg, heads, max(1, args.procs // max(1, world)))
 
     import torch
     import torch.distributed as dist
@@ -335,9 +347,18 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     from cluster_routed_sparse_b200.api import SparseLayer
 
-    steps_in = denoise_inputs(x0, n_calls, seed=100 + rank, device=dev)
+    steps_in = denoise_inputs(x0, n_calls, seed=100 + (h_lo if split else rank), device=dev)
     del x0
-    lay = SparseLayer.from_config(cfg, seed=1234 + rank, tail_merge=args.tail_merge)
+    if split:
+        # this rank's heads of the one layer; the initial centres keep each head's
+        # seeds and the step-0 tau is pooled over all ranks (ac_set_tau_exchange)
+        from cluster_routed_sparse_b200.api import tau_exchange_allreduce
+        lay = SparseLayer.from_config(cfg, seed=1234, H=len(heads), tail_merge=args.tail_merge,
+                                      compensate=1 if args.compensate else 0, unit0=h_lo)
+        lay.set_tau_exchange(tau_exchange_allreduce(device=dev))
+    else:
+        lay = SparseLayer.from_config(cfg, seed=1234 + rank, tail_merge=args.tail_merge,
+                                      compensate=1 if args.compensate else 0)
     O = torch.empty_like(steps_in[0][0])
     flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
 
@@ -380,7 +401,7 @@ def main():
     lay.synchronize()
     ms_local = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     ms = max_over_ranks(ms_local, world, dev, dist if world > 1 else None)
-    value = job_tflops(ms, world, cfg)
+    value = job_tflops(ms, 1 if split else world, cfg)
 
     # stage split (from the same timed calls): step 0 and the warm steps
     step0 = [c for i, c in enumerate(per_call) if i % n_calls == 0]
@@ -406,7 +427,7 @@ def main():
     attn_flops = 4.0 * cfg.d * cnt["kept_pairs"]  # last call (a warm step when there are warm steps)
     achieved = attn_flops / (steady["attn_kernel_ms"] * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": round(achieved / peak_tf, 4), "traffic": attn_traffic_bytes(cfg), "peak_source": peak_src,
+                "frac": round(achieved / peak_tf, 4), "traffic": attn_traffic_bytes(lcfg), "peak_source": peak_src,
                 "kernel": "k_sparse_attn (" + ("warm-step launch" if warm else "step-0 launch") + ")",
                 "algorithmic_flops_per_launch": attn_flops,
                 "computed_tile_flops_per_launch": 4.0 * cfg.d * cnt["computed_pairs"],
@@ -415,7 +436,7 @@ def main():
     # achieved HBM fraction of the reduction stages: the bytes they must read
     # (a tensor of B*H*L*d bf16 per pass) over their measured time
     hbm = peaks.get("hbm_gbs") or 6650.0
-    tensor_bytes = 2.0 * cfg.B * cfg.H * cfg.L * cfg.d
+    tensor_bytes = 2.0 * lcfg.B * lcfg.H * lcfg.L * lcfg.d
     passes = ({"q_cluster_ms": 1 + (cfg.iters_warm + 1) + cfg.iters_warm,   # norms, assignment passes, updates
                "k_cluster_ms": 1 + (cfg.iters_warm + 1) + cfg.iters_warm,
                "stats_sort_ms": 1} if warm else
@@ -431,7 +452,7 @@ def main():
              "reduction_stages_hbm": red,
              "clustering_share": round(clustering_ms / steady["total_ms"], 4),
              "assign_counters_since_create": lay.assign_counters(),
-             "kept_pair_frac": cnt["kept_pairs"] / float(cfg.B * cfg.H * cfg.L * cfg.L),
+             "kept_pair_frac": cnt["kept_pairs"] / float(lcfg.B * lcfg.H * lcfg.L * lcfg.L),
              "tile_efficiency": cnt["kept_pairs"] / max(1, cnt["computed_pairs"])}
     try:
         from cluster_routed_sparse_b200 import _lib as L
@@ -464,7 +485,8 @@ def main():
     # e2e through the asynchronous host-buffer entry point
     e2e = None
     if not args.no_e2e:
-        e2e = time_e2e(lay, steps_in, cfg, args, world, dist if world > 1 else None)
+        e2e = time_e2e(lay, steps_in, lcfg, args, 1 if split else world, dist if world > 1 else None,
+                       job_flops=cfg.steps * dense_flops(cfg) if split else None)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -476,7 +498,8 @@ def main():
 
     if rank == 0:
         out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-               "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+               "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+               "scaling": "strong" if split else "weak",
                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(cfg, args),
                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
                "clocks": clk, "layer_ms_step0": split0["total_ms"],
@@ -516,7 +539,7 @@ def time_sdpa(Q, K, V, reps: int = 3):
     return {"backend": None, "ms": None, "error": last}
 
 
-def time_e2e(lay, steps_in, cfg, args, world, dist):
+def time_e2e(lay, steps_in, cfg, args, world, dist, job_flops=None):
     """The bench steps through the asynchronous host-buffer entry point
     (ac_layer_forward_host_async): every call copies that step's Q, K, V from
     pinned host memory and O back; a call's copies overlap its neighbours'
@@ -550,7 +573,8 @@ def time_e2e(lay, steps_in, cfg, args, world, dist):
         reps.append(ms)
     ms = float(np.median(reps))
     nbytes = cfg.B * cfg.H * cfg.L * cfg.d * 2
-    return {"value": world * n_calls * dense_flops(cfg) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    flops = job_flops if job_flops is not None else world * n_calls * dense_flops(cfg)
+    return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": 3 * nbytes * n_calls, "d2h_bytes_per_step": nbytes * n_calls,
             "ms_per_step": ms, "ms_per_step_reps": [round(x, 2) for x in reps],
             "api": f"ac_layer_forward_host_async x {n_calls} per step, ac_join",

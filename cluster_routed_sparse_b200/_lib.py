@@ -22,7 +22,7 @@ AC_TAU_ABSOLUTE, AC_TAU_MEAN_FACTOR, AC_TAU_PERCENTILE = 0, 1, 2
 (AC_T_INV_NORM_Q, AC_T_LABELS_Q, AC_T_CENT_Q, AC_T_COUNTS_Q, AC_T_PERM_Q, AC_T_OFFS_Q, AC_T_LABELS_K,
  AC_T_DMIN_K, AC_T_CENT_K, AC_T_N_K, AC_T_DENSE, AC_T_COUNTS_K, AC_T_KMAX, AC_T_KMIN, AC_T_SSE, AC_T_COMP,
  AC_T_PERM_K, AC_T_OFFS_K, AC_T_SCORE, AC_T_SEL, AC_T_KSEL, AC_T_TAU, AC_T_STAGES, AC_T_REMOVED_STAGE,
- AC_T_MSE) = range(25)
+ AC_T_MSE, AC_T_FALLBACK_AT) = range(26)
 
 # element type of each tensor id, as a __cuda_array_interface__ typestr
 TENSOR_TYPES = {
@@ -31,7 +31,7 @@ TENSOR_TYPES = {
     AC_T_CENT_K: "<f4", AC_T_N_K: "<i4", AC_T_DENSE: "|u1", AC_T_COUNTS_K: "<i4", AC_T_KMAX: "<i2",
     AC_T_KMIN: "<i2", AC_T_SSE: "<f4", AC_T_COMP: "<f4", AC_T_PERM_K: "<i4", AC_T_OFFS_K: "<i4",
     AC_T_SCORE: "<f4", AC_T_SEL: "<i4", AC_T_KSEL: "<i4", AC_T_TAU: "<f4", AC_T_STAGES: "<i4",
-    AC_T_REMOVED_STAGE: "<i4", AC_T_MSE: "<f4",
+    AC_T_REMOVED_STAGE: "<i4", AC_T_MSE: "<f4", AC_T_FALLBACK_AT: "<i4",
 }
 
 
@@ -41,7 +41,7 @@ TENSOR_RANKS = {
     AC_T_OFFS_Q: 2, AC_T_LABELS_K: 2, AC_T_DMIN_K: 2, AC_T_CENT_K: 3, AC_T_N_K: 1, AC_T_DENSE: 1,
     AC_T_COUNTS_K: 2, AC_T_KMAX: 3, AC_T_KMIN: 3, AC_T_SSE: 2, AC_T_COMP: 1, AC_T_PERM_K: 2,
     AC_T_OFFS_K: 2, AC_T_SCORE: 3, AC_T_SEL: 3, AC_T_KSEL: 1, AC_T_TAU: 1, AC_T_STAGES: 1,
-    AC_T_REMOVED_STAGE: 2, AC_T_MSE: 1,
+    AC_T_REMOVED_STAGE: 2, AC_T_MSE: 1, AC_T_FALLBACK_AT: 1,
 }
 
 
@@ -50,7 +50,8 @@ class ACConfig(ctypes.Structure):
                 ("tau_mode", ctypes.c_int32), ("tau_value", ctypes.c_float), ("topk", ctypes.c_int32),
                 ("iters_q", ctypes.c_int32), ("iters_k", ctypes.c_int32), ("iters_warm", ctypes.c_int32),
                 ("stage_rule", ctypes.c_int32), ("seed", ctypes.c_uint64), ("scale", ctypes.c_float),
-                ("score_mode", ctypes.c_int32), ("tail_merge", ctypes.c_int32), ("unit0", ctypes.c_int32)]
+                ("score_mode", ctypes.c_int32), ("tail_merge", ctypes.c_int32), ("unit0", ctypes.c_int32),
+                ("compensate", ctypes.c_int32)]
 
 
 class ACStageTimes(ctypes.Structure):
@@ -100,6 +101,7 @@ SIGNATURES = {
     "ac_cluster_q_noalloc": (_I, [_P, _I, _I, _I, _I, _I, ctypes.c_uint64, _P, _P, _P, _P, _P]),
     "ac_state_export": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int64)]),
     "ac_set_tau_exchange": (_I, [_P, SUM_U64_FN, _P]),
+    "ac_calibrate_n_max": (_I, [ctypes.POINTER(_I), ctypes.c_int64, ctypes.c_float, ctypes.POINTER(_I)]),
     "ac_tau_mean_from_sums": (_I, [ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64, ctypes.POINTER(ctypes.c_float)]),
     "ac_tau_radix_pick": (_I, [ctypes.POINTER(ctypes.c_uint64), _I, ctypes.POINTER(ctypes.c_uint32)]),
     "ac_state_import": (_I, [_P, _P, ctypes.c_int64]),

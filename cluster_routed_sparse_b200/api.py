@@ -65,6 +65,17 @@ def tau_exchange_allreduce(group=None, device=None):
     return fn
 
 
+def calibrate_n_max(fallback_at, dense_frac: float = 0.15) -> int:
+    """ac_calibrate_n_max: the N_max under which the ceil(dense_frac * n) units
+    (of a stack of layers) with the largest AC_T_FALLBACK_AT fall back to dense
+    attention (AdaCluster Sec. 4.1: the top 15% of layers run full attention)."""
+    vals = [int(x) for x in fallback_at]
+    arr = (ctypes.c_int32 * len(vals))(*vals)
+    out = ctypes.c_int32(0)
+    check(_lib.load().ac_calibrate_n_max(arr, len(vals), float(dense_frac), ctypes.byref(out)))
+    return int(out.value)
+
+
 def tau_mean_from_sums(factor: float, fixed_sum: int, n: int) -> float:
     """ac_tau_mean_from_sums: tau = factor x the mean of the pooled distances,
     from the sum of floor(d_i 2^24) and their number."""
@@ -91,12 +102,13 @@ class SparseLayer:
     def __init__(self, B: int, H: int, L: int, d: int, *, Cq: int, m0: int, n_max: int,
                  tau_mode: int, tau_value: float, topk: int, iters_q: int = 10,
                  iters_k: int = 10, iters_warm: int = 2, seed: int = 1234, scale: float = 0.0,
-                 stage_rule: int = 0, score_mode: int = 0, tail_merge: int = 0, unit0: int = 0):
+                 stage_rule: int = 0, score_mode: int = 0, tail_merge: int = 0, unit0: int = 0,
+                 compensate: int = 0):
         self.lib = _lib.load()
         self.B, self.H, self.L, self.d = B, H, L, d
         self.cfg = ACConfig(Cq, m0, n_max, tau_mode, float(tau_value), topk, iters_q, iters_k,
                             iters_warm, stage_rule, seed & (2**64 - 1), float(scale), score_mode,
-                            tail_merge, unit0)
+                            tail_merge, unit0, compensate)
         self.Cq, self.Ccap = Cq, n_max + m0
         h = ctypes.c_void_p()
         check(self.lib.ac_create(ctypes.byref(self.cfg), B, H, L, d, ctypes.byref(h)))

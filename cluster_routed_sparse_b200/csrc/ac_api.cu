@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <functional>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -362,7 +363,7 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
     CK(launch_iota_rows(c->u_idx, c->u_cnt, BH, L, s), "iota");
     CK(cudaMemsetAsync(c->removed_stage, 0xFF, sizeof(int) * BH * (size_t)L, s), "removed init");
     CK(cudaMemsetAsync(c->tau_acc, 0, sizeof(unsigned long long), s), "tau acc");
-    std::vector<int> done(BH, 0), stages(BH, 0), nk(BH, 0), m(BH, 0), ucnt(BH, L);
+    std::vector<int> done(BH, 0), stages(BH, 0), nk(BH, 0), m(BH, 0), ucnt(BH, L), m_last(BH, 0);
     std::vector<uint8_t> dense(BH, 0);
     for (int t = 0;; ++t) {
         if (t > 0) {
@@ -390,6 +391,7 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
                 continue;
             }
             m[h] = stage_clusters(m0, ucnt[h], L, t, c->cfg.stage_rule);  // line 11
+            m_last[h] = m[h];
             max_m = std::max(max_m, m[h]);
             any = true;
         }
@@ -460,10 +462,12 @@ ac_status cluster_k_step0(ac_ctx *c, const bf16 *K, cudaStream_t s) {
         c->h_n_k[h] = nk[h];
         c->h_dense[h] = dense[h];
         c->h_st_m[h] = stages[h];
+        c->h_u_cnt[h] = dense[h] ? nk[h] : (stages[h] > 1 ? nk[h] - m_last[h] : 0);
     }
     CK(cudaMemcpyAsync(c->n_k, c->h_n_k, sizeof(int) * BH, cudaMemcpyHostToDevice, s), "n_k");
     CK(cudaMemcpyAsync(c->dense, c->h_dense, BH, cudaMemcpyHostToDevice, s), "dense");
     CK(cudaMemcpyAsync(c->stages, c->h_st_m, sizeof(int) * BH, cudaMemcpyHostToDevice, s), "stages");
+    CK(cudaMemcpyAsync(c->fallback_at, c->h_u_cnt, sizeof(int) * BH, cudaMemcpyHostToDevice, s), "fallback");
     CK(cudaStreamSynchronize(s), "stage end sync");  // the staging buffers are reused by the next call
     // line 22: every key to its closest centre among all of C
     Lloyd fin;
@@ -526,6 +530,12 @@ ac_status score_select_impl(ac_ctx *c, int topk, cudaStream_t s) {
     a.err = c->err;
     a.exact_cuda_cores = c->exact_scores;
     a.bound_scale = c->quest_bound_scale;
+    if (c->cfg.compensate) {
+        a.cbias = c->cbias;
+        a.crange = c->crange;
+        a.cgroup = c->cgroup;
+        a.scale = c->scale;
+    }
     CK(launch_score_select(a, s), "score select");
     if (c->cfg.tail_merge) {
         TailMergeArgs t{c->sel, c->ksel, c->dense, c->labels_q, c->perm_q, c->offs_q, c->counts_q, c->counts_k,
@@ -545,10 +555,28 @@ ac_status sparse_attn_impl(ac_ctx *c, const bf16 *Q, const bf16 *K, const bf16 *
     CK(launch_permute_kv_padded(K, V, c->perm_k, c->labels_k, c->offs_k, c->Ccap + 1, c->pgoff, c->Ccap, c->Kp, c->Vp,
                                 c->L, c->Lpad, c->d, c->BH, s),
        "permute k, v");
+    if (c->cfg.compensate) {
+        // member means of the final key clusters (ascending member order, as the
+        // centre update), as bf16 rows of the centroid block
+        UpdateArgs uk{K, nullptr, c->L, nullptr, c->perm_k, c->offs_k, c->Ccap + 1, c->kbar, (int64_t)c->Ccap * c->d,
+                      nullptr, c->n_k, 0, c->BH, c->d, c->Ccap};
+        uk.err = c->err;
+        UpdateArgs uv = uk;
+        uv.X = V;
+        uv.C = c->vbar;
+        CK(launch_update(uk, s), "key means");
+        CK(launch_update(uv, s), "value means");
+        CK(launch_comp_rows(c->kbar, c->vbar, c->n_k, c->Ccap, c->d, c->BH, c->Lpad, c->cgroup, c->Kp, c->Vp, s),
+           "centroid rows");
+    }
     CK(cudaMemsetAsync(c->counters, 0, 8 * sizeof(unsigned long long), s), "counters");
     AttnArgs a{&c->tm_q, c->tm_kg, c->tm_vg, O, pq, oq, cq, c->tile_prefix, c->ranges,
                c->nboxes, c->nrange, c->rbox, c->L, c->Lpad, c->Cq, c->Ccap, c->BH, c->d,
                (float)(c->scale * 1.4426950408889634), c->err, c->counters};
+    if (c->cfg.compensate) {
+        a.crange = c->crange;
+        a.cbias = c->cbias;
+    }
     if (c->timing) CK(cudaEventRecord(c->ev[6], s), "event");
     CK(launch_sparse_attn(a, s), "sparse attention");
     if (c->timing) CK(cudaEventRecord(c->ev[7], s), "event");
@@ -557,14 +585,14 @@ ac_status sparse_attn_impl(ac_ctx *c, const bf16 *Q, const bf16 *K, const bf16 *
 
 void free_all(ac_ctx *c) {
     void *dev[] = {c->inv_q, c->labels_q, c->cent_q, c->counts_q, c->perm_q, c->offs_q, c->labels_k, c->dmin_k,
-                   c->cent_k, c->n_k, c->dense, c->stages, c->removed_stage, c->tau, c->tau_acc, c->counts_k,
+                   c->cent_k, c->n_k, c->dense, c->stages, c->fallback_at, c->removed_stage, c->tau, c->tau_acc, c->counts_k,
                    c->perm_k, c->offs_k, c->kmax, c->kmin, c->sse, c->mse, c->comp, c->u_idx, c->u_idx2,
                    c->u_cnt, c->st_m, c->st_labels, c->st_dist, c->st_perm, c->st_offs, c->st_counts, c->radix,
                    c->score, c->sel, c->ksel, c->ranges, c->nboxes, c->tile_prefix, c->Qp, c->Kp, c->Vp,
                    c->counters, c->hbufQ, c->hbufK, c->hbufV, c->hbufO, c->err, c->chi_q, c->chi_k, c->cn,
                    c->hstat, c->rowsq_k, c->cand, c->amb_list, c->amb_count, c->asg_stats, c->rbox, c->pgoff, c->nrange,
                    c->sort_scratch, c->cnp_k, c->rowsq_u, c->cent_st, c->perm_qm, c->offs_qm, c->counts_qm,
-                   c->tm_scratch, c->kabs};
+                   c->tm_scratch, c->kabs, c->kbar, c->vbar, c->cbias, c->crange};
     for (void *p : dev)
         if (p) cudaFree(p);
     void *host[] = {c->h_u_cnt, c->h_st_m, c->h_n_k, c->h_dense, c->h_err, c->h_xchg};
@@ -603,7 +631,8 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     if (cfg->Cq < 1 || cfg->Cq > L || cfg->m0 < 1 || cfg->m0 > L || cfg->n_max < 1 || cfg->iters_q < 0 ||
         cfg->iters_k < 0 || cfg->iters_warm < 0 || cfg->tau_mode < 0 || cfg->tau_mode > 2 || cfg->topk == 0 ||
         cfg->stage_rule < 0 || cfg->stage_rule > 1 || (cfg->score_mode != 0 && cfg->score_mode != 1) ||
-        cfg->tail_merge < 0 || cfg->tail_merge > 2 || cfg->unit0 < 0 || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
+        cfg->tail_merge < 0 || cfg->tail_merge > 2 || cfg->unit0 < 0 || cfg->compensate < 0 || cfg->compensate > 1 ||
+        (cfg->compensate && cfg->tail_merge) || !(cfg->scale >= 0.f) || std::isnan(cfg->tau_value))
         return AC_ERR_INVALID_ARG;
     if ((int64_t)B * H * L >= (int64_t)1 << 31) return AC_ERR_INVALID_ARG;
     if (cfg->tau_mode == AC_TAU_PERCENTILE && (cfg->tau_value < 1.f || cfg->tau_value > 1000.f))
@@ -627,7 +656,10 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     c->BH = B * H;
     c->Cq = cfg->Cq;
     c->Ccap = cfg->n_max + cfg->m0;
-    c->Lpad = ((L + 7) & ~7) + 8 * c->Ccap + 8;  // keys padded per cluster; the last group stays zero
+    // keys padded per cluster (at most 7 rows each), then the centroid block of
+    // ceil(Ccap / 8) groups, then one group that stays zero
+    c->Lpad = ((L + 7) & ~7) + 8 * c->Ccap + 16;
+    c->cgroup = c->Lpad / 8 - 1 - (c->Ccap + 7) / 8;
     if ((int64_t)c->B * c->H * c->Lpad >= (int64_t)1 << 31) {
         delete c;
         return AC_ERR_INVALID_ARG;
@@ -663,6 +695,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->n_k, BH));
     A(dalloc(&c->dense, BH));
     A(dalloc(&c->stages, BH));
+    A(dalloc(&c->fallback_at, BH));
     A(dalloc(&c->removed_stage, BH * Lz));
     A(dalloc(&c->tau, 1));
     A(dalloc(&c->tau_acc, 1));
@@ -700,6 +733,12 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->hstat, 2 * BH));
     A(dalloc(&c->rowsq_k, BH * Lz));
     A(dalloc(&c->rowsq_u, BH * Lz));
+    if (cfg->compensate) {
+        A(dalloc(&c->kbar, BH * Cc * dz));
+        A(dalloc(&c->vbar, BH * Cc * dz));
+        A(dalloc(&c->cbias, BH * Cq * Cc));
+        A(dalloc(&c->crange, BH * Cq));
+    }
     if (cfg->tail_merge) {
         A(dalloc(&c->perm_qm, BH * Lz));
         A(dalloc(&c->offs_qm, BH * (Cq + 1)));
@@ -736,7 +775,10 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
         cudaMemset(c->dense, 0, BH) != cudaSuccess || cudaMemset(c->n_k, 0, BH * sizeof(int)) != cudaSuccess ||
         // padding rows of Kp / Vp are read (and masked) by the attention: keep them finite
         cudaMemset(c->Kp, 0, BH * (size_t)c->Lpad * dz * sizeof(bf16)) != cudaSuccess ||
-        cudaMemset(c->Vp, 0, BH * (size_t)c->Lpad * dz * sizeof(bf16)) != cudaSuccess) {
+        cudaMemset(c->Vp, 0, BH * (size_t)c->Lpad * dz * sizeof(bf16)) != cudaSuccess ||
+        // an empty cluster's member mean is never written: keep it finite
+        (c->kbar && cudaMemset(c->kbar, 0, BH * Cc * dz * sizeof(float)) != cudaSuccess) ||
+        (c->vbar && cudaMemset(c->vbar, 0, BH * Cc * dz * sizeof(float)) != cudaSuccess)) {
         free_all(c);
         delete c;
         return AC_ERR_CUDA;
@@ -959,6 +1001,7 @@ ac_status ac_get_tensor(ac_ctx *c, int32_t which, void **ptr, int64_t shape[4]) 
         case AC_T_STAGES: p = c->stages; s0 = BH; break;
         case AC_T_REMOVED_STAGE: p = c->removed_stage; s0 = BH; s1 = L; break;
         case AC_T_MSE: p = c->mse; s0 = BH; break;
+        case AC_T_FALLBACK_AT: p = c->fallback_at; s0 = BH; break;
         default: return fail(c, AC_ERR_INVALID_ARG, "unknown tensor id");
     }
     *ptr = p;
@@ -972,6 +1015,27 @@ ac_status ac_get_tensor(ac_ctx *c, int32_t which, void **ptr, int64_t shape[4]) 
 ac_status ac_get_launch_count(int64_t *out) {
     if (!out) return AC_ERR_INVALID_ARG;
     *out = (int64_t)g_launches.load(std::memory_order_relaxed);
+    return AC_OK;
+}
+
+ac_status ac_calibrate_n_max(const int32_t *fallback_at, int64_t n, float dense_frac, int32_t *n_max) {
+    if (!fallback_at || !n_max || n < 1 || !(dense_frac >= 0.f && dense_frac <= 1.f)) return AC_ERR_INVALID_ARG;
+    std::vector<int32_t> v(fallback_at, fallback_at + n);
+    std::sort(v.begin(), v.end(), std::greater<int32_t>());
+    // ceil(dense_frac * n); 1e-4 forgives the rounding of dense_frac to fp32 (0.1f * 10 > 1)
+    const int64_t k = std::max<int64_t>(0, (int64_t)std::ceil((double)dense_frac * (double)n - 1e-4));
+    if (k == 0) {
+        *n_max = v[0] + 1;
+        return AC_OK;
+    }
+    if (v[0] <= 0) return AC_ERR_INVALID_ARG;  // no unit ran more than one stage: none can fall back
+    int32_t t = v[k - 1];
+    if (t <= 0) {  // fewer than k multi-stage units: all of them
+        t = v[0];
+        for (int64_t i = 0; i < n; ++i)
+            if (v[i] > 0) t = v[i];
+    }
+    *n_max = t;
     return AC_OK;
 }
 

@@ -34,6 +34,7 @@ struct ac_ctx {
     int *n_k;          // [BH]
     uint8_t *dense;    // [BH]
     int *stages;       // [BH]
+    int *fallback_at;  // [BH] cluster count at the head of the last stage (see AC_T_FALLBACK_AT)
     int *removed_stage;  // [BH, L]
     float *tau;        // [1]
     unsigned long long *tau_acc;  // [1] fixed-point sum of stage-0 distances
@@ -72,6 +73,14 @@ struct ac_ctx {
     int *offs_qm;      // [BH, Cq+1] first row of each group (owner cluster id)
     int *counts_qm;    // [BH, Cq]  rows of each group (0: merged into another)
     int *tm_scratch;   // [4, BH, Cq] owner, position in group, rows kept, base of handed rows
+    // centroid compensation (cfg.compensate): member means of every key cluster,
+    // written as bf16 rows of a centroid block of Kp / Vp (group cgroup of each
+    // unit), one key range over that block per query cluster (crange), and the
+    // block's per-column addends ln|c| / scale, -inf for the selected clusters
+    float *kbar, *vbar;  // [BH, Ccap, d]
+    float *cbias;        // [BH, Cq, Ccap]
+    int *crange;         // [BH*Cq]  index of the centroid range, -1: none
+    int cgroup;          // first 8-row group of the centroid block within a unit of Kp / Vp
 
     // ---- tensor-core assignment (centres split into bf16 + remainder)
     int Cpad_q, CH_q, Cpad_k, CH_k;  // padded centre rows per unit, centres per chunk
@@ -286,6 +295,8 @@ struct SelectArgs {
     float *kabs = nullptr;         // [BH, Ccap]
     uint32_t *err = nullptr;
     bool exact_cuda_cores = false;  // force the CUDA-core kernels (k_quest_scores + k_score_select)
+    // centroid compensation: per-column addends and the extra key range (null: off)
+    float *cbias = nullptr; int *crange = nullptr; int cgroup = 0; float scale = 1.f;
     float bound_scale = 1.f;        // widens the tensor-core path's error bound (tests of the rescoring)
 };
 cudaError_t launch_score_select(const SelectArgs &a, cudaStream_t s);
@@ -313,8 +324,12 @@ struct AttnArgs {
     int L, Lpad, Cq, Ccap, BH, d;
     float scale_log2;
     uint32_t *err; unsigned long long *counters;
+    const int *crange = nullptr; const float *cbias = nullptr;  // centroid compensation (null: off)
 };
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s);
+// bf16 rows of the centroid block: Kp / Vp row 8 cgroup + c of unit h = kbar / vbar [h, c], c < n_k[h]
+cudaError_t launch_comp_rows(const float *kbar, const float *vbar, const int *n_k, int Ccap, int d, int BH,
+                             int64_t Lpad, int cgroup, bf16 *Kp, bf16 *Vp, cudaStream_t s);
 int attn_max_tiles(int L, int Cq, int BH);
 
 }  // namespace ac

@@ -60,7 +60,9 @@ struct Layout {
     static constexpr uint32_t OFF_MASK = OFF_V + NS * KV_BYTES;  // [4][4] uint32 (tile j in slot j % 4)
     static constexpr uint32_t OFF_RG = OFF_MASK + 64;            // [RG_CACHE] int2 key ranges
     static constexpr uint32_t OFF_RB = OFF_RG + RG_CACHE * 8;    // [RG_CACHE + 1] first box of each range
-    static constexpr uint32_t OFF_BAR = OFF_RB + (RG_CACHE + 1) * 4 + 12;
+    static constexpr uint32_t OFF_CB = OFF_RB + (RG_CACHE + 1) * 4 + 12;  // [4][128] column addends (compensation)
+    static constexpr uint32_t OFF_CT = OFF_CB + 4 * BN * 4;      // [4] tile holds centroid columns
+    static constexpr uint32_t OFF_BAR = OFF_CT + 16;
     static constexpr uint32_t BYTES = OFF_BAR + 256;
     static constexpr uint32_t SMEM = BYTES + 1024;  // 1024-byte alignment slack
 };
@@ -112,6 +114,10 @@ struct AttnParams {
     bf16 *O;
     const int *perm_q, *offs_q, *counts_q, *tile_prefix, *nboxes, *nrange, *rbox;
     const int2 *ranges;  // (first 8-row group in Kp / Vp, keys)
+    // centroid compensation: index of the range over the centroid rows (-1: none)
+    // and, per centroid column, ln|c| / scale, or -inf for a selected or empty cluster
+    const int *crange;
+    const float *cbias;
     int L, Lpad, Cq, Ccap, BH;
     float scale_log2;
     uint32_t *err;
@@ -128,7 +134,7 @@ __device__ __forceinline__ void record_wait_failure(const AttnParams &p, int rol
     }
 }
 
-template <int D>
+template <int D, bool COMP>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_sparse_attn(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     using LY = Layout<D>;
@@ -170,6 +176,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
      (record_wait_failure(p, (role), (bidx), (jj), (par)), false))
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + LY::OFF_BAR + 8 * NBAR);
     uint32_t *masks = reinterpret_cast<uint32_t *>(sm + LY::OFF_MASK);
+    float *cbias_s = reinterpret_cast<float *>(sm + LY::OFF_CB);
+    uint32_t *ctile = reinterpret_cast<uint32_t *>(sm + LY::OFF_CT);
+    const int cr = COMP ? p.crange[hq] : -1;
 
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) {
@@ -262,6 +271,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 break;
             }
             if (lane < 4) masks[4 * (j & 3) + lane] = lane == 0 ? w[0] : lane == 1 ? w[1] : lane == 2 ? w[2] : w[3];
+            if (COMP) {
+                // centroid columns of this tile: the addend ln|c| / scale (-inf
+                // for the selected and the empty clusters), 0 elsewhere
+                const bool cpart = mine && r == cr;
+                const bool anyc = __any_sync(0xFFFFFFFFu, cpart);
+                if (anyc) {
+                    float *cb = cbias_s + (j & 3) * BN;
+                    for (int i = lane; i < BN; i += 32) cb[i] = 0.f;
+                    __syncwarp();
+                    if (cpart) {
+                        const float *src = p.cbias + (int64_t)hq * p.Ccap;
+                        for (int sl = a0; sl < a1; ++sl)
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int ci = 8 * (sl - rb0) + i;
+                                cb[(sl - t0) * 8 + i] = ci < g.y ? src[ci] : 0.f;
+                            }
+                    }
+                }
+                if (lane == 0) ctile[j & 3] = anyc ? 1u : 0u;
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive_expect_tx(BAR(B_KF + s), LY::KV_BYTES);  // releases the masks
             __syncwarp();
@@ -425,6 +455,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         for (int i = 0; i < 32; ++i) r[c][i] = ((vm[c] >> i) & 1u) ? r[c][i] : 0xFF800000u;
                     }
                 }
+                if (COMP && ctile[j & 3]) {
+                    // a centroid column c stands for |c| keys at its member mean:
+                    // its score gains ln|c| / scale (the softmax weight |c| exp(q.k / sqrt d))
+                    const float4 *cb = reinterpret_cast<const float4 *>(cbias_s + (j & 3) * BN);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4) {
+                            const float4 b = cb[c * 8 + i / 4];
+                            r[c][i] = __float_as_uint(__uint_as_float(r[c][i]) + b.x);
+                            r[c][i + 1] = __float_as_uint(__uint_as_float(r[c][i + 1]) + b.y);
+                            r[c][i + 2] = __float_as_uint(__uint_as_float(r[c][i + 2]) + b.z);
+                            r[c][i + 3] = __float_as_uint(__uint_as_float(r[c][i + 3]) + b.w);
+                        }
+                }
                 // Row maximum: 8 independent partial maxima, three-input max.
                 float pm[8];
 #pragma unroll
@@ -575,21 +620,23 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s) {
     p.scale_log2 = a.scale_log2;
     p.err = a.err;
     p.counters = a.counters;
+    p.crange = a.crange;
+    p.cbias = a.cbias;
     const int grid = attn_max_tiles(a.L, a.Cq, a.BH);
+    const bool comp = a.crange != nullptr;
     cudaError_t e;
-    if (a.d == 128) {
-        e = cudaFuncSetAttribute(k_sparse_attn<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Layout<128>::SMEM);
-        if (e != cudaSuccess) return e;
-        k_sparse_attn<128><<<grid, NTHREADS, Layout<128>::SMEM, s>>>(maps, p);
+    auto go = [&](auto kern, uint32_t smem) -> cudaError_t {
+        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        kern<<<grid, NTHREADS, smem, s>>>(maps, p);
         AC_NOTE_LAUNCH();
-    } else {
-        e = cudaFuncSetAttribute(k_sparse_attn<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Layout<64>::SMEM);
-        if (e != cudaSuccess) return e;
-        k_sparse_attn<64><<<grid, NTHREADS, Layout<64>::SMEM, s>>>(maps, p);
-        AC_NOTE_LAUNCH();
-    }
+        return cudaSuccess;
+    };
+    if (a.d == 128)
+        e = comp ? go(k_sparse_attn<128, true>, Layout<128>::SMEM) : go(k_sparse_attn<128, false>, Layout<128>::SMEM);
+    else
+        e = comp ? go(k_sparse_attn<64, true>, Layout<64>::SMEM) : go(k_sparse_attn<64, false>, Layout<64>::SMEM);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -871,6 +871,30 @@ cudaError_t launch_update(const UpdateArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ compensation
+// Centroid block of Kp / Vp (ClusterAttention Sec. 1.2): row 8 cgroup + c of unit
+// h holds the member means of key cluster c, rounded to bf16; d / 8 threads per
+// row and tensor, one block per (cluster, unit).
+__global__ void k_comp_rows(const float *__restrict__ kbar, const float *__restrict__ vbar,
+                            const int *__restrict__ n_k, int Ccap, int d, int64_t Lpad, int cgroup,
+                            bf16 *__restrict__ Kp, bf16 *__restrict__ Vp) {
+    const int c = blockIdx.x, h = blockIdx.y;
+    if (c >= n_k[h]) return;
+    const int per = d / 8, which = threadIdx.x / per, part = threadIdx.x % per;
+    const float4 *src = reinterpret_cast<const float4 *>((which ? vbar : kbar) + ((int64_t)h * Ccap + c) * d) + 2 * part;
+    const float4 x0 = src[0], x1 = src[1];
+    bf16 *dst = (which ? Vp : Kp) + ((int64_t)h * Lpad + (int64_t)cgroup * 8 + c) * d;
+    reinterpret_cast<uint4 *>(dst)[part] = make_uint4(pack_bf16x2(x0.x, x0.y), pack_bf16x2(x0.z, x0.w),
+                                                      pack_bf16x2(x1.x, x1.y), pack_bf16x2(x1.z, x1.w));
+}
+
+cudaError_t launch_comp_rows(const float *kbar, const float *vbar, const int *n_k, int Ccap, int d, int BH,
+                             int64_t Lpad, int cgroup, bf16 *Kp, bf16 *Vp, cudaStream_t s) {
+    k_comp_rows<<<dim3(Ccap, BH), 2 * (d / 8), 0, s>>>(kbar, vbar, n_k, Ccap, d, Lpad, cgroup, Kp, Vp);
+    AC_NOTE_LAUNCH();
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ seeding
 __global__ void k_seed(SeedArgs a) {
     const int h = blockIdx.y;

@@ -83,6 +83,10 @@ struct QuestParams {
     int *sel, *ksel, *nrange, *nboxes, *rbox;
     int2 *ranges;
     uint32_t *err;
+    float *cbias;       // centroid compensation (null: off): [BH, Cq, Ccap] addends, crange [BH*Cq]
+    int *crange;
+    int cgroup;
+    float scale;
     float bound_scale;  // >= 1: widens E (more candidates rescored; the selection is unchanged)
     int Cq, Ccap, BH, topk, warps2;
 };
@@ -508,7 +512,26 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
             rpos += __popc(bw);
             gpos += __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
+        // centroid compensation: the unselected non-empty clusters as pseudo-keys
+        // (one more range, over the centroid block), with their addends ln|c| / scale
+        if (p.cbias) {
+            float *cb = p.cbias + hq * p.Ccap;
+            for (int c = lane; c < nk; c += 32) {
+                const bool sl = (sbits[c >> 5] >> (c & 31)) & 1u;
+                const bool nz = (ne_s[c >> 5] >> (c & 31)) & 1u;
+                cb[c] = (sl || !nz) ? -INFINITY : logf((float)cnt[c]) / p.scale;
+            }
+        }
         if (lane == 0) {
+            if (p.cbias && !dense && ne > k) {
+                rg[rpos] = make_int2(p.cgroup, nk);
+                rb[rpos] = gpos;
+                p.crange[hq] = rpos;
+                ++rpos;
+                gpos += (nk + 7) / 8;
+            } else if (p.crange) {
+                p.crange[hq] = -1;
+            }
             p.nrange[hq] = rpos;
             p.nboxes[hq] = gpos;
             rb[rpos] = gpos;
@@ -551,6 +574,10 @@ cudaError_t launch_quest_d(const SelectArgs &a, cudaStream_t s) {
     p.ranges = a.ranges;
     p.err = a.err;
     p.bound_scale = a.bound_scale >= 1.f ? a.bound_scale : 1.f;
+    p.cbias = a.cbias;
+    p.crange = a.crange;
+    p.cgroup = a.cgroup;
+    p.scale = a.scale;
     p.Cq = a.Cq;
     p.Ccap = a.Ccap;
     p.BH = a.BH;

@@ -218,10 +218,28 @@ __global__ void __launch_bounds__(SEL_THREADS) k_score_select(SelectArgs a) {
         gpos += (cnt[c] + 7) / 8;
         ++rpos;
     }
+    // centroid compensation: the unselected non-empty clusters as pseudo-keys
+    // (one more range, over the centroid block), with their addends ln|c| / scale
+    const bool comp = a.cbias != nullptr && !dense && nonempty > k;
+    if (a.cbias) {
+        float *cb = a.cbias + (int64_t)hq * a.Ccap;
+        for (int c = tid; c < nk; c += SEL_THREADS)
+            cb[c] = (flag[c] || cnt[c] == 0) ? -INFINITY : logf((float)cnt[c]) / a.scale;
+    }
     if (tid == 0) {
-        a.nrange[hq] = nr;
-        a.nboxes[hq] = ng;
-        rbox[nr] = ng;
+        int n_r = nr, n_g = ng;
+        if (comp) {
+            a.ranges[(int64_t)hq * a.Ccap + n_r] = make_int2(a.cgroup, nk);
+            rbox[n_r] = n_g;
+            a.crange[hq] = n_r;
+            ++n_r;
+            n_g += (nk + 7) / 8;
+        } else if (a.crange) {
+            a.crange[hq] = -1;
+        }
+        a.nrange[hq] = n_r;
+        a.nboxes[hq] = n_g;
+        rbox[n_r] = n_g;
     }
 }
 

@@ -102,6 +102,10 @@ typedef struct ac_config {
                             over contexts (ac_set_tau_exchange) clusters each
                             head as a single context over all heads would; 0
                             for a whole layer                                */
+    int32_t compensate;  /* 1: every unselected non-empty key cluster also enters
+                            each query's softmax as one pseudo-key, its member
+                            mean, weighted by its size (ClusterAttention Sec. 1.2,
+                            Eq. (5)-(6)); 0: off.  Not with tail_merge.        */
 } ac_config;
 
 typedef struct ac_ctx ac_ctx;
@@ -258,7 +262,12 @@ typedef enum ac_tensor_id {
     AC_T_STAGES = 22,      /* int32 [BH]   stages run by Algorithm 1            */
     AC_T_REMOVED_STAGE = 23, /* int32 [BH, L] stage that absorbed the key, -1 */
     AC_T_MSE = 24,         /* fp32  [BH]                                        */
-    AC_T_NUM = 25
+    AC_T_FALLBACK_AT = 25, /* int32 [BH]   after step 0: the largest n_max under
+                              which the unit would have fallen back to dense
+                              attention (the cluster count at the head of its
+                              last stage; 0 when stage 0 absorbed every key; for
+                              a unit that fell back, its count then)         */
+    AC_T_NUM = 26
 } ac_tensor_id;
 
 AC_API ac_status ac_get_tensor(ac_ctx *ctx, int32_t which, void **dev_ptr, int64_t shape[4]);
@@ -366,6 +375,18 @@ AC_API ac_status ac_set_tau_exchange(ac_ctx *ctx, ac_sum_u64_fn fn, void *user);
  * rank + 1). */
 AC_API ac_status ac_tau_mean_from_sums(float factor, uint64_t fixed_sum, uint64_t n, float *tau);
 AC_API ac_status ac_tau_radix_pick(const uint64_t *hist, int32_t shift, uint32_t *state);
+
+/* Calibration of N_max over a stack of layers (AdaCluster Sec. 4.1: k_max is
+ * set so that the top 15% of layers, the least compact ones, run full
+ * attention).  Given each unit's AC_T_FALLBACK_AT from a step 0 run with an
+ * n_max large enough that no unit fell back, returns in *n_max the n_max
+ * under which the ceil(dense_frac * n) units with the largest values fall
+ * back: the k-th largest value (units tied with it fall back too).  When fewer
+ * than k units ran more than one stage, *n_max is the smallest positive value
+ * (only the multi-stage units can fall back), or n_max = 1 + max when
+ * dense_frac is 0.  Host only.  Errors: INVALID_ARG (n < 1, dense_frac outside
+ * [0, 1], or no unit ran more than one stage while dense_frac > 0). */
+AC_API ac_status ac_calibrate_n_max(const int32_t *fallback_at, int64_t n, float dense_frac, int32_t *n_max);
 
 /* Number of kernels libac has launched in this process so far (all contexts). */
 AC_API ac_status ac_get_launch_count(int64_t *out);

@@ -32,7 +32,7 @@ def make_layer_ctx(p: orc.Params, B, H, Lq, d) -> SparseLayer:
     return SparseLayer(B, H, Lq, d, Cq=p.Cq, m0=p.m0, n_max=p.n_max, tau_mode=p.tau_mode,
                        tau_value=p.tau_value, topk=p.topk, iters_q=p.iters_q, iters_k=p.iters_k,
                        iters_warm=p.iters_warm, seed=p.seed, stage_rule=p.stage_rule, score_mode=p.score_mode,
-                       tail_merge=p.tail_merge)
+                       tail_merge=p.tail_merge, unit0=p.unit0, compensate=p.compensate)
 
 
 def gpu_state(lay: SparseLayer) -> dict:

@@ -49,7 +49,7 @@ def _create(**kw):
     lib = _lib.load()
     base = dict(Cq=16, m0=32, n_max=128, tau_mode=1, tau_value=0.5, topk=8, iters_q=10, iters_k=10,
                 iters_warm=2, stage_rule=0, seed=1, scale=0.0, score_mode=0, tail_merge=0,
-                unit0=0)
+                unit0=0, compensate=0)
     dims = kw.pop("dims", (1, 2, 4096, 64))
     base.update(kw)
     cfg = _lib.ACConfig(**base)
@@ -70,6 +70,8 @@ def _create(**kw):
     (dict(score_mode=2), _lib.AC_ERR_INVALID_ARG),
     (dict(tail_merge=3), _lib.AC_ERR_INVALID_ARG),
     (dict(unit0=-1), _lib.AC_ERR_INVALID_ARG),
+    (dict(compensate=2), _lib.AC_ERR_INVALID_ARG),
+    (dict(compensate=1, tail_merge=1), _lib.AC_ERR_INVALID_ARG),
     (dict(dims=(1, 2, 0, 64)), _lib.AC_ERR_INVALID_ARG),
     (dict(dims=(1, 2, 4096, 96)), _lib.AC_ERR_UNSUPPORTED),
 ])
