@@ -382,6 +382,50 @@ __global__ void __launch_bounds__(A_THREADS, 1)
                     break;
                 }
                 tc_fence_after();
+                if (FOLD) {
+                    // keys: the whole chunk (up to four 32-column groups) at once;
+                    // its minimum sets the threshold before any column is marked,
+                    // so only columns near the best of the chunk reach the top-4
+                    uint32_t r[4][32];
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        if (g * 32 < N) tmem_ld32(tmem + lane_off + (a * 2 + ti) * ACH + g * 32, r[g]);
+                    tmem_ld_wait();
+                    float gm[4];
+                    float cm = INFINITY;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        float pmn[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+                        if (g * 32 < N) {
+#pragma unroll
+                            for (int q = 0; q < 16; ++q)
+                                pmn[q & 3] = fmin3(pmn[q & 3], __uint_as_float(r[g][2 * q]), __uint_as_float(r[g][2 * q + 1]));
+                        }
+                        gm[g] = fminf(fmin3(pmn[0], pmn[1], pmn[2]), pmn[3]);
+                        cm = fminf(cm, gm[g]);
+                    }
+                    const bool need = cm <= T;
+                    if (__any_sync(0xFFFFFFFFu, need)) {
+                        const float Tn = need ? assign_threshold(fminf(d1, cm), sq, delta, e) : T;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const bool ng = need && g * 32 < N && gm[g] <= Tn;
+                            if (__any_sync(0xFFFFFFFFu, ng)) {
+                                uint32_t msk = 0u;
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) msk |= __uint_as_float(r[g][i]) <= Tn ? (1u << i) : 0u;
+                                if (ng) {
+                                    const int c0 = ch * p.CH + g * 32;
+                                    for (uint32_t mm = msk; mm != 0u; mm &= mm - 1u) {
+                                        const int i = __ffs(mm) - 1;
+                                        top4_insert(pick32(r[g], i), c0 + i, d1, d2, d3, d4, i1, i2, i3, i4);
+                                    }
+                                }
+                            }
+                        }
+                        if (need) T = Tn;
+                    }
+                } else
                 for (int cg = 0; cg < N; cg += 32) {
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_off + (a * 2 + ti) * ACH + cg, r);
