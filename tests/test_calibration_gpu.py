@@ -23,11 +23,12 @@ from cluster_routed_sparse_b200.api import SparseLayer, calibrate_n_max
 
 pytestmark = pytest.mark.gpu
 
-BASE = synth.LayerConfig("stack-L4096-H2-d64", 1, 2, 4096, 64, Cq=16, m0=32, n_max=4000,
-                         tau_mode=synth.TAU_MEAN_FACTOR, tau_value=1.0, topk=8, iters_q=5, iters_k=5)
-STACK = [dataclasses.replace(BASE, name=f"stack-layer{i}", key_components=nc, seed=BASE.seed + 97 * i,
-                             diffuse_heads=dh)
-         for i, (nc, dh) in enumerate([(16, ()), (48, ()), (150, ()), (400, ()), (40, (1,)), (1200, ())])]
+BASE = synth.LayerConfig("stack-L4096-H2-d64", 1, 2, 4096, 64, Cq=16, m0=32, n_max=6000,
+                         tau_mode=synth.TAU_ABSOLUTE, tau_value=4.0, topk=8, iters_q=5, iters_k=5)
+# layers of decreasing compactness: more mixture components per head, one absolute tau
+# for the stack (App. A.5 uses absolute thresholds)
+STACK = [dataclasses.replace(BASE, name=f"stack-layer{i}", key_components=nc, seed=BASE.seed + 97 * i)
+         for i, nc in enumerate([16, 48, 100, 200, 300, 400])]
 
 
 def _ctx(cfg, n_max):
