@@ -283,7 +283,7 @@ def run_reference(args):
 # DRAM bytes (read + write) of one k_sparse_attn launch per head of the bench
 # workload, from an ncu capture of its 8-head reduction, valid only for the
 # kernel source it was taken on: any change to attn_kernel.cu turns it into null.
-ATTN_TRAFFIC = {"sha256_prefix": "f0e4b1ad3dc6ebe4", "bytes_per_head": (313.705472e6 + 132.507648e6) / 8}
+ATTN_TRAFFIC = {"sha256_prefix": "dbcf7fd631eae966", "bytes_per_head": (313612288 + 129535232) / 8}
 
 
 def attn_traffic_bytes(cfg):

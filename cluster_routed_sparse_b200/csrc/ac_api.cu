@@ -717,7 +717,7 @@ ac_status ac_create(const ac_config *cfg, int32_t B, int32_t H, int32_t L, int32
     A(dalloc(&c->st_offs, BH * (m0 + 1)));
     A(dalloc(&c->st_counts, BH * m0));
     A(dalloc(&c->radix, 260));
-    A(dalloc(&c->sort_scratch, BH * 128 * std::max(Cc, Cq)));
+    A(dalloc(&c->sort_scratch, BH * 129 * std::max(Cc, Cq)));  // chunk histograms + label totals
     A(dalloc(&c->score, BH * Cq * Cc));
     A(dalloc(&c->kabs, BH * Cc));
     A(dalloc(&c->sel, BH * Cq * Cc));

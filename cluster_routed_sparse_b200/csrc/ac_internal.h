@@ -56,7 +56,7 @@ struct ac_ctx {
     int *st_offs;      // [BH, m0+1]
     int *st_counts;    // [BH, m0]
     uint32_t *radix;   // [256 + 4] percentile selection scratch
-    int *sort_scratch; // [BH, 128, max(Ccap, Cq)] counting-sort chunk histograms
+    int *sort_scratch; // [BH, 129, max(Ccap, Cq)] counting-sort chunk histograms and label totals
 
     // ---- selection (Algorithm 3 line 9)
     float *score;      // [BH, Cq, Ccap]
@@ -219,7 +219,7 @@ struct SortArgs {
     int *counts;          // [BH, counts_stride] or null
     int counts_stride;
     int BH;
-    int *scratch;         // [BH, 128, max_lab] per-chunk histograms / slots
+    int *scratch;         // [BH, 128, max_lab] per-chunk histograms / slots, then [BH, max_lab] label totals
 };
 cudaError_t launch_counting_sort(const SortArgs &a, cudaStream_t s);
 

@@ -5,6 +5,7 @@
 // sequential operation order and round-to-nearest intrinsics (no fused
 // multiply-add), so labels, permutations and centres are reproducible
 // bit-for-bit run to run.  Member sums are taken in ascending token order.
+#include <cub/block/block_reduce.cuh>
 #include <cub/block/block_scan.cuh>
 
 #include "ac_device.cuh"
@@ -169,54 +170,88 @@ __global__ void __launch_bounds__(SORT_WARPS * 32) k_sort_hist(SortArgs a) {
     for (int l = lane; l < m; l += 32) H[l] = hist[w * m + l];
 }
 
-constexpr int SORT_OFF_THREADS = 1024;
-__global__ void __launch_bounds__(SORT_OFF_THREADS) k_sort_offsets(SortArgs a) {
-    extern __shared__ int tot[];  // [max_lab]
-    typedef cub::BlockScan<int, SORT_OFF_THREADS> Scan;
-    __shared__ typename Scan::TempStorage scan_tmp;
-    const int h = blockIdx.x, tid = threadIdx.x;
+// Pass (2) in two kernels over (unit, block of 32 labels), so that every SM
+// takes part: the lanes of a warp read 32 consecutive labels of one chunk row
+// (coalesced), the 8 warps of a block 16 chunks each.
+//  k_sort_totals:  tot[h, l] = sum over the chunks of the count of label l;
+//  k_sort_offsets: offs[h, l] = sum of tot[h, l'] for l' < l, counts[h, l] = tot,
+//                  and every (label, chunk) histogram entry replaced by the first
+//                  slot of that chunk's rows of the label.
+constexpr int SORT_LB = 32;                        // labels per block
+constexpr int SORT_CPW = SORT_CHUNKS / SORT_WARPS;  // chunks per warp
+
+__global__ void __launch_bounds__(SORT_WARPS * 32) k_sort_totals(SortArgs a, int *tot) {
+    __shared__ int part[SORT_WARPS][SORT_LB];
+    const int h = blockIdx.y, l = blockIdx.x * SORT_LB + (threadIdx.x & 31), w = threadIdx.x >> 5;
+    const int m = a.nlab ? a.nlab[h] : a.nlab_const;
+    if (m <= 0 || blockIdx.x * SORT_LB >= m) return;
+    const int *H = a.scratch + (int64_t)h * SORT_CHUNKS * a.max_lab;
+    int t = 0;
+    if (l < m) {
+#pragma unroll
+        for (int c = 0; c < SORT_CPW; ++c) t += H[(int64_t)(w * SORT_CPW + c) * a.max_lab + l];
+    }
+    part[w][threadIdx.x & 31] = t;
+    __syncthreads();
+    if (w == 0 && l < m) {
+        int s = 0;
+#pragma unroll
+        for (int i = 0; i < SORT_WARPS; ++i) s += part[i][threadIdx.x];
+        tot[(int64_t)h * a.max_lab + l] = s;
+    }
+}
+
+__global__ void __launch_bounds__(SORT_WARPS * 32) k_sort_offsets(SortArgs a, const int *tot) {
+    typedef cub::BlockReduce<int, SORT_WARPS * 32> Red;
+    __shared__ typename Red::TempStorage red_tmp;
+    __shared__ int base_s, lab_off[SORT_LB];
+    __shared__ int part[SORT_WARPS][SORT_LB];
+    const int h = blockIdx.y, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int l0 = blockIdx.x * SORT_LB, l = l0 + lane;
     const int n = a.nrows ? a.nrows[h] : a.nrows_const;
     const int m = a.nlab ? a.nlab[h] : a.nlab_const;
-    if (m <= 0) return;
-    int *H = a.scratch + (int64_t)h * SORT_CHUNKS * a.max_lab;
-    for (int l = tid; l < m; l += SORT_OFF_THREADS) {
-        int t = 0;
-#pragma unroll 8
-        for (int ci = 0; ci < SORT_CHUNKS; ++ci) t += H[(int64_t)ci * a.max_lab + l];
-        tot[l] = t;
-    }
+    if (m <= 0 || l0 >= m) return;
+    const int *T = tot + (int64_t)h * a.max_lab;
+    // rows of every label before this block's
+    int before = 0;
+    for (int i = threadIdx.x; i < l0; i += SORT_WARPS * 32) before += T[i];
+    before = Red(red_tmp).Sum(before);
+    if (threadIdx.x == 0) base_s = before;
     __syncthreads();
-    const int sg = (m + SORT_OFF_THREADS - 1) / SORT_OFF_THREADS;
-    const int l0 = min(m, tid * sg), l1 = min(m, l0 + sg);
-    int local = 0;
-    for (int l = l0; l < l1; ++l) local += tot[l];
-    int run;
-    Scan(scan_tmp).ExclusiveSum(local, run);
-    __syncthreads();
-    for (int l = l0; l < l1; ++l) {
-        const int t = tot[l];
-        tot[l] = run;  // now the label's first slot
-        run += t;
-    }
-    __syncthreads();
-    int *offs = a.offs + (int64_t)h * a.offs_stride;
-    for (int l = tid; l < m; l += SORT_OFF_THREADS) {
-        int slot = tot[l];
-        offs[l] = slot;
-        const int first = slot;
-        for (int c0 = 0; c0 < SORT_CHUNKS; c0 += 8) {
-            int cv[8];
+    if (w == 0) {
+        const int t = l < m ? T[l] : 0;
+        int incl = t;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) cv[u] = H[(int64_t)(c0 + u) * a.max_lab + l];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                H[(int64_t)(c0 + u) * a.max_lab + l] = slot;  // first slot of chunk c0 + u for label l
-                slot += cv[u];
-            }
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
         }
-        if (a.counts) a.counts[(int64_t)h * a.counts_stride + l] = slot - first;
+        lab_off[lane] = base_s + incl - t;
+        if (l < m) {
+            a.offs[(int64_t)h * a.offs_stride + l] = base_s + incl - t;
+            if (a.counts) a.counts[(int64_t)h * a.counts_stride + l] = t;
+        }
+        if (l0 + SORT_LB >= m && lane == 0) a.offs[(int64_t)h * a.offs_stride + m] = n;
     }
-    if (tid == 0) offs[m] = n;
+    // this warp's chunks of label l: their counts, the warp's share, then first slots
+    int *H = a.scratch + (int64_t)h * SORT_CHUNKS * a.max_lab;
+    int cv[SORT_CPW], mine = 0;
+#pragma unroll
+    for (int c = 0; c < SORT_CPW; ++c) {
+        cv[c] = l < m ? H[(int64_t)(w * SORT_CPW + c) * a.max_lab + l] : 0;
+        mine += cv[c];
+    }
+    part[w][lane] = mine;
+    __syncthreads();
+    int slot = lab_off[lane];
+    for (int i = 0; i < w; ++i) slot += part[i][lane];
+    if (l < m) {
+#pragma unroll
+        for (int c = 0; c < SORT_CPW; ++c) {
+            H[(int64_t)(w * SORT_CPW + c) * a.max_lab + l] = slot;  // first slot of this chunk's rows of label l
+            slot += cv[c];
+        }
+    }
 }
 
 __global__ void __launch_bounds__(SORT_WARPS * 32) k_sort_scatter(SortArgs a) {
@@ -340,9 +375,17 @@ cudaError_t launch_counting_sort(const SortArgs &a, cudaStream_t s) {
     k_sort_hist<<<grid, SORT_WARPS * 32, smem, s>>>(a);
     AC_NOTE_LAUNCH();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_sort_offsets<<<a.BH, SORT_OFF_THREADS, (size_t)a.max_lab * sizeof(int), s>>>(a);
-    AC_NOTE_LAUNCH();
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    {
+        // the per-label totals follow the chunk histograms of all units in the scratch
+        int *tot = a.scratch + (int64_t)a.BH * SORT_CHUNKS * a.max_lab;
+        const dim3 g((unsigned)((a.max_lab + SORT_LB - 1) / SORT_LB), (unsigned)a.BH);
+        k_sort_totals<<<g, SORT_WARPS * 32, 0, s>>>(a, tot);
+        AC_NOTE_LAUNCH();
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        k_sort_offsets<<<g, SORT_WARPS * 32, 0, s>>>(a, tot);
+        AC_NOTE_LAUNCH();
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     k_sort_scatter<<<grid, SORT_WARPS * 32, smem, s>>>(a);
     AC_NOTE_LAUNCH();
     return cudaGetLastError();
@@ -762,7 +805,7 @@ cudaError_t launch_member_stream_d(const MsArgs &a, int d, cudaStream_t s) {
 // Per key cluster: count and SSE = the members' exact distances (written in
 // member order by the statistics pass) summed in ascending member order; 0
 // for the slots c >= n_k.  One warp per cluster: 32 distances per load, the
-// next 32 in flight while every lane adds the current ones in order.
+// next 224 in flight while every lane adds the current ones in order.
 __global__ void k_cluster_sse(const int *__restrict__ offs, int offs_stride, const float *__restrict__ dsorted,
                               const int *__restrict__ n_k, int Ccap, int64_t L, int BH, int *__restrict__ counts,
                               float *__restrict__ sse) {
@@ -777,12 +820,22 @@ __global__ void k_cluster_sse(const int *__restrict__ offs, int offs_stride, con
         }
         const float *ds = dsorted + (int64_t)h * L;
         float se = 0.f;
-        float v = beg + lane < end ? ds[beg + lane] : 0.f;
-        for (int j = beg; j < end; j += 32) {
-            const float vn = j + 32 + lane < end ? ds[j + 32 + lane] : 0.f;
-            const int n = min(32, end - j);
-            for (int r = 0; r < n; ++r) se = __fadd_rn(se, __shfl_sync(0xFFFFFFFFu, v, r));
-            v = vn;
+        // eight loads of 32 distances in flight (the largest clusters, thousands
+        // of members, would otherwise wait on every load in turn)
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = beg + 32 * u + lane < end ? ds[beg + 32 * u + lane] : 0.f;
+        for (int j = beg; j < end; j += 256) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int jb = j + 32 * u;
+                if (jb < end) {
+                    const int n = min(32, end - jb);
+                    const float cur = v[u];
+                    v[u] = jb + 256 + lane < end ? ds[jb + 256 + lane] : 0.f;
+                    for (int r = 0; r < n; ++r) se = __fadd_rn(se, __shfl_sync(0xFFFFFFFFu, cur, r));
+                }
+            }
         }
         if (lane == 0) {
             sse[f] = se;

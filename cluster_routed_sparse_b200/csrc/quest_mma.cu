@@ -28,7 +28,9 @@
 //   warp 5     tensor-memory owner and single-thread MMA issuer
 // Phase 2 (selection), one warp per query cluster: the row's scores are staged
 // in shared memory, radix-selected (8-bit digits), rescored where needed, and
-// written out with the key ranges the attention kernel walks.
+// written out with the key ranges the attention kernel walks.  A CTA selects
+// for 16 query clusters, so a head's selection spreads over several SMs; each
+// of them recomputes the head's (small) score GEMM and writes its own rows.
 #include <algorithm>
 
 #include "ac_device.cuh"
@@ -37,7 +39,9 @@
 namespace ac {
 namespace {
 
-constexpr int QM = 128;          // query clusters per CTA (MMA M)
+constexpr int QM = 128;          // query clusters per MMA tile (M)
+constexpr int QR = 16;           // query clusters a CTA selects for (one per warp); the CTAs
+                                 // of one MMA tile each recompute its small GEMM
 constexpr int QN = 64;           // key clusters per chunk (MMA N)
 constexpr int Q_STAGES = 2;
 constexpr int Q_THREADS = 512;
@@ -150,7 +154,9 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
                                               ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x, m0 = blockIdx.y * QM;
+    // this CTA's query clusters r_lo .. r_hi - 1, inside the MMA tile of rows m0 ..
+    const int h = blockIdx.x, r_lo = blockIdx.y * QR, r_hi = min(p.Cq, r_lo + QR);
+    const int m0 = (r_lo / QM) * QM;
     const int rows = min(QM, p.Cq - m0);
     const int nk = p.n_k[h];
     const int nch = (nk + QN - 1) / QN;
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(QBAR(QB_AE + a));
-                if (r < rows) {
+                if (m0 + r >= r_lo && m0 + r < r_hi) {
                     const int c0 = ch * QN;
 #pragma unroll
                     for (int q = 0; q < 2; ++q)
@@ -387,7 +393,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
     const int *pg = p.pgoff + (int64_t)h * p.Ccap;
     const float eps = quest_eps(D);
 
-    for (int r = warp; r < rows; r += p.warps2) {
+    for (int r = r_lo - m0 + warp; r < r_hi - m0; r += p.warps2) {
         const int64_t hq = (int64_t)h * p.Cq + m0 + r;
         float *srow = p.score + hq * p.Ccap;
         for (int c = lane; c < nk; c += 32) Sw[c] = srow[c];
@@ -586,7 +592,7 @@ cudaError_t launch_quest_d(const SelectArgs &a, cudaStream_t s) {
     const int smem = (int)(bytes + 1024);
     cudaError_t e = cudaFuncSetAttribute(k_quest_select_mma<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    k_quest_select_mma<D><<<dim3(a.BH, (a.Cq + QM - 1) / QM), Q_THREADS, smem, s>>>(*a.tm_kmax, *a.tm_kmin, p);
+    k_quest_select_mma<D><<<dim3(a.BH, (a.Cq + QR - 1) / QR), Q_THREADS, smem, s>>>(*a.tm_kmax, *a.tm_kmin, p);
     AC_NOTE_LAUNCH();
     return cudaGetLastError();
 }
