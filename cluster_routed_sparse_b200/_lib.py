@@ -94,6 +94,7 @@ SIGNATURES = {
     "ac_layer_forward_host_async": (_I, [_P, _P, _P, _P, _P, _I, _P]),
     "ac_join": (_I, [_P, _P]),
     "ac_synchronize": (_I, [_P, _P]),
+    "ac_check_wait_timeout": (_I, [_P, ctypes.c_int32, _P]),
     "ac_get_tensor": (_I, [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int64)]),
     "ac_get_attn_counters": (_I, [_P, ctypes.POINTER(ACAttnCounters)]),
     "ac_get_launch_count": (_I, [ctypes.POINTER(ctypes.c_int64)]),

@@ -196,6 +196,11 @@ class SparseLayer:
     def synchronize(self):
         check(self.lib.ac_synchronize(self.ctx, _stream()), self.ctx)
 
+    def check_wait_timeout(self, limit_us: int):
+        """Enqueue the bounded-wait health check (ac_check_wait_timeout); the
+        next synchronize() raises with AC_ERR_TIMEOUT."""
+        check(self.lib.ac_check_wait_timeout(self.ctx, int(limit_us), _stream()), self.ctx)
+
     def tensor(self, which: int) -> torch.Tensor:
         """Device view of an intermediate tensor (ac_get_tensor); valid until the next call."""
         p = ctypes.c_void_p()

@@ -1074,6 +1074,28 @@ ac_status ac_tau_radix_pick(const uint64_t *hist, int32_t shift, uint32_t *state
     return AC_OK;
 }
 
+// One thread waits, with the same bounded loop as the pipelined kernels, on
+// the first phase of an mbarrier that expects one arrival which never comes;
+// when the limit runs out it records DEV_ERR_TIMEOUT and the CTA returns.
+__global__ void k_wait_check(uint32_t *err, uint64_t limit_ns) {
+    __shared__ alignas(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+        if (!mbar_wait_for(smem_u32(&bar), 0, limit_ns)) set_err(err, DEV_ERR_TIMEOUT);
+    }
+}
+
+ac_status ac_check_wait_timeout(ac_ctx *c, int32_t limit_us, void *stream) {
+    if (!c) return AC_ERR_INVALID_ARG;
+    if (limit_us < 1 || limit_us > 2000000)
+        return fail(c, AC_ERR_INVALID_ARG, "ac_check_wait_timeout: limit_us outside 1 .. 2,000,000");
+    k_wait_check<<<1, 32, 0, (cudaStream_t)stream>>>(c->err, (uint64_t)limit_us * 1000ull);
+    AC_NOTE_LAUNCH();
+    CK(cudaGetLastError(), "wait check launch");
+    return AC_OK;
+}
+
 ac_status ac_synchronize(ac_ctx *c, void *stream) {
     if (!c) return AC_ERR_INVALID_ARG;
     ac_status st = ac_join(c, stream);

@@ -106,6 +106,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     }
 }
 
+// As mbar_wait with a caller-chosen time limit (limit_ns, at most kWaitLimitNs);
+// the cycle bound is 4 cycles per nanosecond of the limit, the poll bound the
+// same as mbar_wait's.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    if (limit_ns > kWaitLimitNs) limit_ns = kWaitLimitNs;
+    const long long cycle_limit = (long long)limit_ns * 4;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    const long long c0 = clock64();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 255u &&
+            (globaltimer_ns() - t0 > limit_ns || clock64() - c0 > cycle_limit || it > kWaitLimitPolls))
+            return false;
+    }
+}
+
 // As mbar_wait, but also gives up as soon as another CTA has recorded an error
 // in *abort (so one stuck CTA does not make every CTA sit out its own limit).
 __device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t parity, const uint32_t *abort) {

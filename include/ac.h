@@ -232,6 +232,17 @@ AC_API ac_status ac_join(ac_ctx *ctx, void *stream);
  * recorded on the device (AC_ERR_TIMEOUT, AC_ERR_NONFINITE); clears it. */
 AC_API ac_status ac_synchronize(ac_ctx *ctx, void *stream);
 
+/* Health check of the failure-detection path.  Launches on `stream` one CTA
+ * whose thread waits, with the same bounded loop (globaltimer, clock64 and a
+ * poll count) that the pipelined kernels use on their mbarriers, for a phase
+ * that never completes, with a time limit of limit_us microseconds
+ * (1 .. 2,000,000).  When the limit runs out the kernel records the timeout in
+ * the context's device error word and returns, so the next ac_synchronize
+ * reports AC_ERR_TIMEOUT (and clears it) and the context stays usable.
+ * Errors: AC_ERR_INVALID_ARG for a NULL context or a limit out of range;
+ * AC_ERR_CUDA when the launch fails. */
+AC_API ac_status ac_check_wait_timeout(ac_ctx *ctx, int32_t limit_us, void *stream);
+
 /* Read-only views of intermediate device tensors (for tests and metrics).
  * *dev_ptr receives a device pointer owned by the context, shape[0..3] the
  * extents (unused trailing extents are 1).  Contents are valid after the

@@ -256,3 +256,33 @@ def test_nonfinite_input_is_reported():
         lay.cluster_q(dev(Q))
     assert e.value.status == AC_ERR_NONFINITE
     lay.close()
+
+
+def test_bounded_wait_timeout_is_reported_and_context_stays_usable():
+    """A bounded in-kernel wait on a phase nothing completes ends after its
+    limit with AC_ERR_TIMEOUT on the host; the context then runs the layer to
+    the same output as before the timeout."""
+    import time
+    from cluster_routed_sparse_b200._lib import ACError, AC_ERR_TIMEOUT, AC_ERR_INVALID_ARG
+    cfg = synth.CONFIGS[1]
+    p = _params(cfg)
+    Q, K, V = (dev(x) for x in synth.make_layer(cfg))
+    lay = make_layer_ctx(p, *Q.shape)
+    O0 = lay.forward(Q, K, V).clone()
+    lay.synchronize()
+    for bad in (0, -5, 2000001):
+        with pytest.raises(ACError) as e:
+            lay.check_wait_timeout(bad)
+        assert e.value.status == AC_ERR_INVALID_ARG
+    t0 = time.perf_counter()
+    lay.check_wait_timeout(20000)
+    with pytest.raises(ACError) as e:
+        lay.synchronize()
+    waited = time.perf_counter() - t0
+    assert e.value.status == AC_ERR_TIMEOUT
+    assert 0.019 <= waited < 1.5, waited
+    lay.synchronize()  # the error word was cleared
+    O1 = lay.forward(Q, K, V)
+    lay.synchronize()
+    assert torch.equal(O0, O1)
+    lay.close()
