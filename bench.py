@@ -282,18 +282,24 @@ def run_reference(args):
 # ---------------------------------------------------------------- main
 # DRAM bytes (read + write) of one k_sparse_attn launch per head of the bench
 # workload, from an ncu capture of its 8-head reduction, valid only for the
-# kernel source it was taken on: any change to attn_kernel.cu turns it into null.
-ATTN_TRAFFIC = {"sha256_prefix": "dbcf7fd631eae966", "bytes_per_head": (313612288 + 129535232) / 8}
+# kernel source it was taken on: any change to attn_kernel.cu or to the device
+# helpers it includes (ac_device.cuh) turns it into null.
+ATTN_TRAFFIC = {"sha256_prefix": "e7c279346a778c59", "bytes_per_head": (313656320 + 128224768) / 8}
+
+
+def attn_source_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("attn_kernel.cu", "ac_device.cuh"):
+        with open(os.path.join(ROOT, "cluster_routed_sparse_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def attn_traffic_bytes(cfg):
-    import hashlib
     if cfg.name != "wan14b-L75600-H40-d128":
         return None
-    src = os.path.join(ROOT, "cluster_routed_sparse_b200", "csrc", "attn_kernel.cu")
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()
-    if not digest.startswith(ATTN_TRAFFIC["sha256_prefix"]):
+    if not attn_source_digest().startswith(ATTN_TRAFFIC["sha256_prefix"]):
         return None
     return round(ATTN_TRAFFIC["bytes_per_head"] * cfg.H)
 

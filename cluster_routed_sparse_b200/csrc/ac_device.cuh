@@ -208,6 +208,67 @@ __device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem,
         : "memory");
 }
 
+// Eight tcgen05.mma (SS) into one accumulator in one asm block, for issuing
+// threads that share their sub-partition with busy warps.  Product 0 takes the
+// descriptors as given, product k = 1..7 adds Ak to the low word of A's and Bk
+// to the low word of B's (offsets in 16-byte units; the caller keeps every
+// operand inside shared memory, so the 14-bit address field does not carry).
+// Product 0 accumulates when acc != 0, the others always.
+template <uint32_t A1, uint32_t A2, uint32_t A3, uint32_t A4, uint32_t A5, uint32_t A6, uint32_t A7,
+          uint32_t B1, uint32_t B2, uint32_t B3, uint32_t B4, uint32_t B5, uint32_t B6, uint32_t B7>
+__device__ __forceinline__ void mma8_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t.reg .b32 alo, ahi, blo, bhi, x, y;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+        "mov.b64 {alo, ahi}, %1;\n\tmov.b64 {blo, bhi}, %2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "add.u32 x, alo, %5;\n\tadd.u32 y, blo, %12;\n\tmov.b64 da, {x, ahi};\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, t;\n\t"
+        "add.u32 x, alo, %6;\n\tadd.u32 y, blo, %13;\n\tmov.b64 da, {x, ahi};\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, t;\n\t"
+        "add.u32 x, alo, %7;\n\tadd.u32 y, blo, %14;\n\tmov.b64 da, {x, ahi};\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, t;\n\t"
+        "add.u32 x, alo, %8;\n\tadd.u32 y, blo, %15;\n\tmov.b64 da, {x, ahi};\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, t;\n\t"
+        "add.u32 x, alo, %9;\n\tadd.u32 y, blo, %16;\n\tmov.b64 da, {x, ahi};\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, t;\n\t"
+        "add.u32 x, alo, %10;\n\tadd.u32 y, blo, %17;\n\tmov.b64 da, {x, ahi};\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, t;\n\t"
+        "add.u32 x, alo, %11;\n\tadd.u32 y, blo, %18;\n\tmov.b64 da, {x, ahi};\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, t;\n\t}"
+        ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "n"(A1), "n"(A2), "n"(A3), "n"(A4), "n"(A5),
+        "n"(A6), "n"(A7), "n"(B1), "n"(B2), "n"(B3), "n"(B4), "n"(B5), "n"(B6), "n"(B7)
+        : "memory");
+}
+
+// Eight tcgen05.mma (TS: A from tensor memory at a + 8 k columns) into one
+// accumulator; B descriptor k is {b_lo + B_STEP * k, b_hi}.
+template <uint32_t B_STEP>
+__device__ __forceinline__ void mma8_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t.reg .b32 blo, bhi, y, ta;\n\t.reg .b64 db;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+        "mov.b64 {blo, bhi}, %2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "add.u32 y, blo, %5;\n\tadd.u32 ta, %1, 8;\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, t;\n\t"
+        "add.u32 y, blo, %6;\n\tadd.u32 ta, %1, 16;\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, t;\n\t"
+        "add.u32 y, blo, %7;\n\tadd.u32 ta, %1, 24;\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, t;\n\t"
+        "add.u32 y, blo, %8;\n\tadd.u32 ta, %1, 32;\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, t;\n\t"
+        "add.u32 y, blo, %9;\n\tadd.u32 ta, %1, 40;\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, t;\n\t"
+        "add.u32 y, blo, %10;\n\tadd.u32 ta, %1, 48;\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, t;\n\t"
+        "add.u32 y, blo, %11;\n\tadd.u32 ta, %1, 56;\n\tmov.b64 db, {y, bhi};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, t;\n\t}"
+        ::"r"(d), "r"(a), "l"(bdesc), "r"(idesc), "r"(acc), "n"(B_STEP), "n"(2 * B_STEP), "n"(3 * B_STEP),
+        "n"(4 * B_STEP), "n"(5 * B_STEP), "n"(6 * B_STEP), "n"(7 * B_STEP)
+        : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread completes.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)

@@ -347,25 +347,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) {
             constexpr uint32_t IQK = idesc_bf16_f32(BM, BN, false);
             constexpr uint32_t IPV = idesc_bf16_f32(BM, D, true);
+            // Descriptors are formed once; a product's descriptor is its base
+            // plus the operand's offset in 16-byte units (the address field
+            // cannot carry: every offset stays inside shared memory).
+            const uint64_t dq0 = sdesc_sw128(sbase + LY::OFF_Q, 16, 1024);
+            const uint64_t dk0 = sdesc_sw128(sbase + LY::OFF_K, 16, LY::BOX_BYTES);
+            const uint64_t dv0 = sdesc_sw128(sbase + LY::OFF_V, 1024, LY::BOX_BYTES);
             auto issue_s = [&](int i, int j) {
-                const uint32_t qa = sbase + LY::OFF_Q + i * LY::Q_TILE;
-                const uint32_t ka = sbase + LY::OFF_K + (j % NS) * LY::KV_BYTES;
+                const uint64_t dq = dq0 + (uint64_t)((i * LY::Q_TILE) >> 4);
+                const uint64_t dk = dk0 + (uint64_t)(((j % NS) * LY::KV_BYTES) >> 4);
+                // K16 step kk reads Q at (kk / 4) x BM x 128 B (its column half) plus
+                // (kk % 4) x 32 B and K at (kk / 4) x 1024 B plus (kk % 4) x 32 B; the
+                // template arguments are these offsets in 16-byte units
+                if constexpr (D == 128) {
+                    constexpr uint32_t QH = (BM * 128) >> 4;
+                    mma8_ss<2, 4, 6, QH, QH + 2, QH + 4, QH + 6, 2, 4, 6, 64, 66, 68, 70>(tmem + i * BN, dq, dk, IQK, 0u);
+                } else {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qoff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                    const uint32_t koff = (kk >> 2) * 1024 + (kk & 3) * 32;
-                    tc_mma_bf16(tmem + i * BN, sdesc_sw128(qa + qoff, 16, 1024),
-                                sdesc_sw128(ka + koff, 16, LY::BOX_BYTES), IQK, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        tc_mma_bf16(tmem + i * BN, dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), IQK, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(BAR(B_SF + i));
             };
             auto issue_pv = [&](int i, int j) {
-                const uint32_t va = sbase + LY::OFF_V + (j % NS) * LY::KV_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    tc_mma_bf16_ts(tmem + 256 + i * 128, tmem + i * BN + kk * 8,
-                                   sdesc_sw128(va + kk * 2 * LY::BOX_BYTES, 1024, LY::BOX_BYTES), IPV,
-                                   (j > 0 || kk > 0) ? 1u : 0u);
+                const uint64_t dv = dv0 + (uint64_t)(((j % NS) * LY::KV_BYTES) >> 4);
+                constexpr uint32_t VSTEP = (2 * LY::BOX_BYTES) / 16;
+                mma8_ts<VSTEP>(tmem + 256 + i * 128, tmem + i * BN, dv, IPV, j > 0 ? 1u : 0u);
             };
             if (!WAIT(3, B_QF, 0, 0)) ok = false;
             if (ok && n_tiles > 0) {
