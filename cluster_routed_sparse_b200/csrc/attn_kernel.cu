@@ -27,6 +27,9 @@
 // sums and representable in bf16.
 // MMA order per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): while one
 // softmax warpgroup works on its S, the tensor core runs the other's products.
+// The issuing thread shares its SM sub-partition with two softmax warps, so
+// it spends as few instructions per product as it can: descriptors are formed
+// once and each group of eight products is one asm block.
 // Every mbarrier wait is bounded; on timeout the CTA records an error, drains
 // what it issued and frees its TMEM.
 #include "ac_device.cuh"
