@@ -55,3 +55,26 @@ def test_single_rank_needs_no_process_group():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(12.5, 1, "cpu") == 12.5
+
+
+def test_attention_traffic_is_tied_to_the_captured_sources(tmp_path, monkeypatch):
+    """roofline.traffic is an ncu figure of one kernel version: it is reported
+    for the bench workload only while the hashed kernel sources are the ones
+    it was captured on, and turns null once either file changes."""
+    sys.path.insert(0, ROOT)
+    import shutil
+    import bench
+    from cluster_routed_sparse_b200 import synth
+    cfg = synth.CONFIGS[bench.CONFIG_ID]
+    assert cfg.name == "wan14b-L75600-H40-d128"
+    assert bench.attn_traffic_bytes(cfg) == round(bench.ATTN_TRAFFIC["bytes_per_head"] * cfg.H)
+    assert all(bench.attn_traffic_bytes(c) is None for c in synth.CONFIGS.values() if c.name != cfg.name)
+    csrc = tmp_path / "cluster_routed_sparse_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in ("attn_kernel.cu", "ac_device.cuh"):
+        shutil.copy(os.path.join(ROOT, "cluster_routed_sparse_b200", "csrc", name), csrc / name)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.attn_traffic_bytes(cfg) is not None
+    with open(csrc / "ac_device.cuh", "a") as f:
+        f.write("\n// edited\n")
+    assert bench.attn_traffic_bytes(cfg) is None
