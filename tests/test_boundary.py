@@ -87,6 +87,7 @@ def test_null_arguments_rejected():
     assert lib.ac_synchronize(None, None) == _lib.AC_ERR_INVALID_ARG
     assert lib.ac_join(None, None) == _lib.AC_ERR_INVALID_ARG
     assert lib.ac_layer_forward_host_async(None, None, None, None, None, 0, None) == _lib.AC_ERR_INVALID_ARG
+    assert lib.ac_check_wait_timeout(None, 1000, None) == _lib.AC_ERR_INVALID_ARG
     assert lib.ac_last_error_string(None) == b""
 
 
